@@ -1,0 +1,165 @@
+/*
+ * pivot.h -- C ABI of the PIVOT group-shared sparse-attention indexer for
+ * NVIDIA B200 (sm_100a).
+ *
+ * What is computed (PIVOT, picx.dev summary of the paper, sections
+ * "Introduction and Theoretical Foundation" and "Methodology"):
+ *
+ *   Eq. (1)  I_{t,s} = sum_{j<H} w_{t,j} * ReLU(q_{t,j} . k_s),  T_t = TopK(I_{t,:}, k)
+ *   Eq. (2)  prefill groups: positions [i*g, min(i*g+g, L))
+ *   Eq. (3)  decode group: the current token and its g-1 MTP draft tokens
+ *   Eq. (4)  proxy: q-bar_j = mean_t q_{t,j},  w-bar_j = mean_t w_{t,j}   (t in the group)
+ *   Eq. (5)  proxy score  I-bar_s = sum_j w-bar_j ReLU(q-bar_j . k_s),  s <= last group position
+ *   Eq. (6)  PIVOT-Reuse:  T_t = TopK({I-bar_s : s <= t}, k) for every member t
+ *   Eq. (7)  PIVOT-Refine candidates  C = TopK({I-bar_s : s <= last group position}, c)
+ *   Eq. (8)  member re-scoring  I_{t,s} for s in C
+ *   Eq. (9)  T_t = TopK({I_{t,s} : s in C, s <= t}, k)
+ *
+ * Conventions fixed by this library where the pages are silent:
+ *   - the proxy scans the prefix up to the group's LAST position; each member
+ *     t then masks s <= t (so Refine with c >= L equals the dense indexer);
+ *   - the pooled q-bar is rounded to nearest-even to the input dtype (it is
+ *     the operand of the scan); w-bar stays fp32;
+ *   - TopK order: larger score first, equal scores -> lower key index; -0.0
+ *     and +0.0 are equal;
+ *   - an output row holds its valid indices first, in unspecified order, and
+ *     -1 in the remaining slots.  Dense and Reuse rows hold min(k, t+1)
+ *     indices; Refine rows hold min(k, |C cap [0,t]|) (= min(k, t+1) when
+ *     c >= k+g-1).  Indices are positions local to the sequence.
+ *   - decode: sequence b holds P_b cached keys (positions 0..P_b-1, the
+ *     group's own rows included); its g query rows are positions
+ *     P_b-g .. P_b-1 (current token first, then the drafts).
+ *
+ * Memory: every tensor pointer is a DEVICE pointer owned by the caller,
+ * row-major and contiguous: q_I [rows, H, d], w_I [rows, H] (fp32),
+ * k_I [key rows, d], indices [rows, k] (int32), scores [rows, k] (fp32).
+ * q_I and k_I are bf16 (bit patterns) or fp32 (pivot_dtype); q_I, k_I and
+ * the workspace must be 16-byte aligned, and d must be a multiple of 8.
+ * The library allocates nothing: scratch comes from the caller's workspace
+ * (size from the *_workspace_size call for the current device).
+ *
+ * Execution: every call is asynchronous on `stream`; none synchronises the
+ * host, except pivot_last_device_status.  Calls that share a workspace must
+ * be ordered on the device (same stream or events).
+ *
+ * Errors are returned, never thrown; no device assert or trap is used.
+ * Invalid arguments are rejected on the host before any launch.  Inputs
+ * must be finite (a precondition, not checked).  Device-side waits are
+ * bounded; a wait that runs out records PIVOT_ERR_DEVICE_TIMEOUT in the
+ * workspace, which pivot_last_device_status reports.
+ */
+#ifndef PIVOT_H_
+#define PIVOT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define PIVOT_API __attribute__((visibility("default")))
+#else
+#define PIVOT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *pivot_stream_t; /* same type as cudaStream_t; NULL = legacy default stream */
+
+typedef enum { PIVOT_BF16 = 0, PIVOT_F32 = 1 } pivot_dtype; /* dtype of q_I and k_I (w_I is fp32) */
+
+typedef enum {
+  PIVOT_OK = 0,
+  PIVOT_ERR_INVALID_ARG = 1,       /* null pointer, non-positive size, k > c, misalignment ... */
+  PIVOT_ERR_UNSUPPORTED_SHAPE = 2, /* g > 16, L >= 2^31, ... */
+  PIVOT_ERR_WORKSPACE_TOO_SMALL = 3,
+  PIVOT_ERR_CUDA = 4,              /* a CUDA runtime/driver call failed (see pivot_last_cuda_error) */
+  PIVOT_ERR_DEVICE_TIMEOUT = 5,    /* a bounded device wait ran out (reported by pivot_last_device_status) */
+  PIVOT_ERR_DEVICE_BOUNDS = 6
+} pivot_status;
+
+typedef enum { PIVOT_OP_DENSE = 0, PIVOT_OP_REUSE = 1, PIVOT_OP_REFINE = 2 } pivot_op;
+
+/* Workspace bytes needed by pivot_indexer_dense / pivot_reuse / pivot_refine
+ * (op = PIVOT_OP_*) for these sizes on the CURRENT device.  c is ignored
+ * unless op == PIVOT_OP_REFINE, g unless op != PIVOT_OP_DENSE.  Returns 0 for
+ * arguments the call would reject. */
+PIVOT_API size_t pivot_workspace_size(int op, int64_t L, int H, int d, int k, int c, int g, pivot_dtype dt);
+
+/* Eq. (1): the dense DSA indexer, T_t for t = 0..L-1.
+ * q_I [L,H,d], w_I [L,H], k_I [L,d] -> indices [L,k]; scores_opt [L,k] (or
+ * NULL) receives I_{t,s} of each returned index (-inf in padded slots). */
+PIVOT_API pivot_status pivot_indexer_dense(const void *q_I, const float *w_I, const void *k_I, int64_t L, int H, int d,
+                                 pivot_dtype dt, int k, int32_t *indices, float *scores_opt, void *ws,
+                                 size_t ws_bytes, pivot_stream_t stream);
+
+/* Eq. (2), (4)-(6): PIVOT-Reuse with prefill groups of g (1 <= g <= 16).
+ * scores_opt receives the proxy scores I-bar_s of the returned indices. */
+PIVOT_API pivot_status pivot_reuse(const void *q_I, const float *w_I, const void *k_I, int64_t L, int H, int d,
+                         pivot_dtype dt, int k, int g, int32_t *indices, float *scores_opt, void *ws,
+                         size_t ws_bytes, pivot_stream_t stream);
+
+/* Eq. (2), (4), (5), (7)-(9): PIVOT-Refine with prefill groups of g and c
+ * candidates (k <= c; the pages use c = 2k).  scores_opt receives the member
+ * scores I_{t,s}.  cand_opt [ceil(L/g), c] (or NULL) receives each group's
+ * candidate set C_i (valid entries first, unordered, -1 padded) and
+ * cand_scores_opt the proxy scores of those candidates. */
+PIVOT_API pivot_status pivot_refine(const void *q_I, const float *w_I, const void *k_I, int64_t L, int H, int d,
+                          pivot_dtype dt, int k, int c, int g, int32_t *indices, float *scores_opt,
+                          int32_t *cand_opt, float *cand_scores_opt, void *ws, size_t ws_bytes,
+                          pivot_stream_t stream);
+
+/* Workspace bytes for the decode calls below.  key_offsets_host [B+1] is the
+ * host copy of the key offsets (key_offsets_host[0] = 0, non-decreasing,
+ * every P_b = key_offsets_host[b+1] - key_offsets_host[b] >= g). */
+PIVOT_API size_t pivot_varlen_workspace_size(int op, int B, const int64_t *key_offsets_host, int H, int d, int k, int c,
+                                   int g, pivot_dtype dt);
+
+/* Eq. (3)-(6): PIVOT-Reuse for a batch of B MTP decode groups.
+ * q [B*g,H,d] (rows b*g..b*g+g-1 = sequence b's current token then drafts),
+ * w [B*g,H], k_cache [sum P_b, d] (sequence b's keys are rows
+ * key_offsets[b] .. key_offsets[b+1]-1), key_offsets_dev / key_offsets_host
+ * [B+1] (same values, device and host copies) -> indices [B*g,k] of
+ * positions local to each sequence. */
+PIVOT_API pivot_status pivot_reuse_varlen(const void *q, const float *w, const void *k_cache, const int64_t *key_offsets_dev,
+                                const int64_t *key_offsets_host, int B, int H, int d, pivot_dtype dt, int k, int g,
+                                int32_t *indices, float *scores_opt, void *ws, size_t ws_bytes,
+                                pivot_stream_t stream);
+
+/* Eq. (3)-(5), (7)-(9): PIVOT-Refine for a batch of B MTP decode groups;
+ * arguments as pivot_reuse_varlen plus c, cand_opt [B,c], cand_scores_opt. */
+PIVOT_API pivot_status pivot_refine_varlen(const void *q, const float *w, const void *k_cache,
+                                 const int64_t *key_offsets_dev, const int64_t *key_offsets_host, int B, int H,
+                                 int d, pivot_dtype dt, int k, int c, int g, int32_t *indices, float *scores_opt,
+                                 int32_t *cand_opt, float *cand_scores_opt, void *ws, size_t ws_bytes,
+                                 pivot_stream_t stream);
+
+/* Synchronises `stream`, then reads the device status word that the last
+ * call using workspace `ws` left: PIVOT_OK, PIVOT_ERR_DEVICE_TIMEOUT or
+ * PIVOT_ERR_DEVICE_BOUNDS (or PIVOT_ERR_CUDA if the sync/copy failed). */
+PIVOT_API pivot_status pivot_last_device_status(const void *ws, pivot_stream_t stream);
+
+/* Human-readable name of a status code (static string). */
+PIVOT_API const char *pivot_status_string(pivot_status s);
+
+/* Text of the last CUDA error seen by this library in the calling thread ("" if none). */
+PIVOT_API const char *pivot_last_cuda_error(void);
+
+/* Which kernel path a call with these arguments takes on the current device:
+ * 1 = tcgen05 tensor-core path (bf16, H = 64, d in {64,128}), 0 = CUDA-core
+ * path, -1 = the call would be rejected. */
+PIVOT_API int pivot_path(int op, int64_t L, int H, int d, int k, int c, int g, pivot_dtype dt);
+
+/* Bound (nanoseconds of wall-clock time) on every device-side wait; default
+ * 2e9.  Test hook: flags bit 0 makes the scan kernel wait on a barrier that
+ * nothing signals, so that the bound runs out and the timeout path is
+ * exercised without hanging the GPU. */
+PIVOT_API void pivot_set_device_timeout_ns(uint64_t ns);
+PIVOT_API void pivot_set_debug_flags(int flags);
+
+PIVOT_API int pivot_version(void); /* 100 * major + minor */
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PIVOT_H_ */

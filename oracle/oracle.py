@@ -50,6 +50,7 @@ def lib():
         L.orc_scores.argtypes = [P, P, I32, I32, P, I32, P, I64, I64, P]
         L.orc_proxy_scores.argtypes = [P, P, P, I32, I64, I32, I32, I32, I64, P]
         L.orc_proxy_scores.restype = I64
+        L.orc_scores_batch.argtypes = [P, P, I64, I32, I32, P, I32, P, P, P, I64, P]
         L.orc_topn.argtypes = [P, P, I64, I64, P, P]
         L.orc_topn.restype = I64
         L.orc_threads.restype = I32
@@ -197,3 +198,41 @@ def topn(f, n, idx=None):
     val = np.empty_like(out, dtype=np.float64)
     cnt = lib().orc_topn(_p(f), _p(ii), f.size, n, _p(out), _p(val))
     return out[:cnt], val[:cnt]
+
+
+def scores_batch(qv, wv, k, key_rows=None, plen=None, key_base=None, m=None):
+    """Scores of n vectors against key lists (key_rows [n,m], -1 = none) or
+    prefixes (plen [n]); returns [n, m] float64 with NaN where undefined."""
+    k = _c(k)
+    qv, wv = _c(qv, np.float64), _c(wv, np.float64)
+    n, H = wv.shape
+    d = k.shape[1]
+    kr = None if key_rows is None else _c(key_rows, np.int64)
+    pl = None if plen is None else _c(plen, np.int64)
+    kb = None if key_base is None else _c(key_base, np.int64)
+    if m is None:
+        m = kr.shape[1] if kr is not None else int(pl.max())
+    out = np.empty((n, m), np.float64)
+    lib().orc_scores_batch(_p(qv), _p(wv), n, H, d, _p(k), _dt(k), _p(kb), _p(kr), _p(pl), m, _p(out))
+    return out
+
+
+def query_rows(q, w, rows):
+    """Widened query rows: ([n, H*d], [n, H]) doubles."""
+    rows = list(rows)
+    _, H, d = q.shape
+    qv = np.empty((len(rows), H * d), np.float64)
+    wv = np.empty((len(rows), H), np.float64)
+    for i, r in enumerate(rows):
+        qv[i], wv[i] = query_row(q, w, int(r))
+    return qv, wv
+
+
+def proxies(q, w, member_lists):
+    """Eq. (4) proxies of several groups: ([n, H*d], [n, H]) doubles."""
+    _, H, d = q.shape
+    qv = np.empty((len(member_lists), H * d), np.float64)
+    wv = np.empty((len(member_lists), H), np.float64)
+    for i, rows in enumerate(member_lists):
+        qv[i], wv[i] = proxy(q, w, rows)
+    return qv, wv

@@ -120,15 +120,18 @@ void orc_proxy(const void *q, const float *w, int dtype, int H, int d,
 }
 
 /* Eq. (1) / (5) / (8): score of one (query or proxy) against key k_s.
- * k is [*, d]; key row s. */
+ * k is [*, d]; key row s.  The key row is widened to double first. */
 static double orc_score_one(const double *qv, const double *wv, int H, int d,
                             const void *k, int dtype, int64_t s)
 {
+    double kr[1024];
+    for (int x = 0; x < d; x++)
+        kr[x] = orc_elem(k, dtype, s * (int64_t)d + x);
     double total = 0.0;
     for (int j = 0; j < H; j++) {
         double dot = 0.0;
         for (int x = 0; x < d; x++)
-            dot += qv[j * d + x] * orc_elem(k, dtype, s * (int64_t)d + x);
+            dot += qv[j * d + x] * kr[x];
         double relu = dot > 0.0 ? dot : 0.0;
         total += wv[j] * relu;
     }
@@ -144,6 +147,29 @@ void orc_scores(const double *qv, const double *wv, int H, int d,
     for (int64_t i = 0; i < n; i++) {
         int64_t s = keys ? keys[i] : key_lo + i;
         out[i] = orc_score_one(qv, wv, H, d, k, dtype, s);
+    }
+}
+
+/* Scores of n vectors (qv [n, H*d], wv [n, H]) against key rows, in parallel
+ * over the vectors; out is [n, m].  Vector r reads keys from row
+ * key_base[r] (0 when key_base == NULL) onward.  With key_rows ([n, m]) entry
+ * i is the score against key key_rows[r*m+i] (NaN where that is < 0);
+ * otherwise entry s < plen[r] is the score against key s (NaN beyond). */
+void orc_scores_batch(const double *qv, const double *wv, int64_t n, int H, int d,
+                      const void *k, int dtype, const int64_t *key_base,
+                      const int64_t *key_rows, const int64_t *plen, int64_t m,
+                      double *out)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < n; r++) {
+        int64_t base = key_base ? key_base[r] : 0;
+        const double *q = qv + r * (int64_t)H * d;
+        const double *w = wv + r * (int64_t)H;
+        for (int64_t i = 0; i < m; i++) {
+            int64_t s = key_rows ? key_rows[r * m + i] : i;
+            int ok = key_rows ? (s >= 0) : (i < plen[r]);
+            out[r * m + i] = ok ? orc_score_one(q, w, H, d, k, dtype, base + s) : NAN;
+        }
     }
 }
 

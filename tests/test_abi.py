@@ -1,0 +1,77 @@
+"""CPU-side checks of the C ABI: the library builds, loads and exports every
+symbol include/pivot.h declares; host-side validation and sizing need no GPU."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import top_token_selection_proxy_b200 as P
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from top_token_selection_proxy_b200 import build
+
+    build.build()
+    return P.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "pivot.h")).read()
+    return sorted(set(re.findall(r"PIVOT_API\s+[\w\s\*]+?\b(pivot_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(P.EXPORTS) == names
+
+
+def test_version_and_status_strings(lib):
+    assert lib.pivot_version() == 100
+    for code, name in P.STATUS.items():
+        assert lib.pivot_status_string(code).decode() == name
+
+
+def test_workspace_sizes_positive_and_monotone(lib):
+    a = P.workspace_size(P.OP_REFINE, 8192, 64, 128, 2048, 4096, 8)
+    b = P.workspace_size(P.OP_REFINE, 131072, 64, 128, 2048, 4096, 8)
+    assert 0 < a < b
+    assert P.workspace_size(P.OP_DENSE, 512, 4, 32, 16, 16, 1, P.F32) > 0
+    assert P.workspace_size(P.OP_REUSE, 100, 64, 128, 8, 8, 17) == 0  # g > 16 rejected
+    assert P.workspace_size(P.OP_REFINE, 100, 64, 128, 8, 4, 4) == 0  # c < k rejected
+
+
+def test_path_selection(lib):
+    assert P.path(P.OP_REFINE, 131072, 64, 128, 2048, 4096, 8, P.BF16) == 1
+    assert P.path(P.OP_DENSE, 131072, 64, 64, 2048, 2048, 1, P.BF16) == 1
+    assert P.path(P.OP_REFINE, 512, 4, 32, 16, 32, 4, P.F32) == 0
+    assert P.path(P.OP_REUSE, 512, 32, 128, 16, 16, 4, P.BF16) == 0
+    assert P.path(P.OP_REUSE, 0, 64, 128, 16, 16, 4, P.BF16) == -1
+
+
+def test_invalid_arguments_rejected_before_launch(lib):
+    # null pointers, zero sizes, k > c, bad g: rejected on the host (no device needed)
+    nul = None
+    buf = ctypes.create_string_buffer(1024)
+    ptr = ctypes.cast(buf, ctypes.c_void_p)
+    assert lib.pivot_indexer_dense(nul, nul, nul, 16, 4, 32, 0, 4, nul, nul, nul, 0, nul) == 1
+    assert lib.pivot_reuse(ptr, ptr, ptr, 0, 4, 32, 0, 4, 2, ptr, nul, ptr, 1024, nul) == 1
+    assert lib.pivot_refine(ptr, ptr, ptr, 64, 4, 32, 0, 8, 4, 2, ptr, nul, nul, nul, ptr, 1024, nul) == 1
+    assert lib.pivot_reuse(ptr, ptr, ptr, 64, 4, 32, 0, 4, 32, ptr, nul, ptr, 1024, nul) == 2
+    assert lib.pivot_indexer_dense(ptr, ptr, ptr, 64, 4, 30, 0, 4, ptr, nul, ptr, 1024, nul) == 1  # d % 8
+    off = np.array([0, 3, 10], np.int64)  # P_0 = 3 < g = 4
+    assert lib.pivot_varlen_workspace_size(1, 2, off.ctypes.data_as(ctypes.c_void_p), 64, 128, 8, 8, 4, 0) == 0
+
+
+def test_workspace_too_small_rejected(lib):
+    buf = ctypes.create_string_buffer(4096)
+    ptr = ctypes.c_void_p((ctypes.addressof(buf) + 15) // 16 * 16)
+    st = lib.pivot_reuse(ptr, ptr, ptr, 1024, 64, 128, 0, 16, 4, ptr, None, ptr, 256, None)
+    assert st == 3

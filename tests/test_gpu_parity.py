@@ -1,0 +1,350 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle.
+
+Small cases are checked on every row/group; the long workloads on a seeded
+sample of groups (always including the first and last group and the groups
+whose prefix straddles c and k+g-1), at the sizes and launch configuration
+the bench uses.  Refine is checked in two levels: the GPU candidate set C_i
+against the oracle's proxy scores, then the member rows against the oracle
+re-scoring over the GPU's own C_i.
+"""
+import numpy as np
+import pytest
+import torch
+
+import top_token_selection_proxy_b200 as P
+from parity import check_row, summarize
+from top_token_selection_proxy_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from top_token_selection_proxy_b200 import build
+
+    build.build()
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    P.set_device_timeout_ns(2_000_000_000)
+    P.set_debug_flags(0)
+
+
+def dev(x):
+    if x.dtype == np.uint16:
+        return torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def host(t):
+    return None if t is None else t.cpu().numpy()
+
+
+def members(L, g, i):
+    return list(range(i * g, min(i * g + g, L)))
+
+
+# ---------------------------------------------------------------- checkers
+
+
+def check_dense(orc, x, idx, sc, rows, topk, key_base=None, pos=None):
+    q, w, k = x["q"], x["w"], x["k"]
+    rows = list(rows)
+    pos = rows if pos is None else list(pos)
+    qv, wv = orc.query_rows(q, w, rows)
+    F = orc.scores_batch(qv, wv, k, plen=np.array(pos) + 1, key_base=key_base)
+    fails = []
+    for i, (r, t) in enumerate(zip(rows, pos)):
+        fails += check_row(idx[r], None if sc is None else sc[r], np.arange(t + 1), F[i, :t + 1],
+                           min(topk, t + 1), orc, f"dense row {r}")
+    return fails
+
+
+def check_reuse(orc, x, idx, sc, groups, topk, g):
+    q, w, k = x["q"], x["w"], x["k"]
+    L = q.shape[0]
+    mem = [members(L, g, i) for i in groups]
+    qv, wv = orc.proxies(q, w, mem)
+    F = orc.scores_batch(qv, wv, k, plen=np.array([m[-1] + 1 for m in mem]))
+    fails = []
+    for gi, m in enumerate(mem):
+        for t in m:
+            fails += check_row(idx[t], None if sc is None else sc[t], np.arange(t + 1), F[gi, :t + 1],
+                               min(topk, t + 1), orc, f"reuse g={g} t={t}")
+    return fails
+
+
+def check_refine(orc, x, idx, sc, cand, csc, groups, topk, c, g):
+    q, w, k = x["q"], x["w"], x["k"]
+    L = q.shape[0]
+    mem = [members(L, g, i) for i in groups]
+    qv, wv = orc.proxies(q, w, mem)
+    F = orc.scores_batch(qv, wv, k, plen=np.array([m[-1] + 1 for m in mem]))
+    fails = []
+    for gi, (i, m) in enumerate(zip(groups, mem)):
+        e = m[-1]
+        fails += check_row(cand[i], None if csc is None else csc[i], np.arange(e + 1), F[gi, :e + 1],
+                           min(c, e + 1), orc, f"C_{i}")
+    rows = [t for m in mem for t in m]
+    grp_of = [i for i, m in zip(groups, mem) for _ in m]
+    qv, wv = orc.query_rows(q, w, rows)
+    C = np.stack([cand[i] for i in grp_of]).astype(np.int64)
+    M = orc.scores_batch(qv, wv, k, key_rows=C)
+    for r, (t, i) in enumerate(zip(rows, grp_of)):
+        ok = (C[r] >= 0) & (C[r] <= t)
+        E, f = C[r][ok], M[r][ok]
+        fails += check_row(idx[t], None if sc is None else sc[t], E, f, min(topk, E.size), orc,
+                           f"refine g={g} t={t}")
+    return fails
+
+
+def run_all(x, topk, c, g, scores=True):
+    q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
+    d_idx, d_sc = P.indexer_dense(q, w, k, topk, scores=scores)
+    u_idx, u_sc = P.reuse(q, w, k, topk, g, scores=scores)
+    r_idx, r_sc, r_c, r_cs = P.refine(q, w, k, topk, c, g, scores=scores, cand=True)
+    torch.cuda.synchronize()
+    return {n: host(v) for n, v in dict(d_idx=d_idx, d_sc=d_sc, u_idx=u_idx, u_sc=u_sc, r_idx=r_idx,
+                                        r_sc=r_sc, r_c=r_c, r_cs=r_cs).items()}
+
+
+def full_check(orc, x, res, topk, c, g, groups=None, dense_rows=None):
+    L = x["q"].shape[0]
+    G = (L + g - 1) // g
+    groups = list(range(G)) if groups is None else list(groups)
+    dense_rows = list(range(L)) if dense_rows is None else list(dense_rows)
+    fails = check_dense(orc, x, res["d_idx"], res["d_sc"], dense_rows, topk)
+    fails += check_reuse(orc, x, res["u_idx"], res["u_sc"], groups, topk, g)
+    fails += check_refine(orc, x, res["r_idx"], res["r_sc"], res["r_c"], res["r_cs"], groups, topk, c, g)
+    return fails
+
+
+# ---------------------------------------------------------------- small workloads, every row
+
+
+def test_tiny_config_every_group(orc):
+    s = inputs.TINY
+    x = inputs.make_prefill(s)
+    assert P.path(P.OP_REFINE, s.L, s.H, s.d, s.k, s.c, s.g, P.F32) == 0
+    res = run_all(x, s.k, s.c, s.g)
+    fails = full_check(orc, x, res, s.k, s.c, s.g)
+    assert not fails, summarize(fails)
+
+
+@pytest.mark.parametrize("g", [4, 8, 16])
+def test_tensor_core_path_every_group(orc, g):
+    # ragged: L is not a multiple of 128 keys, of g, nor of 4 groups per work item;
+    # k and c small enough that the streaming selection cuts back several times
+    L, H, d, topk, c = 1337, 64, 128, 64, 128
+    x = inputs.random_prefill(L, H, d, inputs.BF16, seed=100 + g, rho=0.95, heavy=0.01)
+    assert P.path(P.OP_REFINE, L, H, d, topk, c, g, P.BF16) == 1
+    res = run_all(x, topk, c, g)
+    fails = full_check(orc, x, res, topk, c, g)
+    assert not fails, summarize(fails)
+
+
+def test_tensor_core_d64(orc):
+    L, H, d, topk, c, g = 700, 64, 64, 32, 64, 8
+    x = inputs.random_prefill(L, H, d, inputs.BF16, seed=7, rho=0.9, heavy=0.02)
+    assert P.path(P.OP_REFINE, L, H, d, topk, c, g, P.BF16) == 1
+    res = run_all(x, topk, c, g)
+    fails = full_check(orc, x, res, topk, c, g)
+    assert not fails, summarize(fails)
+
+
+def test_cuda_core_path_bf16_odd_heads(orc):
+    L, H, d, topk, c, g = 300, 8, 40, 10, 20, 3
+    x = inputs.random_prefill(L, H, d, inputs.BF16, seed=9)
+    assert P.path(P.OP_REFINE, L, H, d, topk, c, g, P.BF16) == 0
+    res = run_all(x, topk, c, g)
+    fails = full_check(orc, x, res, topk, c, g)
+    assert not fails, summarize(fails)
+
+
+# ---------------------------------------------------------------- edge cases
+
+
+@pytest.mark.parametrize("L", [1, 2, 127, 128, 129])
+def test_short_sequences(orc, L):
+    x = inputs.random_prefill(L, 64, 128, inputs.BF16, seed=L)
+    topk, c, g = 8, 16, 4
+    res = run_all(x, topk, c, g)
+    fails = full_check(orc, x, res, topk, c, g)
+    assert not fails, summarize(fails)
+
+
+def test_k_larger_than_prefix_and_c_ge_L(orc):
+    # c >= L: C_i is the whole prefix, so Refine rows equal dense rows (Eq. 7-9 reduce to Eq. 1)
+    L, topk, c, g = 300, 256, 512, 8
+    x = inputs.random_prefill(L, 64, 128, inputs.BF16, seed=11)
+    res = run_all(x, topk, c, g)
+    fails = full_check(orc, x, res, topk, c, g)
+    assert not fails, summarize(fails)
+    for t in range(L):
+        a = set(res["r_idx"][t][res["r_idx"][t] >= 0].tolist())
+        b = set(res["d_idx"][t][res["d_idx"][t] >= 0].tolist())
+        assert a == b, t
+
+
+def test_ties_zero_queries_lowest_index(orc):
+    """All-zero queries: every score is +-0 -> each row is exactly 0..min(k,t+1)-1."""
+    L, H, d, topk, c, g = 400, 64, 128, 32, 64, 8
+    x = inputs.random_prefill(L, H, d, inputs.BF16, seed=12)
+    x["q"][:] = 0
+    x["w"][:] = -1.0
+    res = run_all(x, topk, c, g)
+    for name in ("d_idx", "u_idx", "r_idx"):
+        for t in range(L):
+            n = min(topk, t + 1)
+            assert sorted(res[name][t][:n].tolist()) == list(range(n)), (name, t)
+            assert (res[name][t][n:] == -1).all()
+
+
+def test_duplicate_keys_lower_index(orc):
+    L, H, d, topk, c, g = 512, 64, 128, 16, 32, 4
+    x = inputs.random_prefill(L, H, d, inputs.BF16, seed=13)
+    x["k"][100:200] = x["k"][50]  # many exact ties in every score
+    res = run_all(x, topk, c, g)
+    fails = full_check(orc, x, res, topk, c, g)
+    assert not fails, summarize(fails)
+
+
+def test_reuse_g1_equals_dense_on_gpu():
+    L, topk = 1000, 32
+    x = inputs.random_prefill(L, 64, 128, inputs.BF16, seed=14)
+    q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
+    a, _ = P.indexer_dense(q, w, k, topk)
+    b, _ = P.reuse(q, w, k, topk, 1)
+    assert torch.equal(a.sort(dim=1).values, b.sort(dim=1).values)
+
+
+# ---------------------------------------------------------------- the workloads at full size
+
+
+def test_prefill_8k_sampled(orc):
+    s = inputs.PREFILL_8K
+    x = inputs.make_prefill(s)
+    res = run_all(x, s.k, s.c, s.g)
+    G = (s.L + s.g - 1) // s.g
+    groups = inputs.sample_groups(G, s.g, s.k, s.c, 96, s.seed + 1000)
+    rows = sorted({int(t) for i in groups for t in members(s.L, s.g, int(i))})[::4]
+    fails = full_check(orc, x, res, s.k, s.c, s.g, groups=groups, dense_rows=rows)
+    assert not fails, summarize(fails)
+
+
+@pytest.mark.parametrize("rho", inputs.SWEEP_RHO)
+@pytest.mark.parametrize("g", inputs.SWEEP_G)
+def test_sweep_32k_sampled(orc, g, rho):
+    s = inputs.sweep_32k(g, rho)
+    x = inputs.make_prefill(s)
+    q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
+    u_idx, _ = P.reuse(q, w, k, s.k, g)
+    r_idx, r_sc, r_c, r_cs = P.refine(q, w, k, s.k, s.c, g, scores=True, cand=True)
+    torch.cuda.synchronize()
+    G = (s.L + g - 1) // g
+    groups = inputs.sample_groups(G, g, s.k, s.c, 24, s.seed + 1000 + g)
+    fails = check_reuse(orc, x, host(u_idx), None, groups, s.k, g)
+    fails += check_refine(orc, x, host(r_idx), host(r_sc), host(r_c), host(r_cs), groups, s.k, s.c, g)
+    assert not fails, summarize(fails)
+
+
+@pytest.fixture(scope="module")
+def long_inputs():
+    return inputs.make_prefill(inputs.LONG_128K)
+
+
+def test_long_128k_refine_reuse_dense_sampled(orc, long_inputs):
+    s = inputs.LONG_128K
+    x = long_inputs
+    q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
+    r_idx, r_sc, r_c, r_cs = P.refine(q, w, k, s.k, s.c, s.g, scores=True, cand=True)
+    u_idx, u_sc = P.reuse(q, w, k, s.k, s.g, scores=True)
+    d_idx, d_sc = P.indexer_dense(q, w, k, s.k, scores=True)
+    torch.cuda.synchronize()
+    G = (s.L + s.g - 1) // s.g
+    groups = inputs.sample_groups(G, s.g, s.k, s.c, 256, s.seed + 1000)
+    fails = check_refine(orc, x, host(r_idx), host(r_sc), host(r_c), host(r_cs), groups, s.k, s.c, s.g)
+    fails += check_reuse(orc, x, host(u_idx), host(u_sc), groups[::4], s.k, s.g)
+    rows = [int(i) * s.g + (int(i) % s.g) for i in groups[::2]]
+    fails += check_dense(orc, x, host(d_idx), host(d_sc), rows, s.k)
+    assert not fails, summarize(fails)
+
+
+def test_decode_batch_every_sequence(orc):
+    s = inputs.DECODE
+    x = inputs.make_decode(s)
+    off = x["offsets"]
+    q, w, kc = dev(x["q"]), dev(x["w"]), dev(x["k"])
+    u_idx, u_sc = P.reuse_varlen(q, w, kc, off, s.k, s.g, scores=True)
+    r_idx, r_sc, r_c, r_cs = P.refine_varlen(q, w, kc, off, s.k, s.c, s.g, scores=True, cand=True)
+    torch.cuda.synchronize()
+    u_idx, u_sc, r_idx, r_sc, r_c, r_cs = map(host, (u_idx, u_sc, r_idx, r_sc, r_c, r_cs))
+    B, g = s.B, s.g
+    mem = [list(range(b * g, b * g + g)) for b in range(B)]
+    qv, wv = orc.proxies(x["q"], x["w"], mem)
+    Pb = np.diff(off)
+    F = orc.scores_batch(qv, wv, x["k"], plen=Pb, key_base=off[:-1])
+    fails = []
+    for b in range(B):
+        fails += check_row(r_c[b], r_cs[b], np.arange(Pb[b]), F[b, :Pb[b]], min(s.c, Pb[b]), orc, f"C_{b}")
+        for r in range(g):
+            t = Pb[b] - g + r
+            fails += check_row(u_idx[b * g + r], u_sc[b * g + r], np.arange(t + 1), F[b, :t + 1],
+                               min(s.k, t + 1), orc, f"decode reuse b={b} r={r}")
+    rows = list(range(B * g))
+    qv, wv = orc.query_rows(x["q"], x["w"], rows)
+    C = np.repeat(r_c.astype(np.int64), g, axis=0)
+    M = orc.scores_batch(qv, wv, x["k"], key_rows=C, key_base=np.repeat(off[:-1], g))
+    for row in rows:
+        b, r = divmod(row, g)
+        t = Pb[b] - g + r
+        ok = (C[row] >= 0) & (C[row] <= t)
+        fails += check_row(r_idx[row], r_sc[row], C[row][ok], M[row][ok], min(s.k, int(ok.sum())), orc,
+                           f"decode refine b={b} r={r}")
+    assert not fails, summarize(fails)
+
+
+def test_decode_small_ragged(orc):
+    spec = inputs.DecodeSpec("small", B=5, p_lo=4, p_hi=3000, H=64, d=128, k=64, c=128, g=4, seed=21)
+    x = inputs.make_decode(spec)
+    off = x["offsets"]
+    q, w, kc = dev(x["q"]), dev(x["w"]), dev(x["k"])
+    u_idx, _ = P.reuse_varlen(q, w, kc, off, spec.k, spec.g)
+    r_idx, _, r_c, _ = P.refine_varlen(q, w, kc, off, spec.k, spec.c, spec.g, cand=True)
+    o_u, _, _, _ = orc.decode(x["q"], x["w"], x["k"], off, spec.k, spec.c, spec.g, 0)
+    o_r, _, _, _ = orc.decode(x["q"], x["w"], x["k"], off, spec.k, spec.c, spec.g, 1, cand_in=host(r_c))
+    for got, want in ((host(u_idx), o_u), (host(r_idx), o_r)):
+        for row in range(got.shape[0]):
+            a = set(got[row][got[row] >= 0].tolist())
+            b = set(want[row][want[row] >= 0].tolist())
+            assert len(a ^ b) <= 2, (row, len(a ^ b))
+
+
+# ---------------------------------------------------------------- failure paths (no GPU fault)
+
+
+def test_forced_device_timeout_is_reported_and_context_survives(orc):
+    L, topk, g = 600, 16, 4
+    x = inputs.random_prefill(L, 64, 128, inputs.BF16, seed=15)
+    q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
+    ws = P.Workspace()
+    try:
+        P.set_device_timeout_ns(50_000_000)
+        P.set_debug_flags(1)
+        P.reuse(q, w, k, topk, g, ws=ws)
+        assert P.last_device_status(ws) == 5  # PIVOT_ERR_DEVICE_TIMEOUT
+    finally:
+        P.set_debug_flags(0)
+        P.set_device_timeout_ns(2_000_000_000)
+    idx, sc = P.reuse(q, w, k, topk, g, ws=ws, scores=True)
+    assert P.last_device_status(ws) == 0
+    fails = check_reuse(orc, x, host(idx), host(sc), range((L + g - 1) // g), topk, g)
+    assert not fails, summarize(fails)
+
+
+def test_invalid_calls_raise():
+    x = inputs.random_prefill(64, 64, 128, inputs.BF16, seed=16)
+    q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
+    with pytest.raises(P.PivotError):
+        P.refine(q, w, k, 32, 16, 4)  # c < k
+    with pytest.raises(P.PivotError):
+        P.reuse(q, w, k, 8, 17)  # g > 16

@@ -1,0 +1,267 @@
+"""PIVOT group-shared sparse-attention indexer for NVIDIA B200 (sm_100a).
+
+Thin ctypes binding of ``libpivot.so`` (the C ABI in ``include/pivot.h``).
+It only marshals arguments: every step of the indexer runs in the library's
+CUDA kernels.  PyTorch provides device memory and streams.  There is no CPU
+fallback: if the library is missing or a CUDA device is absent, calls raise.
+
+PIVOT (picx.dev summary of the paper, Methodology, Eq. 1-9): the dense DSA
+indexer scores I_{t,s} = sum_j w_{t,j} ReLU(q_{t,j} . k_s) and keeps the top k
+keys per query; PIVOT pools each group of g queries into a mean proxy, scans
+the prefix once per group, and either reuses the proxy top-k (Reuse) or
+re-scores the proxy top-c per member (Refine).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpivot.so")
+
+OP_DENSE, OP_REUSE, OP_REFINE = 0, 1, 2
+BF16, F32 = 0, 1
+
+STATUS = {
+    0: "PIVOT_OK",
+    1: "PIVOT_ERR_INVALID_ARG",
+    2: "PIVOT_ERR_UNSUPPORTED_SHAPE",
+    3: "PIVOT_ERR_WORKSPACE_TOO_SMALL",
+    4: "PIVOT_ERR_CUDA",
+    5: "PIVOT_ERR_DEVICE_TIMEOUT",
+    6: "PIVOT_ERR_DEVICE_BOUNDS",
+}
+
+# every symbol include/pivot.h declares
+EXPORTS = (
+    "pivot_workspace_size", "pivot_indexer_dense", "pivot_reuse", "pivot_refine",
+    "pivot_varlen_workspace_size", "pivot_reuse_varlen", "pivot_refine_varlen",
+    "pivot_last_device_status", "pivot_status_string", "pivot_last_cuda_error", "pivot_path",
+    "pivot_set_device_timeout_ns", "pivot_set_debug_flags", "pivot_version",
+)
+
+
+class PivotError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}" + (f" ({detail})" if detail else ""))
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libpivot.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m top_token_selection_proxy_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, I64, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+        L.pivot_workspace_size.argtypes = [I, I64, I, I, I, I, I, I]
+        L.pivot_workspace_size.restype = SZ
+        L.pivot_varlen_workspace_size.argtypes = [I, I, P, I, I, I, I, I, I]
+        L.pivot_varlen_workspace_size.restype = SZ
+        L.pivot_indexer_dense.argtypes = [P, P, P, I64, I, I, I, I, P, P, P, SZ, P]
+        L.pivot_reuse.argtypes = [P, P, P, I64, I, I, I, I, I, P, P, P, SZ, P]
+        L.pivot_refine.argtypes = [P, P, P, I64, I, I, I, I, I, I, P, P, P, P, P, SZ, P]
+        L.pivot_reuse_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P]
+        L.pivot_refine_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P, SZ, P]
+        for f in ("pivot_indexer_dense", "pivot_reuse", "pivot_refine", "pivot_reuse_varlen",
+                  "pivot_refine_varlen", "pivot_last_device_status"):
+            getattr(L, f).restype = I
+        L.pivot_last_device_status.argtypes = [P, P]
+        L.pivot_status_string.argtypes = [I]
+        L.pivot_status_string.restype = ctypes.c_char_p
+        L.pivot_last_cuda_error.restype = ctypes.c_char_p
+        L.pivot_path.argtypes = [I, I64, I, I, I, I, I, I]
+        L.pivot_path.restype = I
+        L.pivot_set_device_timeout_ns.argtypes = [ctypes.c_uint64]
+        L.pivot_set_debug_flags.argtypes = [I]
+        L.pivot_version.restype = I
+        _lib = L
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"q/k must be bfloat16 or float32, got {t.dtype}")
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise PivotError(st, where, lib().pivot_last_cuda_error().decode())
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+class Workspace:
+    """Caller-owned scratch for the library (a torch uint8 buffer that grows on demand)."""
+
+    def __init__(self, device=None):
+        self.device = device
+        self.buf: Optional[torch.Tensor] = None
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.device or "cuda")
+        return self.buf
+
+
+_default_ws: dict = {}
+
+
+def _ws_for(ws: Optional[Workspace], dev) -> Workspace:
+    if ws is not None:
+        return ws
+    key = str(dev)
+    if key not in _default_ws:
+        _default_ws[key] = Workspace(dev)
+    return _default_ws[key]
+
+
+def workspace_size(op: int, L: int, H: int, d: int, k: int, c: int, g: int, dtype: int = BF16) -> int:
+    return int(lib().pivot_workspace_size(op, L, H, d, k, c, g, dtype))
+
+
+def varlen_workspace_size(op: int, offsets_host, H: int, d: int, k: int, c: int, g: int, dtype: int = BF16) -> int:
+    off = torch.as_tensor(offsets_host, dtype=torch.int64).contiguous()
+    return int(lib().pivot_varlen_workspace_size(op, off.numel() - 1, ctypes.c_void_p(off.data_ptr()), H, d, k, c,
+                                                 g, dtype))
+
+
+def path(op: int, L: int, H: int, d: int, k: int, c: int, g: int, dtype: int = BF16) -> int:
+    """1 = tcgen05 tensor-core path, 0 = CUDA-core path, -1 = rejected."""
+    return int(lib().pivot_path(op, L, H, d, k, c, g, dtype))
+
+
+def _prefill_common(q, w, k):
+    _need_cuda(q, w, k)
+    if q.dim() != 3 or w.dim() != 2 or k.dim() != 2:
+        raise ValueError("expected q [L,H,d], w [L,H], k [L,d]")
+    L, H, d = q.shape
+    if w.shape != (L, H) or k.shape != (L, d) or w.dtype != torch.float32 or k.dtype != q.dtype:
+        raise ValueError("shape/dtype mismatch between q, w and k")
+    return L, H, d, _dt(q)
+
+
+def indexer_dense(q, w, k, topk: int, *, scores: bool = False, out=None, ws: Optional[Workspace] = None,
+                  stream=None):
+    """Eq. (1): dense indexer.  Returns (indices [L,topk] int32, scores [L,topk] f32 or None)."""
+    L, H, d, dt = _prefill_common(q, w, k)
+    idx = out if out is not None else torch.empty((L, topk), dtype=torch.int32, device=q.device)
+    sc = torch.empty((L, topk), dtype=torch.float32, device=q.device) if scores else None
+    nbytes = workspace_size(OP_DENSE, L, H, d, topk, topk, 1, dt)
+    W = _ws_for(ws, q.device).get(nbytes)
+    _check(lib().pivot_indexer_dense(_ptr(q), _ptr(w), _ptr(k), L, H, d, dt, topk, _ptr(idx), _ptr(sc), _ptr(W),
+                                     W.numel(), _stream(stream)), "pivot_indexer_dense")
+    return idx, sc
+
+
+def reuse(q, w, k, topk: int, g: int, *, scores: bool = False, out=None, ws: Optional[Workspace] = None,
+          stream=None):
+    """Eq. (4)-(6): PIVOT-Reuse.  Returns (indices, proxy scores or None)."""
+    L, H, d, dt = _prefill_common(q, w, k)
+    idx = out if out is not None else torch.empty((L, topk), dtype=torch.int32, device=q.device)
+    sc = torch.empty((L, topk), dtype=torch.float32, device=q.device) if scores else None
+    nbytes = workspace_size(OP_REUSE, L, H, d, topk, topk, g, dt)
+    W = _ws_for(ws, q.device).get(nbytes)
+    _check(lib().pivot_reuse(_ptr(q), _ptr(w), _ptr(k), L, H, d, dt, topk, g, _ptr(idx), _ptr(sc), _ptr(W),
+                             W.numel(), _stream(stream)), "pivot_reuse")
+    return idx, sc
+
+
+def refine(q, w, k, topk: int, c: int, g: int, *, scores: bool = False, cand: bool = False, out=None,
+           ws: Optional[Workspace] = None, stream=None):
+    """Eq. (4),(5),(7)-(9): PIVOT-Refine.  Returns (indices, member scores|None, C|None, C scores|None)."""
+    L, H, d, dt = _prefill_common(q, w, k)
+    G = (L + g - 1) // g
+    idx = out if out is not None else torch.empty((L, topk), dtype=torch.int32, device=q.device)
+    sc = torch.empty((L, topk), dtype=torch.float32, device=q.device) if scores else None
+    cd = torch.empty((G, c), dtype=torch.int32, device=q.device) if cand else None
+    cs = torch.empty((G, c), dtype=torch.float32, device=q.device) if (cand and scores) else None
+    nbytes = workspace_size(OP_REFINE, L, H, d, topk, c, g, dt)
+    W = _ws_for(ws, q.device).get(nbytes)
+    _check(lib().pivot_refine(_ptr(q), _ptr(w), _ptr(k), L, H, d, dt, topk, c, g, _ptr(idx), _ptr(sc), _ptr(cd),
+                              _ptr(cs), _ptr(W), W.numel(), _stream(stream)), "pivot_refine")
+    return idx, sc, cd, cs
+
+
+def _varlen_common(q, w, kc, offsets, g):
+    _need_cuda(q, w, kc)
+    off_h = torch.as_tensor(offsets, dtype=torch.int64).cpu().contiguous()
+    B = off_h.numel() - 1
+    if q.dim() != 3 or q.shape[0] != B * g or w.shape != (B * g, q.shape[1]) or kc.shape[1] != q.shape[2]:
+        raise ValueError("expected q [B*g,H,d], w [B*g,H], k_cache [sum P, d]")
+    off_d = off_h.to(q.device)
+    return B, q.shape[1], q.shape[2], _dt(q), off_h, off_d
+
+
+def reuse_varlen(q, w, k_cache, offsets, topk: int, g: int, *, scores: bool = False,
+                 ws: Optional[Workspace] = None, stream=None):
+    """Eq. (3)-(6) for a batch of MTP decode groups.  Returns (indices [B*g,topk], scores|None)."""
+    B, H, d, dt, off_h, off_d = _varlen_common(q, w, k_cache, offsets, g)
+    idx = torch.empty((B * g, topk), dtype=torch.int32, device=q.device)
+    sc = torch.empty((B * g, topk), dtype=torch.float32, device=q.device) if scores else None
+    nbytes = varlen_workspace_size(OP_REUSE, off_h, H, d, topk, topk, g, dt)
+    W = _ws_for(ws, q.device).get(nbytes)
+    _check(lib().pivot_reuse_varlen(_ptr(q), _ptr(w), _ptr(k_cache), _ptr(off_d), _ptr(off_h), B, H, d, dt, topk,
+                                    g, _ptr(idx), _ptr(sc), _ptr(W), W.numel(), _stream(stream)),
+           "pivot_reuse_varlen")
+    return idx, sc
+
+
+def refine_varlen(q, w, k_cache, offsets, topk: int, c: int, g: int, *, scores: bool = False, cand: bool = False,
+                  ws: Optional[Workspace] = None, stream=None):
+    """Eq. (3)-(5),(7)-(9) for a batch of MTP decode groups."""
+    B, H, d, dt, off_h, off_d = _varlen_common(q, w, k_cache, offsets, g)
+    idx = torch.empty((B * g, topk), dtype=torch.int32, device=q.device)
+    sc = torch.empty((B * g, topk), dtype=torch.float32, device=q.device) if scores else None
+    cd = torch.empty((B, c), dtype=torch.int32, device=q.device) if cand else None
+    cs = torch.empty((B, c), dtype=torch.float32, device=q.device) if (cand and scores) else None
+    nbytes = varlen_workspace_size(OP_REFINE, off_h, H, d, topk, c, g, dt)
+    W = _ws_for(ws, q.device).get(nbytes)
+    _check(lib().pivot_refine_varlen(_ptr(q), _ptr(w), _ptr(k_cache), _ptr(off_d), _ptr(off_h), B, H, d, dt, topk,
+                                     c, g, _ptr(idx), _ptr(sc), _ptr(cd), _ptr(cs), _ptr(W), W.numel(),
+                                     _stream(stream)), "pivot_refine_varlen")
+    return idx, sc, cd, cs
+
+
+def last_device_status(ws: Workspace, stream=None) -> int:
+    """Synchronise the stream and return the device status code of the last call on ``ws``."""
+    return int(lib().pivot_last_device_status(_ptr(ws.buf), _stream(stream)))
+
+
+def set_device_timeout_ns(ns: int) -> None:
+    lib().pivot_set_device_timeout_ns(int(ns))
+
+
+def set_debug_flags(flags: int) -> None:
+    lib().pivot_set_debug_flags(int(flags))
+
+
+__all__ = [
+    "lib", "LIB_PATH", "EXPORTS", "PivotError", "Workspace", "workspace_size", "varlen_workspace_size", "path",
+    "indexer_dense", "reuse", "refine", "reuse_varlen", "refine_varlen", "last_device_status",
+    "set_device_timeout_ns", "set_debug_flags", "OP_DENSE", "OP_REUSE", "OP_REFINE", "BF16", "F32", "STATUS",
+]

@@ -1,0 +1,568 @@
+// api.cu -- host side of the C ABI declared in include/pivot.h: argument
+// validation, workspace carving, TMA descriptors and the launch sequence of
+// each entry point.  Allocates nothing; every launch goes on the caller's
+// stream and no call synchronises the host (pivot_last_device_status aside).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "kernels.cuh"
+
+using namespace pivot;
+
+namespace {
+
+thread_local char g_cuda_err[256] = "";
+uint64_t g_timeout_ns = 2000000000ull;
+int g_debug_flags = 0;
+
+constexpr size_t kHdr = 256;     // status word + counters
+constexpr int kStatusOff = 0;    // int
+constexpr int kCounterOff = 64;  // 4 x uint32
+
+pivot_status cuda_fail(cudaError_t e, const char* what) {
+  snprintf(g_cuda_err, sizeof(g_cuda_err), "%s: %s", what, cudaGetErrorString(e));
+  return PIVOT_ERR_CUDA;
+}
+
+int num_sms() {
+  static std::mutex mu;
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  std::lock_guard<std::mutex> lk(mu);
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- TMA descriptor
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [rows, d] (d contiguous), 64-column x box_rows boxes, 128-byte swizzle.
+bool make_kmap(CUtensorMap* m, const void* base, int64_t rows, int d, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- shapes and paths
+bool tc_shape(int H, int d, pivot_dtype dt) { return dt == PIVOT_BF16 && H == 64 && (d == 64 || d == 128); }
+
+pivot_status check_common(int64_t L, int H, int d, pivot_dtype dt, int k, int c, int g, int op) {
+  if (L <= 0 || H <= 0 || d <= 0 || k <= 0 || g <= 0) return PIVOT_ERR_INVALID_ARG;
+  if (dt != PIVOT_BF16 && dt != PIVOT_F32) return PIVOT_ERR_INVALID_ARG;
+  if (d % 8 != 0) return PIVOT_ERR_INVALID_ARG;
+  if (op == PIVOT_OP_REFINE && (c < k || c <= 0)) return PIVOT_ERR_INVALID_ARG;
+  if (g > 16 || L >= (int64_t)0x7FFFFFF0 || k > 65536 || (op == PIVOT_OP_REFINE && c > 16384) || H > 1024 ||
+      d > 1024)
+    return PIVOT_ERR_UNSUPPORTED_SHAPE;
+  return PIVOT_OK;
+}
+
+int sel_size(int op, int k, int c, int g) {
+  return op == PIVOT_OP_DENSE ? k : (op == PIVOT_OP_REUSE ? k + g - 1 : c);
+}
+int sel_cap(int n_sel) { return (int)align_up((size_t)2 * n_sel + 256, 256); }
+
+struct Carve {
+  char* base;
+  size_t off = 0;
+  template <typename T>
+  T* take(size_t count) {
+    off = align_up(off, 256);
+    T* p = reinterpret_cast<T*>(base ? base + off : nullptr);
+    off += count * sizeof(T);
+    return p;
+  }
+};
+
+// Workspace of the prefill calls; with base == nullptr only sizes are computed.
+struct PrefillWs {
+  int* status;
+  unsigned* counters;
+  uint64_t* selbuf;
+  int32_t* cand;
+  uint32_t* keys;
+  uint64_t* sscratch;
+  float* fscratch;
+  int grid, simt_grid;
+  int64_t simt_per_block;
+  size_t bytes;
+};
+
+PrefillWs carve_prefill(void* base, int op, int64_t L, int H, int d, int k, int c, int g, pivot_dtype dt,
+                        bool user_cand) {
+  PrefillWs w{};
+  Carve cv{reinterpret_cast<char*>(base)};
+  char* hdr = cv.take<char>(kHdr);
+  w.status = reinterpret_cast<int*>(hdr ? hdr + kStatusOff : nullptr);
+  w.counters = reinterpret_cast<unsigned*>(hdr ? hdr + kCounterOff : nullptr);
+  const int sms = num_sms();
+  const int64_t gs = (op == PIVOT_OP_DENSE) ? 1 : g;
+  const int64_t n_groups = (L + gs - 1) / gs;
+  if (tc_shape(H, d, dt)) {
+    const int nb = 256 / H;
+    const int64_t n_items = (n_groups + nb - 1) / nb;
+    w.grid = (int)std::min<int64_t>(sms, n_items);
+    const int n_sel = sel_size(op, k, c, g);
+    w.selbuf = cv.take<uint64_t>((size_t)sms * nb * sel_cap(n_sel));
+    if (op == PIVOT_OP_REFINE) {
+      if (!user_cand) w.cand = cv.take<int32_t>((size_t)n_groups * c);
+      w.keys = cv.take<uint32_t>((size_t)L * c);
+    }
+  } else {
+    w.simt_grid = (int)std::min<int64_t>(2 * sms, n_groups);
+    w.simt_per_block = L + (op == PIVOT_OP_REFINE ? c : 0);
+    w.sscratch = cv.take<uint64_t>((size_t)(2 * sms) * w.simt_per_block);
+    w.fscratch = cv.take<float>((size_t)(2 * sms) * ((size_t)H * d + H));
+  }
+  w.bytes = align_up(cv.off, 256);
+  return w;
+}
+
+struct DecodeWs {
+  int* status;
+  unsigned* counters;
+  int32_t* item_seq;
+  int64_t *item_s0, *item_s1;
+  int32_t* seq_item0;
+  uint64_t* selbuf;
+  uint64_t* partial;
+  uint32_t* partial_cnt;
+  uint64_t* mscratch;
+  int32_t* cand;
+  uint32_t* keys;
+  uint64_t* sscratch;
+  float* fscratch;
+  int grid, mgrid, simt_grid, n_items;
+  int64_t chunk, simt_per_block;
+  size_t bytes;
+};
+
+DecodeWs carve_decode(void* base, int op, int B, const int64_t* off, int H, int d, int k, int c, int g,
+                      pivot_dtype dt, bool user_cand) {
+  DecodeWs w{};
+  Carve cv{reinterpret_cast<char*>(base)};
+  char* hdr = cv.take<char>(kHdr);
+  w.status = reinterpret_cast<int*>(hdr ? hdr + kStatusOff : nullptr);
+  w.counters = reinterpret_cast<unsigned*>(hdr ? hdr + kCounterOff : nullptr);
+  const int sms = num_sms();
+  int64_t total = 0, pmax = 0;
+  for (int b = 0; b < B; ++b) {
+    const int64_t P = off[b + 1] - off[b];
+    total += P;
+    pmax = std::max(pmax, P);
+  }
+  if (tc_shape(H, d, dt)) {
+    const int n_sel = sel_size(op, k, c, g);
+    // chunks of at least 2*n_sel keys, ~4 chunks per SM over the batch
+    const int64_t target = (total + 4 * (int64_t)sms - 1) / (4 * (int64_t)sms);
+    w.chunk = (int64_t)align_up((size_t)std::max<int64_t>(2 * (int64_t)n_sel, target), 128);
+    int64_t items = 0;
+    for (int b = 0; b < B; ++b) {
+      const int64_t P = off[b + 1] - off[b];
+      items += std::max<int64_t>(1, (P + w.chunk - 1) / w.chunk);
+    }
+    w.n_items = (int)items;
+    w.grid = (int)std::min<int64_t>(sms, items);
+    w.mgrid = std::min(B, sms);
+    w.item_seq = cv.take<int32_t>(items);
+    w.item_s0 = cv.take<int64_t>(items);
+    w.item_s1 = cv.take<int64_t>(items);
+    w.seq_item0 = cv.take<int32_t>((size_t)B + 1);
+    w.selbuf = cv.take<uint64_t>((size_t)sms * (256 / H) * sel_cap(n_sel));
+    w.partial = cv.take<uint64_t>((size_t)items * n_sel);
+    w.partial_cnt = cv.take<uint32_t>(items);
+    w.mscratch = cv.take<uint64_t>((size_t)w.mgrid * n_sel);
+    if (op == PIVOT_OP_REFINE) {
+      if (!user_cand) w.cand = cv.take<int32_t>((size_t)B * c);
+      w.keys = cv.take<uint32_t>((size_t)B * g * c);
+    }
+  } else {
+    w.simt_grid = std::min(B, 2 * sms);
+    w.simt_per_block = pmax + (op == PIVOT_OP_REFINE ? c : 0);
+    w.sscratch = cv.take<uint64_t>((size_t)(2 * sms) * w.simt_per_block);
+    w.fscratch = cv.take<float>((size_t)(2 * sms) * ((size_t)H * d + H));
+  }
+  w.bytes = align_up(cv.off, 256);
+  return w;
+}
+
+pivot_status check_offsets(int B, const int64_t* off, int g) {
+  if (B <= 0 || !off || off[0] != 0) return PIVOT_ERR_INVALID_ARG;
+  for (int b = 0; b < B; ++b)
+    if (off[b + 1] - off[b] < g) return PIVOT_ERR_INVALID_ARG;
+  if (off[B] >= (int64_t)0x7FFFFFF0) return PIVOT_ERR_UNSUPPORTED_SHAPE;
+  return PIVOT_OK;
+}
+
+ScanArgs scan_base(const void* q, const float* w, int H, int d, int g, int n_sel, int k, int mode, int64_t n_groups,
+                   int n_items, uint64_t* selbuf, int cap, unsigned* counter, int* status) {
+  ScanArgs a{};
+  a.q = reinterpret_cast<const uint16_t*>(q);
+  a.w = w;
+  a.H = H;
+  a.D = d;
+  a.g = g;
+  a.n_sel = n_sel;
+  a.topk = k;
+  a.nb = 256 / H;
+  a.mode = mode;
+  a.n_groups = n_groups;
+  a.n_items = n_items;
+  a.selbuf = selbuf;
+  a.cap = cap;
+  a.counter = counter;
+  a.status = status;
+  a.timeout_ns = g_timeout_ns;
+  a.debug_flags = g_debug_flags;
+  return a;
+}
+
+// ---------------------------------------------------------------- prefill driver
+pivot_status run_prefill(int op, const void* q, const float* w, const void* k_I, int64_t L, int H, int d,
+                         pivot_dtype dt, int k, int c, int g, int32_t* indices, float* scores, int32_t* cand_opt,
+                         float* cand_scores, void* ws, size_t ws_bytes, cudaStream_t s) {
+  g_cuda_err[0] = 0;
+  if (op == PIVOT_OP_DENSE) g = 1;
+  pivot_status st = check_common(L, H, d, dt, k, c, g, op);
+  if (st != PIVOT_OK) return st;
+  if (!q || !w || !k_I || !indices || !ws) return PIVOT_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_I) || !aligned16(ws)) return PIVOT_ERR_INVALID_ARG;
+  const PrefillWs need = carve_prefill(nullptr, op, L, H, d, k, c, g, dt, cand_opt != nullptr);
+  if (ws_bytes < need.bytes) return PIVOT_ERR_WORKSPACE_TOO_SMALL;
+  const PrefillWs W = carve_prefill(ws, op, L, H, d, k, c, g, dt, cand_opt != nullptr);
+  cudaError_t e = cudaMemsetAsync(ws, 0, kHdr, s);
+  if (e != cudaSuccess) return cuda_fail(e, "memset");
+  const int64_t n_groups = (L + g - 1) / g;
+
+  if (!tc_shape(H, d, dt)) {
+    SimtArgs a{};
+    a.q = q;
+    a.w = w;
+    a.k = k_I;
+    a.is_bf16 = dt == PIVOT_BF16;
+    a.L = L;
+    a.H = H;
+    a.D = d;
+    a.g = g;
+    a.c = c;
+    a.topk = k;
+    a.variant = op;
+    a.n_groups = n_groups;
+    a.out_idx = indices;
+    a.out_scores = scores;
+    a.cand_out = cand_opt;
+    a.cand_scores = cand_scores;
+    a.scratch = W.sscratch;
+    a.scratch_per_block = W.simt_per_block;
+    a.fscratch = W.fscratch;
+    e = launch_simt(a, W.simt_grid, s);
+    return e == cudaSuccess ? PIVOT_OK : cuda_fail(e, "simt kernel");
+  }
+
+  CUtensorMap kmap;
+  if (!make_kmap(&kmap, k_I, L, d, 128)) return cuda_fail(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+  const int nb = 256 / H;
+  const int n_sel = sel_size(op, k, c, g);
+  const int n_items = (int)((n_groups + nb - 1) / nb);
+  const int mode = op == PIVOT_OP_DENSE ? EMIT_DENSE : (op == PIVOT_OP_REUSE ? EMIT_REUSE : EMIT_CAND);
+  ScanArgs a = scan_base(q, w, H, d, g, n_sel, k, mode, n_groups, n_items, W.selbuf, sel_cap(n_sel),
+                         W.counters + 0, W.status);
+  a.L = L;
+  a.out_idx = indices;
+  a.out_scores = scores;
+  int32_t* cand = cand_opt ? cand_opt : W.cand;
+  a.cand = cand;
+  a.cand_scores = cand_scores;
+  e = launch_scan(a, &kmap, W.grid, s);
+  if (e != cudaSuccess) return cuda_fail(e, "scan kernel");
+  if (op != PIVOT_OP_REFINE) return PIVOT_OK;
+
+  RefineArgs r{};
+  r.q = reinterpret_cast<const uint16_t*>(q);
+  r.w = w;
+  r.k = reinterpret_cast<const uint16_t*>(k_I);
+  r.L = L;
+  r.H = H;
+  r.D = d;
+  r.g = g;
+  r.c = c;
+  r.topk = k;
+  r.mc = 512 / H;
+  r.n_groups = n_groups;
+  r.n_items = (int)(n_groups * ((g + r.mc - 1) / r.mc));
+  r.cand = cand;
+  r.key_off = nullptr;
+  r.keys = W.keys;
+  r.counter = W.counters + 1;
+  r.status = W.status;
+  r.timeout_ns = g_timeout_ns;
+  e = launch_refine(r, nullptr, (int)std::min<int64_t>(num_sms(), r.n_items), s);
+  if (e != cudaSuccess) return cuda_fail(e, "refine kernel");
+
+  RowSelArgs rs{};
+  rs.keys = W.keys;
+  rs.cand = cand;
+  rs.n_rows = L;
+  rs.L = L;
+  rs.key_off = nullptr;
+  rs.g = g;
+  rs.c = c;
+  rs.topk = k;
+  rs.out_idx = indices;
+  rs.out_scores = scores;
+  e = launch_rowselect(rs, (int)std::min<int64_t>(8 * num_sms(), L), s);
+  return e == cudaSuccess ? PIVOT_OK : cuda_fail(e, "rowselect kernel");
+}
+
+// ---------------------------------------------------------------- decode driver
+pivot_status run_decode(int op, const void* q, const float* w, const void* kc, const int64_t* off_dev,
+                        const int64_t* off_host, int B, int H, int d, pivot_dtype dt, int k, int c, int g,
+                        int32_t* indices, float* scores, int32_t* cand_opt, float* cand_scores, void* ws,
+                        size_t ws_bytes, cudaStream_t s) {
+  g_cuda_err[0] = 0;
+  pivot_status st = check_common(1, H, d, dt, k, c, g, op);
+  if (st != PIVOT_OK) return st;
+  if ((st = check_offsets(B, off_host, g)) != PIVOT_OK) return st;
+  if (!q || !w || !kc || !off_dev || !indices || !ws) return PIVOT_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kc) || !aligned16(ws)) return PIVOT_ERR_INVALID_ARG;
+  const DecodeWs need = carve_decode(nullptr, op, B, off_host, H, d, k, c, g, dt, cand_opt != nullptr);
+  if (ws_bytes < need.bytes) return PIVOT_ERR_WORKSPACE_TOO_SMALL;
+  const DecodeWs W = carve_decode(ws, op, B, off_host, H, d, k, c, g, dt, cand_opt != nullptr);
+  cudaError_t e = cudaMemsetAsync(ws, 0, kHdr, s);
+  if (e != cudaSuccess) return cuda_fail(e, "memset");
+
+  if (!tc_shape(H, d, dt)) {
+    SimtArgs a{};
+    a.q = q;
+    a.w = w;
+    a.k = kc;
+    a.is_bf16 = dt == PIVOT_BF16;
+    a.L = 0;
+    a.H = H;
+    a.D = d;
+    a.g = g;
+    a.c = c;
+    a.topk = k;
+    a.variant = op;
+    a.n_groups = B;
+    a.key_off = off_dev;
+    a.out_idx = indices;
+    a.out_scores = scores;
+    a.cand_out = cand_opt;
+    a.cand_scores = cand_scores;
+    a.scratch = W.sscratch;
+    a.scratch_per_block = W.simt_per_block;
+    a.fscratch = W.fscratch;
+    e = launch_simt(a, W.simt_grid, s);
+    return e == cudaSuccess ? PIVOT_OK : cuda_fail(e, "simt kernel");
+  }
+
+  e = launch_plan_items(off_dev, B, W.chunk, W.item_seq, W.item_s0, W.item_s1, W.seq_item0, s);
+  if (e != cudaSuccess) return cuda_fail(e, "plan kernel");
+  CUtensorMap kmap;
+  if (!make_kmap(&kmap, kc, off_host[B], d, 128)) return cuda_fail(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+  const int n_sel = sel_size(op, k, c, g);
+  ScanArgs a = scan_base(q, w, H, d, g, n_sel, k, EMIT_PARTIAL, B, W.n_items, W.selbuf, sel_cap(n_sel),
+                         W.counters + 0, W.status);
+  a.L = 0;
+  a.key_off = off_dev;
+  a.item_seq = W.item_seq;
+  a.item_s0 = W.item_s0;
+  a.item_s1 = W.item_s1;
+  a.partial = W.partial;
+  a.partial_cnt = W.partial_cnt;
+  e = launch_scan(a, &kmap, W.grid, s);
+  if (e != cudaSuccess) return cuda_fail(e, "scan kernel");
+
+  int32_t* cand = cand_opt ? cand_opt : W.cand;
+  MergeArgs m{};
+  m.partial = W.partial;
+  m.partial_cnt = W.partial_cnt;
+  m.seq_item0 = W.seq_item0;
+  m.n_sel = n_sel;
+  m.B = B;
+  m.g = g;
+  m.topk = k;
+  m.mode = op == PIVOT_OP_REUSE ? EMIT_REUSE : EMIT_CAND;
+  m.key_off = off_dev;
+  m.scratch = W.mscratch;
+  m.cap = n_sel;
+  m.cand = cand;
+  m.cand_scores = cand_scores;
+  m.out_idx = indices;
+  m.out_scores = scores;
+  e = launch_merge(m, W.mgrid, s);
+  if (e != cudaSuccess) return cuda_fail(e, "merge kernel");
+  if (op == PIVOT_OP_REUSE) return PIVOT_OK;
+
+  RefineArgs r{};
+  r.q = reinterpret_cast<const uint16_t*>(q);
+  r.w = w;
+  r.k = reinterpret_cast<const uint16_t*>(kc);
+  r.L = 0;
+  r.H = H;
+  r.D = d;
+  r.g = g;
+  r.c = c;
+  r.topk = k;
+  r.mc = 512 / H;
+  r.n_groups = B;
+  r.n_items = B * ((g + r.mc - 1) / r.mc);
+  r.cand = cand;
+  r.key_off = off_dev;
+  r.keys = W.keys;
+  r.counter = W.counters + 1;
+  r.status = W.status;
+  r.timeout_ns = g_timeout_ns;
+  e = launch_refine(r, nullptr, std::min(num_sms(), r.n_items), s);
+  if (e != cudaSuccess) return cuda_fail(e, "refine kernel");
+
+  RowSelArgs rs{};
+  rs.keys = W.keys;
+  rs.cand = cand;
+  rs.n_rows = (int64_t)B * g;
+  rs.L = 0;
+  rs.key_off = off_dev;
+  rs.g = g;
+  rs.c = c;
+  rs.topk = k;
+  rs.out_idx = indices;
+  rs.out_scores = scores;
+  e = launch_rowselect(rs, (int)std::min<int64_t>(8 * num_sms(), rs.n_rows), s);
+  return e == cudaSuccess ? PIVOT_OK : cuda_fail(e, "rowselect kernel");
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t pivot_workspace_size(int op, int64_t L, int H, int d, int k, int c, int g, pivot_dtype dt) {
+  if (op < 0 || op > 2) return 0;
+  if (op == PIVOT_OP_DENSE) g = 1;
+  if (check_common(L, H, d, dt, k, c, g, op) != PIVOT_OK) return 0;
+  return carve_prefill(nullptr, op, L, H, d, k, c, g, dt, false).bytes;
+}
+
+size_t pivot_varlen_workspace_size(int op, int B, const int64_t* off, int H, int d, int k, int c, int g,
+                                   pivot_dtype dt) {
+  if (op != PIVOT_OP_REUSE && op != PIVOT_OP_REFINE) return 0;
+  if (check_common(1, H, d, dt, k, c, g, op) != PIVOT_OK || check_offsets(B, off, g) != PIVOT_OK) return 0;
+  return carve_decode(nullptr, op, B, off, H, d, k, c, g, dt, false).bytes;
+}
+
+pivot_status pivot_indexer_dense(const void* q_I, const float* w_I, const void* k_I, int64_t L, int H, int d,
+                                 pivot_dtype dt, int k, int32_t* indices, float* scores_opt, void* ws,
+                                 size_t ws_bytes, pivot_stream_t stream) {
+  return run_prefill(PIVOT_OP_DENSE, q_I, w_I, k_I, L, H, d, dt, k, k, 1, indices, scores_opt, nullptr, nullptr,
+                     ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+pivot_status pivot_reuse(const void* q_I, const float* w_I, const void* k_I, int64_t L, int H, int d,
+                         pivot_dtype dt, int k, int g, int32_t* indices, float* scores_opt, void* ws,
+                         size_t ws_bytes, pivot_stream_t stream) {
+  return run_prefill(PIVOT_OP_REUSE, q_I, w_I, k_I, L, H, d, dt, k, k, g, indices, scores_opt, nullptr, nullptr,
+                     ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+pivot_status pivot_refine(const void* q_I, const float* w_I, const void* k_I, int64_t L, int H, int d,
+                          pivot_dtype dt, int k, int c, int g, int32_t* indices, float* scores_opt,
+                          int32_t* cand_opt, float* cand_scores_opt, void* ws, size_t ws_bytes,
+                          pivot_stream_t stream) {
+  return run_prefill(PIVOT_OP_REFINE, q_I, w_I, k_I, L, H, d, dt, k, c, g, indices, scores_opt, cand_opt,
+                     cand_scores_opt, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+pivot_status pivot_reuse_varlen(const void* q, const float* w, const void* k_cache, const int64_t* key_offsets_dev,
+                                const int64_t* key_offsets_host, int B, int H, int d, pivot_dtype dt, int k, int g,
+                                int32_t* indices, float* scores_opt, void* ws, size_t ws_bytes,
+                                pivot_stream_t stream) {
+  return run_decode(PIVOT_OP_REUSE, q, w, k_cache, key_offsets_dev, key_offsets_host, B, H, d, dt, k, k, g, indices,
+                    scores_opt, nullptr, nullptr, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+pivot_status pivot_refine_varlen(const void* q, const float* w, const void* k_cache,
+                                 const int64_t* key_offsets_dev, const int64_t* key_offsets_host, int B, int H,
+                                 int d, pivot_dtype dt, int k, int c, int g, int32_t* indices, float* scores_opt,
+                                 int32_t* cand_opt, float* cand_scores_opt, void* ws, size_t ws_bytes,
+                                 pivot_stream_t stream) {
+  return run_decode(PIVOT_OP_REFINE, q, w, k_cache, key_offsets_dev, key_offsets_host, B, H, d, dt, k, c, g,
+                    indices, scores_opt, cand_opt, cand_scores_opt, ws, ws_bytes,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+pivot_status pivot_last_device_status(const void* ws, pivot_stream_t stream) {
+  if (!ws) return PIVOT_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "stream sync");
+  int st = 0;
+  e = cudaMemcpy(&st, reinterpret_cast<const char*>(ws) + kStatusOff, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "status copy");
+  if (st & DEV_ERR_TIMEOUT) return PIVOT_ERR_DEVICE_TIMEOUT;
+  if (st & DEV_ERR_BOUNDS) return PIVOT_ERR_DEVICE_BOUNDS;
+  return PIVOT_OK;
+}
+
+const char* pivot_status_string(pivot_status s) {
+  switch (s) {
+    case PIVOT_OK: return "PIVOT_OK";
+    case PIVOT_ERR_INVALID_ARG: return "PIVOT_ERR_INVALID_ARG";
+    case PIVOT_ERR_UNSUPPORTED_SHAPE: return "PIVOT_ERR_UNSUPPORTED_SHAPE";
+    case PIVOT_ERR_WORKSPACE_TOO_SMALL: return "PIVOT_ERR_WORKSPACE_TOO_SMALL";
+    case PIVOT_ERR_CUDA: return "PIVOT_ERR_CUDA";
+    case PIVOT_ERR_DEVICE_TIMEOUT: return "PIVOT_ERR_DEVICE_TIMEOUT";
+    case PIVOT_ERR_DEVICE_BOUNDS: return "PIVOT_ERR_DEVICE_BOUNDS";
+  }
+  return "PIVOT_ERR_UNKNOWN";
+}
+
+const char* pivot_last_cuda_error(void) { return g_cuda_err; }
+
+int pivot_path(int op, int64_t L, int H, int d, int k, int c, int g, pivot_dtype dt) {
+  if (op < 0 || op > 2) return -1;
+  if (op == PIVOT_OP_DENSE) g = 1;
+  if (check_common(L, H, d, dt, k, c, g, op) != PIVOT_OK) return -1;
+  return tc_shape(H, d, dt) ? 1 : 0;
+}
+
+void pivot_set_device_timeout_ns(uint64_t ns) { g_timeout_ns = ns; }
+void pivot_set_debug_flags(int flags) { g_debug_flags = flags; }
+int pivot_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,237 @@
+// aux.cu -- the non-tensor-core kernels of the library:
+//   * rowselect_kernel  Eq. (9): per member row, the top-k of its candidates'
+//                       re-scored keys (written by the refine kernel);
+//   * plan_kernel       decode: split each sequence's prefix into chunks;
+//   * merge_kernel      decode: exact top-n of the union of a sequence's
+//                       chunk-partial top-n lists, then emit C (Refine) or the
+//                       Reuse rows (Eq. 6);
+//   * simt_kernel       portable CUDA-core path (fp32 inputs, or shapes the
+//                       tensor-core kernels do not take): Eq. (1)/(4)-(9) per
+//                       group with the same exact selection.
+// PIVOT: picx.dev summary of the paper, Methodology, Eq. (1)-(9).
+#include <cuda_bf16.h>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+#include "select.cuh"
+
+namespace pivot {
+
+// ------------------------------------------------------------------ Eq. (9)
+__global__ void __launch_bounds__(256) rowselect_kernel(const RowSelArgs a) {
+  extern __shared__ uint64_t sbuf[];  // c packed entries of the row
+  __shared__ SelSmem S;
+  const Group<256> G{(int)threadIdx.x, 0};
+  for (int64_t row = blockIdx.x; row < a.n_rows; row += gridDim.x) {
+    const int64_t grp = row / a.g;
+    int64_t P;
+    if (a.key_off)
+      P = a.key_off[grp + 1] - a.key_off[grp];
+    else
+      P = min64(grp * a.g + a.g, a.L);
+    const uint32_t n_c = (uint32_t)min64(a.c, P);
+    const uint32_t* kr = a.keys + row * (int64_t)a.c;
+    const int32_t* cr = a.cand + grp * (int64_t)a.c;
+    uint32_t nv = 0;
+    for (uint32_t i = G.tid; i < n_c; i += 256) {
+      const uint32_t key = __ldg(kr + i);
+      const int32_t id = __ldg(cr + i);
+      const bool ok = key != 0u && id >= 0;
+      sbuf[i] = ok ? pack_entry(key, (uint32_t)id) : 0ull;
+      nv += ok ? 1u : 0u;
+    }
+    uint32_t total;
+    group_offsets<256>(nv, &total, S, G);
+    G.sync();
+    const uint64_t th =
+        (total <= (uint32_t)a.topk) ? 1ull : radix_threshold<256>(sbuf, n_c, a.topk, a.topk, S, G);
+    emit_row<256>(sbuf, n_c, 0xFFFFFFFFu, th - 1ull, a.out_idx + row * a.topk,
+                  a.out_scores ? a.out_scores + row * a.topk : nullptr, (uint32_t)a.topk, S, G);
+    G.sync();
+  }
+}
+
+cudaError_t launch_rowselect(const RowSelArgs& a, int grid, cudaStream_t s) {
+  const size_t smem = (size_t)a.c * sizeof(uint64_t);
+  cudaFuncSetAttribute(rowselect_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  rowselect_kernel<<<grid, 256, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ decode plan
+// Sequence b (P_b keys) is cut into max(1, ceil(P_b / chunk)) near-equal chunks.
+__global__ void plan_kernel(const int64_t* __restrict__ key_off, int B, int64_t chunk, int32_t* item_seq,
+                            int64_t* item_s0, int64_t* item_s1, int32_t* seq_item0) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  int it = 0;
+  for (int b = 0; b < B; ++b) {
+    seq_item0[b] = it;
+    const int64_t P = key_off[b + 1] - key_off[b];
+    const int64_t n = max64(1, (P + chunk - 1) / chunk);
+    for (int64_t c = 0; c < n; ++c) {
+      item_seq[it] = b;
+      item_s0[it] = P * c / n;
+      item_s1[it] = P * (c + 1) / n;
+      ++it;
+    }
+  }
+  seq_item0[B] = it;
+}
+
+cudaError_t launch_plan_items(const int64_t* key_off, int B, int64_t chunk, int32_t* item_seq, int64_t* item_s0,
+                              int64_t* item_s1, int32_t* seq_item0, cudaStream_t s) {
+  plan_kernel<<<1, 32, 0, s>>>(key_off, B, chunk, item_seq, item_s0, item_s1, seq_item0);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ decode merge
+__global__ void __launch_bounds__(256) merge_kernel(const MergeArgs a) {
+  __shared__ SelSmem S;
+  __shared__ uint64_t bot[16];
+  __shared__ uint32_t nbot;
+  const Group<256> G{(int)threadIdx.x, 0};
+  uint64_t* scr = a.scratch + (uint64_t)blockIdx.x * a.cap;
+  for (int b = blockIdx.x; b < a.B; b += gridDim.x) {
+    const int i0 = a.seq_item0[b], i1 = a.seq_item0[b + 1];
+    const uint64_t* region = a.partial + (uint64_t)i0 * a.n_sel;
+    const uint32_t n = (uint32_t)(i1 - i0) * (uint32_t)a.n_sel;
+    uint32_t real = 0;
+    for (int i = i0; i < i1; ++i) real += a.partial_cnt[i];
+    const uint64_t th = (real <= (uint32_t)a.n_sel) ? 1ull : radix_threshold<256>(region, n, a.n_sel, a.n_sel, S, G);
+    const uint32_t m = compact_ge<256>(region, scr, n, th, S, G);
+    const int64_t P = a.key_off[b + 1] - a.key_off[b];
+    if (a.mode == EMIT_CAND) {
+      emit_row<256>(scr, m, 0xFFFFFFFFu, 0ull, a.cand + (int64_t)b * a.n_sel,
+                    a.cand_scores ? a.cand_scores + (int64_t)b * a.n_sel : nullptr, (uint32_t)a.n_sel, S, G);
+    } else {
+      emit_reuse<256>(scr, m, a.topk, P - a.g, a.g, (int64_t)b * a.g, a.out_idx, a.out_scores, S, bot, &nbot, G);
+    }
+    G.sync();
+  }
+}
+
+cudaError_t launch_merge(const MergeArgs& a, int grid, cudaStream_t s) {
+  merge_kernel<<<grid, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ portable path
+__device__ __forceinline__ float ld_elem(const void* p, int is_bf16, int64_t i) {
+  if (is_bf16) return __uint_as_float((uint32_t)(reinterpret_cast<const uint16_t*>(p)[i]) << 16);
+  return reinterpret_cast<const float*>(p)[i];
+}
+
+// sum_j w_j ReLU(q_j . k_s) with q/w in fp32 shared/global scratch
+__device__ __forceinline__ float simt_score(const float* qv, const float* wv, int H, int D, const void* k,
+                                            int is_bf16, int64_t krow) {
+  float total = 0.f;
+  for (int j = 0; j < H; ++j) {
+    float dot = 0.f;
+    for (int x = 0; x < D; ++x) dot = fmaf(qv[j * D + x], ld_elem(k, is_bf16, krow * D + x), dot);
+    total = fmaf(wv[j], fmaxf(dot, 0.f), total);
+  }
+  return total;
+}
+
+__global__ void __launch_bounds__(256) simt_kernel(const SimtArgs a) {
+  __shared__ SelSmem S;
+  __shared__ uint64_t bot[16];
+  __shared__ uint32_t nbot, cnt2;
+  const Group<256> G{(int)threadIdx.x, 0};
+  const int H = a.H, D = a.D;
+  float* qv = a.fscratch + (int64_t)blockIdx.x * (H * D + H);
+  float* wv = qv + H * D;
+  uint64_t* buf = a.scratch + (int64_t)blockIdx.x * a.scratch_per_block;
+  uint64_t* mb = buf + (a.scratch_per_block - a.c);  // member entries (Refine)
+  for (int64_t grp = blockIdx.x; grp < a.n_groups; grp += gridDim.x) {
+    int64_t kbase, P, mrow0, t_first, orow0;
+    int nm;
+    if (a.key_off) {
+      kbase = a.key_off[grp];
+      P = a.key_off[grp + 1] - kbase;
+      mrow0 = grp * a.g;
+      nm = a.g;
+      t_first = P - a.g;
+      orow0 = grp * a.g;
+    } else {
+      kbase = 0;
+      mrow0 = grp * a.g;
+      nm = (int)min64(a.g, a.L - mrow0);
+      P = mrow0 + nm;
+      t_first = mrow0;
+      orow0 = mrow0;
+    }
+    // Eq. (4): proxy = per-head mean, rounded to the input dtype (one member: the query itself)
+    for (int i = G.tid; i < H * D; i += 256) {
+      float s = 0.f;
+      for (int m = 0; m < nm; ++m) s += ld_elem(a.q, a.is_bf16, (mrow0 + m) * (int64_t)H * D + i);
+      float v = nm > 1 ? __fdiv_rn(s, (float)nm) : s;
+      if (a.is_bf16) v = __bfloat162float(__float2bfloat16_rn(v));
+      qv[i] = v;
+    }
+    for (int j = G.tid; j < H; j += 256) {
+      float s = 0.f;
+      for (int m = 0; m < nm; ++m) s += a.w[(mrow0 + m) * H + j];
+      wv[j] = nm > 1 ? __fdiv_rn(s, (float)nm) : s;
+    }
+    G.sync();
+    // Eq. (5) (Eq. (1) when g == 1) over the causal prefix s <= group end
+    for (int64_t s = G.tid; s < P; s += 256)
+      buf[s] = pack_entry(score_key(simt_score(qv, wv, H, D, a.k, a.is_bf16, kbase + s)), (uint32_t)s);
+    G.sync();
+    const uint32_t n = (uint32_t)P;
+    if (a.variant == 0) {
+      const uint64_t th = radix_threshold<256>(buf, n, a.topk, a.topk, S, G);
+      const uint32_t m = compact_ge<256>(buf, buf, n, th, S, G);
+      emit_row<256>(buf, m, 0xFFFFFFFFu, 0ull, a.out_idx + orow0 * a.topk,
+                    a.out_scores ? a.out_scores + orow0 * a.topk : nullptr, (uint32_t)a.topk, S, G);
+    } else if (a.variant == 1) {
+      const uint32_t nsel = (uint32_t)(a.topk + a.g - 1);
+      const uint64_t th = radix_threshold<256>(buf, n, nsel, nsel, S, G);
+      const uint32_t m = compact_ge<256>(buf, buf, n, th, S, G);
+      emit_reuse<256>(buf, m, a.topk, t_first, nm, orow0, a.out_idx, a.out_scores, S, bot, &nbot, G);
+    } else {
+      const uint64_t th = radix_threshold<256>(buf, n, a.c, a.c, S, G);  // Eq. (7)
+      const uint32_t m = compact_ge<256>(buf, buf, n, th, S, G);
+      if (a.cand_out)
+        emit_row<256>(buf, m, 0xFFFFFFFFu, 0ull, a.cand_out + grp * a.c,
+                      a.cand_scores ? a.cand_scores + grp * a.c : nullptr, (uint32_t)a.c, S, G);
+      for (int r = 0; r < nm; ++r) {
+        const int64_t t = t_first + r;
+        const int64_t qrow = mrow0 + r;
+        G.sync();
+        for (int i = G.tid; i < H * D; i += 256) qv[i] = ld_elem(a.q, a.is_bf16, qrow * (int64_t)H * D + i);
+        for (int j = G.tid; j < H; j += 256) wv[j] = a.w[qrow * H + j];
+        if (G.tid == 0) cnt2 = 0;
+        G.sync();
+        for (uint32_t i0 = 0; i0 < m; i0 += 256) {  // Eq. (8) over s in C, s <= t
+          const uint32_t i = i0 + G.tid;
+          bool pass = false;
+          uint64_t val = 0;
+          if (i < m) {
+            const uint32_t s = entry_idx(buf[i]);
+            if ((int64_t)s <= t) {
+              val = pack_entry(score_key(simt_score(qv, wv, H, D, a.k, a.is_bf16, kbase + s)), s);
+              pass = true;
+            }
+          }
+          warp_append(pass, val, mb, &cnt2);
+        }
+        G.sync();
+        const uint32_t n2 = cnt2;
+        const uint64_t th2 = radix_threshold<256>(mb, n2, a.topk, a.topk, S, G);  // Eq. (9)
+        const uint32_t m2 = compact_ge<256>(mb, mb, n2, th2, S, G);
+        emit_row<256>(mb, m2, 0xFFFFFFFFu, 0ull, a.out_idx + (orow0 + r) * a.topk,
+                      a.out_scores ? a.out_scores + (orow0 + r) * a.topk : nullptr, (uint32_t)a.topk, S, G);
+      }
+    }
+    G.sync();
+  }
+}
+
+cudaError_t launch_simt(const SimtArgs& a, int grid, cudaStream_t s) {
+  simt_kernel<<<grid, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace pivot

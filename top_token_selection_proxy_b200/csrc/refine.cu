@@ -1,0 +1,343 @@
+// refine.cu -- K2: PIVOT-Refine candidate re-scoring on tcgen05.
+//
+// PIVOT (picx.dev summary of the paper, Methodology, "Two Variants"):
+//   Eq. (8)  I_{t,s} = sum_j w_{t,j} ReLU(q_{t,j} . k_s)   for s in C (the
+//            group's proxy top-c) and every member t of the group.
+// The causal mask s <= t is applied per member.  This kernel produces the
+// per-member scores of all c candidates as order-preserving 32-bit keys
+// (0 = masked / no candidate); the member top-k (Eq. 9) is taken by the
+// row-select kernel.
+//
+// One persistent CTA per SM; a work item is (group, chunk of MC = 512/H
+// members).  Per item the members' query rows (MC*H rows x D, bf16) are the
+// MMA's B operand in shared memory (K-major, 128-byte swizzle).  Warps 5-7
+// gather 128 candidate key rows per tile with 16-byte cp.async into a
+// swizzled A tile (2-stage ring); warp 4 issues
+//     D[128 candidates x (members*H)] = K_gathered . Q_members^T
+// as up to two N=256 MMAs into two TMEM accumulators; warps 0-3 (one thread
+// per candidate lane) apply ReLU, weight each head by the member's own w and
+// sum the H heads per member in registers, then write the member's key row.
+#include <cuda_bf16.h>
+
+#include <cstddef>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+#include "select.cuh"
+
+namespace pivot {
+
+template <int H, int D>
+struct RefCfg {
+  static constexpr int NROW = 512;      // B rows (members * H) per item
+  static constexpr int MC = NROW / H;   // members per item
+  static constexpr int KB = D / 64;
+  static constexpr int BM = 128;
+  static constexpr int STAGES = 2;
+  static constexpr int A_BYTES = BM * D * 2;
+  static constexpr int B_BYTES = NROW * D * 2;
+  static constexpr int THREADS = 256;
+  static constexpr int NPROD = 96;      // gather threads (warps 5-7)
+};
+
+struct RefTail {
+  uint64_t full[2], empty[2], accf[2], acce[2];
+  uint32_t tmem_slot;
+  int item, nm, ntiles, nhalf, n_c;
+  volatile int abort_flag;
+  int64_t grp, key_base, qrow0, t0, orow0;
+  alignas(16) float w[512];  // read as float4
+};
+static_assert(offsetof(RefTail, w) % 16 == 0, "w must be 16-byte aligned");
+
+template <int H, int D>
+constexpr size_t refine_smem() {
+  using C = RefCfg<H, D>;
+  return 1024 + C::B_BYTES + C::STAGES * C::A_BYTES + sizeof(RefTail);
+}
+
+template <int H, int D>
+__global__ void __launch_bounds__(256, 1) refine_kernel(const RefineArgs a, uint32_t* __restrict__ out_keys) {
+  using C = RefCfg<H, D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sB = smem;
+  uint8_t* sA = smem + C::B_BYTES;
+  RefTail& T = *reinterpret_cast<RefTail*>(smem + C::B_BYTES + C::STAGES * C::A_BYTES);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&T.full[s], C::NPROD);
+      mbar_init(&T.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&T.accf[b], 1);
+      mbar_init(&T.acce[b], 128);
+    }
+    T.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(&T.tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = T.tmem_slot;
+
+  uint32_t p_st = 0, p_ph = 0;
+  uint32_t m_st = 0, m_ph = 0, m_ab = 0, m_aph = 0;
+  uint32_t e_ab = 0, e_aph = 0;
+  const int chunks = (a.g + C::MC - 1) / C::MC;
+  const bool decode = (a.key_off != nullptr);
+
+  for (;;) {
+    if (tid == 0) {
+      const int item = (int)atomicAdd(a.counter, 1u);
+      T.item = item;
+      if (item < a.n_items) {
+        // longest prefix first: prefill groups in descending order
+        const int64_t grp = decode ? (int64_t)(item / chunks) : (a.n_groups - 1 - item / chunks);
+        const int mc = item % chunks;
+        const int r0 = mc * C::MC;
+        int64_t P, nmem_g;
+        if (decode) {
+          P = a.key_off[grp + 1] - a.key_off[grp];
+          nmem_g = a.g;
+          T.key_base = a.key_off[grp];
+          T.qrow0 = grp * a.g + r0;
+          T.t0 = P - a.g + r0;
+          T.orow0 = grp * a.g + r0;
+        } else {
+          const int64_t first = grp * a.g;
+          const int64_t last = min64(first + a.g, a.L) - 1;
+          P = last + 1;
+          nmem_g = last - first + 1;
+          T.key_base = 0;
+          T.qrow0 = first + r0;
+          T.t0 = first + r0;
+          T.orow0 = first + r0;
+        }
+        T.grp = grp;
+        T.nm = (int)max64(0, min64(C::MC, nmem_g - r0));
+        T.n_c = (int)min64(a.c, P);
+        T.ntiles = (T.n_c + C::BM - 1) / C::BM;
+        T.nhalf = (T.nm * H + 255) / 256;
+      }
+    }
+    __syncthreads();
+    const int item = T.item;
+    if (item >= a.n_items || T.abort_flag) break;
+    const int nm = T.nm, ntiles = T.ntiles, nhalf = T.nhalf, n_c = T.n_c;
+    const int32_t* cand = a.cand + T.grp * (int64_t)a.c;
+
+    // ---------------------------------------------------------------- members' q rows -> B, w -> smem
+    {
+      constexpr int XC = D / 8;
+      const int units = nm * H * XC;
+      for (int u = tid; u < units; u += C::THREADS) {
+        const int xc = u % XC;
+        const int n = u / XC;  // = member * H + head
+        const uint4 v =
+            __ldg(reinterpret_cast<const uint4*>(a.q + (T.qrow0 * H + n) * (int64_t)D) + xc);
+        const int kb = xc >> 3, ch = xc & 7;
+        *reinterpret_cast<uint4*>(sB + kb * (C::NROW * 128) + n * 128 + ((ch ^ (n & 7)) << 4)) = v;
+      }
+      for (int u = tid; u < nm * H; u += C::THREADS) T.w[u] = __ldg(a.w + T.qrow0 * H + u);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (nm == 0 || ntiles == 0) {
+      __syncthreads();
+      continue;
+    }
+
+    if (warp >= 5) {
+      // ------------------------------------------------------------ gather producers
+      const int ptid = tid - 160;
+      constexpr int XC = D / 8;
+      int prev = -1;
+      bool ok = true;
+      for (int j = 0; j < ntiles; ++j) {
+        if (!mbar_wait(&T.empty[p_st], p_ph ^ 1u, a.timeout_ns, &T.abort_flag)) {
+          T.abort_flag = 1;
+          atomicOr(a.status, DEV_ERR_TIMEOUT);
+          ok = false;
+          break;
+        }
+        uint8_t* dst = sA + p_st * C::A_BYTES;
+        for (int u = ptid; u < C::BM * XC; u += C::NPROD) {
+          const int row = u / XC, xc = u % XC;
+          const int slot = j * C::BM + row;
+          const int s = (slot < n_c) ? __ldg(cand + slot) : -1;
+          const bool valid = s >= 0;
+          const uint16_t* src = a.k + (T.key_base + (valid ? s : 0)) * (int64_t)D + xc * 8;
+          const int kb = xc >> 3, ch = xc & 7;
+          cp_async_16_zfill(dst + kb * (C::BM * 128) + row * 128 + ((ch ^ (row & 7)) << 4), src, valid);
+        }
+        cp_async_commit();
+        if (prev >= 0) {
+          cp_async_wait<1>();
+          fence_proxy_async_smem();
+          mbar_arrive(&T.full[prev]);
+        }
+        prev = (int)p_st;
+        if (++p_st == C::STAGES) {
+          p_st = 0;
+          p_ph ^= 1u;
+        }
+      }
+      cp_async_wait<0>();
+      if (ok && prev >= 0) {
+        fence_proxy_async_smem();
+        mbar_arrive(&T.full[prev]);
+      }
+    } else if (warp == 4) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        const uint32_t baddr = smem_u32(sB);
+        for (int j = 0; j < ntiles; ++j) {
+          if (!mbar_wait(&T.full[m_st], m_ph, a.timeout_ns, &T.abort_flag)) {
+            T.abort_flag = 1;
+            atomicOr(a.status, DEV_ERR_TIMEOUT);
+            break;
+          }
+          const uint32_t aaddr = smem_u32(sA + m_st * C::A_BYTES);
+          bool ok = true;
+          for (int h = 0; h < nhalf; ++h) {
+            if (!mbar_wait(&T.acce[m_ab], m_aph ^ 1u, a.timeout_ns, &T.abort_flag)) {
+              T.abort_flag = 1;
+              atomicOr(a.status, DEV_ERR_TIMEOUT);
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const int nh = min(256, nm * H - 256 * h);
+            const uint32_t idesc = idesc_bf16_f32(C::BM, nh);
+            const uint32_t dtm = tmem + m_ab * 256u;
+#pragma unroll
+            for (int kb = 0; kb < C::KB; ++kb)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = sw128_kmajor_desc(aaddr + kb * (C::BM * 128) + kk * 32);
+                const uint64_t bd = sw128_kmajor_desc(baddr + kb * (C::NROW * 128) + h * 256 * 128 + kk * 32);
+                umma_bf16(dtm, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+              }
+            umma_commit(&T.accf[m_ab]);
+            if (++m_ab == 2) {
+              m_ab = 0;
+              m_aph ^= 1u;
+            }
+          }
+          if (!ok) break;
+          umma_commit(&T.empty[m_st]);
+          if (++m_st == C::STAGES) {
+            m_st = 0;
+            m_ph ^= 1u;
+          }
+        }
+      }
+    } else {
+      // ------------------------------------------------------------ epilogue (warps 0-3)
+      const int q4 = warp;  // TMEM lane quarter
+      const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+      constexpr int MPH = 256 / H;  // members per accumulator half
+      bool stop = false;
+      for (int j = 0; j < ntiles && !stop; ++j) {
+        const int slot = j * C::BM + q4 * 32 + lane;
+        const int s = (slot < n_c) ? __ldg(cand + slot) : -1;
+        for (int h = 0; h < nhalf; ++h) {
+          const bool ok = mbar_wait(&T.accf[e_ab], e_aph, a.timeout_ns, &T.abort_flag);
+          float sc[MPH];
+          if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int ml = 0; ml < MPH; ++ml) {
+              const int r = h * MPH + ml;
+              float part[4] = {0.f, 0.f, 0.f, 0.f};
+              if (r < nm) {
+#pragma unroll
+                for (int h0 = 0; h0 < H; h0 += 32) {
+                  uint32_t v[32];
+                  tmem_ld32(tmem + lane_base + e_ab * 256u + (uint32_t)(ml * H + h0), v);
+                  tmem_wait_ld();
+                  const float4* wv = reinterpret_cast<const float4*>(&T.w[r * H + h0]);
+#pragma unroll
+                  for (int i = 0; i < 8; ++i) {
+                    const float4 w4 = wv[i];
+                    part[0] = fmaf(w4.x, fmaxf(__uint_as_float(v[4 * i + 0]), 0.f), part[0]);
+                    part[1] = fmaf(w4.y, fmaxf(__uint_as_float(v[4 * i + 1]), 0.f), part[1]);
+                    part[2] = fmaf(w4.z, fmaxf(__uint_as_float(v[4 * i + 2]), 0.f), part[2]);
+                    part[3] = fmaf(w4.w, fmaxf(__uint_as_float(v[4 * i + 3]), 0.f), part[3]);
+                  }
+                }
+              }
+              sc[ml] = (part[0] + part[1]) + (part[2] + part[3]);
+            }
+            tc_fence_before();
+            mbar_arrive(&T.acce[e_ab]);
+          } else {
+            T.abort_flag = 1;
+            atomicOr(a.status, DEV_ERR_TIMEOUT);
+          }
+          if (++e_ab == 2) {
+            e_ab = 0;
+            e_aph ^= 1u;
+          }
+          if (named_bar_or(1, 128, T.abort_flag != 0)) {
+            stop = true;
+            break;
+          }
+          // Eq. (8) with the member's causal mask s <= t; key 0 marks "not eligible"
+          if (slot < a.c) {
+#pragma unroll
+            for (int ml = 0; ml < MPH; ++ml) {
+              const int r = h * MPH + ml;
+              if (r < nm) {
+                const int64_t t = T.t0 + r;
+                const bool valid = (s >= 0) && ((int64_t)s <= t);
+                out_keys[(T.orow0 + r) * (int64_t)a.c + slot] = valid ? score_key(sc[ml]) : 0u;
+              }
+            }
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  __syncthreads();
+  if (T.abort_flag) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 200000ull) {
+    }
+  }
+  if (warp == 4) tmem_dealloc(tmem, 512);
+}
+
+size_t refine_smem_bytes(int H, int D, int /*mc*/) {
+  if (H == 64 && D == 128) return refine_smem<64, 128>();
+  if (H == 64 && D == 64) return refine_smem<64, 64>();
+  return 0;
+}
+
+cudaError_t launch_refine(const RefineArgs& a, const CUtensorMap* /*qmap*/, int grid, cudaStream_t s) {
+  const size_t smem = refine_smem_bytes(a.H, a.D, a.mc);
+  uint32_t* keys = a.keys;
+  if (a.H == 64 && a.D == 128) {
+    auto k = refine_kernel<64, 128>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, 256, smem, s>>>(a, keys);
+  } else if (a.H == 64 && a.D == 64) {
+    auto k = refine_kernel<64, 64>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, 256, smem, s>>>(a, keys);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace pivot

@@ -1,0 +1,412 @@
+// scan.cu -- K1: fused proxy pooling + proxy scan + streaming exact select.
+//
+// PIVOT (picx.dev summary of the paper, Methodology):
+//   Eq. (4)  q-bar_j = mean of q_{t,j} over the group, w-bar_j = mean of w_{t,j}
+//   Eq. (5)  I-bar_s = sum_j w-bar_j ReLU(q-bar_j . k_s),  s <= group end
+//   Eq. (6)/(7) the group's top-(k+g-1) (Reuse) or top-c (Refine) by I-bar
+//   Eq. (1)  the dense indexer is the same scan with g = 1 and n_sel = k.
+//
+// One persistent CTA per SM.  A work item is a block of NB = 256/H groups
+// (consecutive, so their prefixes are nearly equal), scheduled longest
+// prefix first from an atomic counter.  Per item:
+//   * all threads pool the NB proxies (fp32 sum, divide by |G|, round to
+//     bf16) straight into the MMA's B operand in shared memory (K-major,
+//     128-byte swizzle) and w-bar into shared memory;
+//   * warp 0 streams 128-key tiles of k_I with TMA (4-stage ring);
+//   * warp 1 issues tcgen05.mma  D[128 keys x N] = K_tile . Proxy^T  into one
+//     of two 256-column TMEM accumulators (double buffered);
+//   * warps 2-5 (one thread per key / TMEM lane) load the accumulator row,
+//     apply ReLU, weight by w-bar and sum the H heads of each group in
+//     registers, mask s > group end, and feed the scores to a per-group
+//     streaming exact selection: packed (score, index) entries above the
+//     group's running threshold are appended to an L2-resident buffer; when a
+//     buffer fills it is cut back (radix threshold + compaction) and the
+//     threshold rises.  No score matrix ever reaches HBM.
+//   * at the end of the item the epilogue warps run the exact top-n_sel and
+//     emit rows (dense / Reuse), the candidate set C_i (Refine), or a
+//     chunk's partial top-n_sel (decode).
+#include <cuda_bf16.h>
+
+#include <cstddef>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+#include "select.cuh"
+
+namespace pivot {
+
+template <int H, int D>
+struct ScanCfg {
+  static constexpr int NB = 256 / H;  // groups per work item
+  static constexpr int N = NB * H;    // MMA N (256)
+  static constexpr int KB = D / 64;   // 128-byte k-blocks per row
+  static constexpr int BM = 128;      // keys per tile (MMA M)
+  static constexpr int STAGES = 4;
+  static constexpr int A_BYTES = BM * D * 2;
+  static constexpr int B_BYTES = N * D * 2;
+  static constexpr int THREADS = 192;
+  static constexpr int NEPI = 128;
+  static_assert(NB <= 16, "at most 16 groups per item");
+};
+
+struct ScanTail {
+  uint64_t full[4], empty[4], accf[2], acce[2];
+  uint64_t never;  // a barrier nothing arrives on (forced-timeout test hook)
+  uint32_t tmem_slot;
+  int item, nb_act, ntiles;
+  volatile int abort_flag;
+  int64_t row_base, s_begin, s_end, grp0;
+  int64_t e[16];      // last member position of each group (causal mask of the proxy)
+  int64_t mrow0[16];  // first q row of each group's members
+  int nmem[16];
+  uint32_t cnt[16];
+  uint64_t tau[16];
+  uint64_t bot[16];
+  uint32_t nbot;
+  SelSmem sel;
+  alignas(16) float wbar[256];  // read as float4
+};
+static_assert(offsetof(ScanTail, wbar) % 16 == 0, "wbar must be 16-byte aligned");
+
+template <int H, int D>
+constexpr size_t scan_smem() {
+  using C = ScanCfg<H, D>;
+  return 1024 + C::B_BYTES + C::STAGES * C::A_BYTES + sizeof(ScanTail);
+}
+
+template <int H, int D>
+__global__ void __launch_bounds__(192, 1) scan_kernel(const __grid_constant__ CUtensorMap kmap, const ScanArgs a) {
+  using C = ScanCfg<H, D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sB = smem;
+  uint8_t* sA = smem + C::B_BYTES;
+  ScanTail& T = *reinterpret_cast<ScanTail*>(smem + C::B_BYTES + C::STAGES * C::A_BYTES);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&T.full[s], 1);
+      mbar_init(&T.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&T.accf[b], 1);
+      mbar_init(&T.acce[b], C::NEPI);
+    }
+    mbar_init(&T.never, 1);
+    T.abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&kmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(&T.tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = T.tmem_slot;
+
+  uint32_t p_st = 0, p_ph = 0;                          // producer ring position
+  uint32_t m_st = 0, m_ph = 0, m_ab = 0, m_aph = 0;     // MMA: ring + accumulator
+  uint32_t e_ab = 0, e_aph = 0;                         // epilogue: accumulator
+  uint64_t* selbase = a.selbuf + (uint64_t)blockIdx.x * C::NB * (uint64_t)a.cap;
+  const Group<128> EG{tid - 64, 1};
+  const bool decode = (a.mode == EMIT_PARTIAL);
+
+  for (;;) {
+    // ---------------------------------------------------------------- item geometry
+    if (tid == 0) {
+      const int item = (int)atomicAdd(a.counter, 1u);
+      T.item = item;
+      if (item < a.n_items) {
+        if (!decode) {
+          const int64_t blk = (int64_t)a.n_items - 1 - item;  // longest prefix first
+          const int64_t g0 = blk * C::NB;
+          const int nb_act = (int)min64(C::NB, a.n_groups - g0);
+          T.grp0 = g0;
+          T.nb_act = nb_act;
+          for (int b = 0; b < C::NB; ++b) {
+            const int64_t grp = g0 + b;
+            if (b < nb_act) {
+              const int64_t t0 = grp * a.g;
+              const int64_t t1 = min64(t0 + a.g, a.L);
+              T.mrow0[b] = t0;
+              T.nmem[b] = (int)(t1 - t0);
+              T.e[b] = t1 - 1;
+            } else {
+              T.mrow0[b] = 0;
+              T.nmem[b] = 0;
+              T.e[b] = -1;
+            }
+          }
+          T.row_base = 0;
+          T.s_begin = 0;
+          T.s_end = T.e[nb_act - 1] + 1;
+        } else {
+          const int b = a.item_seq[item];
+          const int64_t P = a.key_off[b + 1] - a.key_off[b];
+          T.grp0 = b;
+          T.nb_act = 1;
+          for (int x = 0; x < C::NB; ++x) {
+            T.mrow0[x] = (x == 0) ? (int64_t)b * a.g : 0;
+            T.nmem[x] = (x == 0) ? a.g : 0;
+            T.e[x] = (x == 0) ? P - 1 : -1;
+          }
+          T.row_base = a.key_off[b];
+          T.s_begin = a.item_s0[item];
+          T.s_end = a.item_s1[item];
+        }
+        T.ntiles = (int)((T.s_end - T.s_begin + C::BM - 1) / C::BM);
+        for (int b = 0; b < C::NB; ++b) {
+          T.cnt[b] = 0;
+          T.tau[b] = 0;
+        }
+      }
+    }
+    __syncthreads();
+    const int item = T.item;
+    if (item >= a.n_items || T.abort_flag) break;
+    const int nb_act = T.nb_act;
+    const int ntiles = T.ntiles;
+
+    // ---------------------------------------------------------------- Eq. (4): pool proxies into B
+    {
+      constexpr int XC = D / 8;  // 16-byte chunks per row
+      for (int u = tid; u < C::NB * H * XC; u += C::THREADS) {
+        const int xc = u % XC;
+        const int hj = (u / XC) % H;
+        const int b = u / (XC * H);
+        const int n = b * H + hj;
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+        const int nm = T.nmem[b];
+        const int64_t r0 = T.mrow0[b];
+        for (int mm = 0; mm < nm; ++mm) {
+          const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.q + ((r0 + mm) * H + hj) * (int64_t)D) + xc);
+          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[2 * i] += __uint_as_float(wv[i] << 16);
+            acc[2 * i + 1] += __uint_as_float(wv[i] & 0xFFFF0000u);
+          }
+        }
+        uint32_t pk[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float lo = acc[2 * i], hi = acc[2 * i + 1];
+          if (nm > 1) {
+            lo = __fdiv_rn(lo, (float)nm);
+            hi = __fdiv_rn(hi, (float)nm);
+          }
+          const __nv_bfloat162 h2 = __floats2bfloat162_rn(lo, hi);
+          pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        const int kb = xc >> 3, ch = xc & 7;
+        uint8_t* dst = sB + kb * (C::N * 128) + n * 128 + ((ch ^ (n & 7)) << 4);
+        *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      for (int u = tid; u < C::NB * H; u += C::THREADS) {
+        const int b = u / H, hj = u % H;
+        const int nm = T.nmem[b];
+        const int64_t r0 = T.mrow0[b];
+        float s = 0.f;
+        for (int mm = 0; mm < nm; ++mm) s += __ldg(a.w + (r0 + mm) * H + hj);
+        T.wbar[u] = nm > 1 ? __fdiv_rn(s, (float)nm) : s;
+      }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+
+    if (warp == 0) {
+      // ------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        const int64_t row0 = T.row_base + T.s_begin;
+        for (int j = 0; j < ntiles; ++j) {
+          if (!mbar_wait(&T.empty[p_st], p_ph ^ 1u, a.timeout_ns, &T.abort_flag)) {
+            T.abort_flag = 1;
+            atomicOr(a.status, DEV_ERR_TIMEOUT);
+            break;
+          }
+          mbar_arrive_expect_tx(&T.full[p_st], C::A_BYTES);
+          uint8_t* dst = sA + p_st * C::A_BYTES;
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_2d(dst + kb * (C::BM * 128), &kmap, &T.full[p_st], kb * 64, (int)(row0 + (int64_t)j * C::BM));
+          if (++p_st == C::STAGES) {
+            p_st = 0;
+            p_ph ^= 1u;
+          }
+        }
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t idesc = idesc_bf16_f32(C::BM, C::N);
+        const uint32_t baddr = smem_u32(sB);
+        for (int j = 0; j < ntiles; ++j) {
+          if (!mbar_wait(&T.full[m_st], m_ph, a.timeout_ns, &T.abort_flag) ||
+              !mbar_wait(&T.acce[m_ab], m_aph ^ 1u, a.timeout_ns, &T.abort_flag)) {
+            T.abort_flag = 1;
+            atomicOr(a.status, DEV_ERR_TIMEOUT);
+            break;
+          }
+          tc_fence_after();
+          const uint32_t aaddr = smem_u32(sA + m_st * C::A_BYTES);
+          const uint32_t dtm = tmem + m_ab * 256u;
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = sw128_kmajor_desc(aaddr + kb * (C::BM * 128) + kk * 32);
+              const uint64_t bd = sw128_kmajor_desc(baddr + kb * (C::N * 128) + kk * 32);
+              umma_bf16(dtm, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+            }
+          umma_commit(&T.empty[m_st]);
+          umma_commit(&T.accf[m_ab]);
+          if (++m_st == C::STAGES) {
+            m_st = 0;
+            m_ph ^= 1u;
+          }
+          if (++m_ab == 2) {
+            m_ab = 0;
+            m_aph ^= 1u;
+          }
+        }
+      }
+    } else {
+      // ------------------------------------------------------------ epilogue + select
+      const int q4 = warp & 3;  // TMEM lane quarter this warp may access
+      const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+      const uint32_t need = (uint32_t)a.n_sel;
+      const uint32_t cap = (uint32_t)a.cap;
+      for (int j = 0; j < ntiles; ++j) {
+        float sc[C::NB];
+        bool ok;
+        if ((a.debug_flags & 1) && j == 0)
+          ok = mbar_wait(&T.never, 0u, a.timeout_ns, &T.abort_flag);  // runs out by design
+        else
+          ok = mbar_wait(&T.accf[e_ab], e_aph, a.timeout_ns, &T.abort_flag);
+        if (!ok) {
+          T.abort_flag = 1;
+          atomicOr(a.status, DEV_ERR_TIMEOUT);
+        }
+        if (ok) {
+          tc_fence_after();
+#pragma unroll
+          for (int b = 0; b < C::NB; ++b) {
+            float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int h0 = 0; h0 < H; h0 += 32) {
+              uint32_t r[32];
+              tmem_ld32(tmem + lane_base + e_ab * 256u + (uint32_t)(b * H + h0), r);
+              tmem_wait_ld();
+              const float4* wv = reinterpret_cast<const float4*>(&T.wbar[b * H + h0]);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float4 w4 = wv[i];
+                part[0] = fmaf(w4.x, fmaxf(__uint_as_float(r[4 * i + 0]), 0.f), part[0]);
+                part[1] = fmaf(w4.y, fmaxf(__uint_as_float(r[4 * i + 1]), 0.f), part[1]);
+                part[2] = fmaf(w4.z, fmaxf(__uint_as_float(r[4 * i + 2]), 0.f), part[2]);
+                part[3] = fmaf(w4.w, fmaxf(__uint_as_float(r[4 * i + 3]), 0.f), part[3]);
+              }
+            }
+            sc[b] = (part[0] + part[1]) + (part[2] + part[3]);
+          }
+          tc_fence_before();
+          mbar_arrive(&T.acce[e_ab]);
+        }
+        if (++e_ab == 2) {
+          e_ab = 0;
+          e_aph ^= 1u;
+        }
+        if (named_bar_or(1, 128, T.abort_flag != 0)) break;  // uniform across the epilogue warps
+        // streaming selection: append entries above each group's threshold
+        const int64_t s = T.s_begin + (int64_t)j * C::BM + q4 * 32 + lane;
+#pragma unroll
+        for (int b = 0; b < C::NB; ++b) {
+          if (b < nb_act) {
+            const bool valid = (s < T.s_end) && (s <= T.e[b]);
+            const uint64_t p = pack_entry(score_key(sc[b]), (uint32_t)s);
+            warp_append(valid && p > T.tau[b], p, selbase + (uint64_t)b * cap, &T.cnt[b]);
+          }
+        }
+        EG.sync();
+        for (int b = 0; b < nb_act; ++b) {
+          const uint32_t n = T.cnt[b];
+          if (n > cap - 128u) {  // cut back: keep a superset of the best `need`
+            uint64_t* buf = selbase + (uint64_t)b * cap;
+            const uint32_t maxk = need + (cap - 128u - need) / 2u;
+            const uint64_t th = radix_threshold<128>(buf, n, need, maxk, T.sel, EG);
+            const uint32_t m = compact_ge<128>(buf, buf, n, th, T.sel, EG);
+            if (EG.tid == 0) {
+              T.cnt[b] = m;
+              T.tau[b] = th - 1ull;  // admit x >= th from now on
+            }
+            EG.sync();
+          }
+        }
+      }
+      // ---------------------------------------------------------------- final exact selection + emit
+      if (!named_bar_or(1, 128, T.abort_flag != 0)) {
+        for (int b = 0; b < nb_act; ++b) {
+          uint64_t* buf = selbase + (uint64_t)b * cap;
+          const uint32_t n = T.cnt[b];
+          const uint64_t th = radix_threshold<128>(buf, n, need, need, T.sel, EG);
+          const uint32_t m = compact_ge<128>(buf, buf, n, th, T.sel, EG);
+          const int64_t grp = T.grp0 + b;
+          if (a.mode == EMIT_DENSE) {
+            emit_row<128>(buf, m, 0xFFFFFFFFu, 0ull, a.out_idx + grp * a.topk,
+                          a.out_scores ? a.out_scores + grp * a.topk : nullptr, (uint32_t)a.topk, T.sel, EG);
+          } else if (a.mode == EMIT_CAND) {
+            emit_row<128>(buf, m, 0xFFFFFFFFu, 0ull, a.cand + grp * a.n_sel,
+                          a.cand_scores ? a.cand_scores + grp * a.n_sel : nullptr, need, T.sel, EG);
+          } else if (a.mode == EMIT_REUSE) {
+            emit_reuse<128>(buf, m, a.topk, T.mrow0[b], T.nmem[b], T.mrow0[b], a.out_idx, a.out_scores, T.sel,
+                            T.bot, &T.nbot, EG);
+          } else {  // EMIT_PARTIAL: the chunk's exact top-n_sel, zero padded
+            uint64_t* dst = a.partial + (uint64_t)item * need;
+            for (uint32_t i = EG.tid; i < need; i += 128) dst[i] = (i < m) ? buf[i] : 0ull;
+            if (EG.tid == 0) a.partial_cnt[item] = m;
+          }
+          EG.sync();
+        }
+      }
+    }
+    __syncthreads();  // item done: B, the stage ring and the select state are free
+  }
+
+  __syncthreads();
+  if (T.abort_flag) {  // let in-flight async copies / MMAs drain before releasing TMEM
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 200000ull) {
+    }
+  }
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+size_t scan_smem_bytes(int H, int D) {
+  if (H == 64 && D == 128) return scan_smem<64, 128>();
+  if (H == 64 && D == 64) return scan_smem<64, 64>();
+  return 0;
+}
+
+cudaError_t launch_scan(const ScanArgs& a, const CUtensorMap* kmap, int grid, cudaStream_t s) {
+  const size_t smem = scan_smem_bytes(a.H, a.D);
+  if (a.H == 64 && a.D == 128) {
+    auto k = scan_kernel<64, 128>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, 192, smem, s>>>(*kmap, a);
+  } else if (a.H == 64 && a.D == 64) {
+    auto k = scan_kernel<64, 64>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<grid, 192, smem, s>>>(*kmap, a);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace pivot

@@ -1,0 +1,286 @@
+// select.cuh -- exact TopK machinery used by every kernel of the library.
+//
+// TopK order of the indexer (PIVOT, picx.dev summary, Eq. 1 "T_t = TopK"):
+// larger score first; equal scores -> lower key index first; -0.0 == +0.0.
+// Each (score, index) pair is packed into one uint64 whose unsigned order is
+// exactly that order:
+//     packed = orderkey(score) << 32 | (0xFFFFFFFF - index)
+// so all packed values of one row are distinct and "the n best" is "the n
+// largest packed values".  Selection is a most-significant-digit radix
+// select (8-bit digits, shared-memory histogram) followed by a stream
+// compaction, run by a group of NT threads that sync on one named barrier.
+#pragma once
+#include <cstdint>
+#include "ptx.cuh"
+
+namespace pivot {
+
+__device__ __forceinline__ uint32_t score_key(float x) {
+  uint32_t b = __float_as_uint(x);
+  if (b == 0x80000000u) b = 0u;  // -0.0 ties with +0.0
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_score(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+__device__ __forceinline__ uint64_t pack_entry(uint32_t key, uint32_t idx) {
+  return ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - idx);
+}
+__device__ __forceinline__ uint32_t entry_idx(uint64_t p) { return 0xFFFFFFFFu - (uint32_t)p; }
+__device__ __forceinline__ float entry_score(uint64_t p) { return key_score((uint32_t)(p >> 32)); }
+
+struct SelSmem {
+  uint32_t hist[256];
+  uint32_t warp_tot[32];
+  uint32_t scal[4];
+};
+
+// A group of NT threads (NT multiple of 32, tid in [0, NT)) synchronised by
+// named barrier `bar` (bar 0 with NT == blockDim.x is __syncthreads).
+template <int NT>
+struct Group {
+  int tid;
+  int bar;
+  __device__ __forceinline__ void sync() const { named_bar_sync(bar, NT); }
+};
+
+// Warp-aggregated append of `val` (when `pass`) to buf[*cnt ...]; the whole warp calls.
+__device__ __forceinline__ void warp_append(bool pass, uint64_t val, uint64_t* buf, uint32_t* cnt) {
+  const uint32_t m = __ballot_sync(0xFFFFFFFFu, pass);
+  if (m == 0u) return;
+  const int leader = __ffs(m) - 1;
+  uint32_t base = 0;
+  if ((int)lane_id() == leader) base = atomicAdd(cnt, (uint32_t)__popc(m));
+  base = __shfl_sync(0xFFFFFFFFu, base, leader);
+  if (pass) buf[base + __popc(m & lanemask_lt())] = val;
+}
+
+// Returns a threshold T such that count{ buf[i] >= T } lies in [need, max_keep]
+// (exactly `need` when max_keep == need).  Requires need <= n.  All NT threads
+// call it and get the same T.  T == 0 keeps everything.
+template <int NT>
+__device__ uint64_t radix_threshold(const uint64_t* buf, uint32_t n, uint32_t need, uint32_t max_keep,
+                                    SelSmem& S, const Group<NT>& G) {
+  if (n <= max_keep) return 0ull;
+  uint64_t prefix = 0;
+  uint32_t above = 0;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    for (int i = G.tid; i < 256; i += NT) S.hist[i] = 0u;
+    G.sync();
+    for (uint32_t i0 = 0; i0 < n; i0 += NT) {  // uniform trip count: whole warps stay converged
+      const uint32_t i = i0 + G.tid;
+      uint32_t bin = 256u;  // 256 = not counted
+      if (i < n) {
+        const uint64_t x = buf[i];
+        if (shift == 56 || (x >> (shift + 8)) == prefix) bin = (uint32_t)(x >> shift) & 255u;
+      }
+      // warp-aggregated histogram update: one atomic per distinct bin in the warp
+      const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
+      if (bin < 256u && (int)lane_id() == __ffs(peers) - 1) atomicAdd(&S.hist[bin], (uint32_t)__popc(peers));
+    }
+    G.sync();
+    if (G.tid < 32) {
+      const int l = G.tid;
+      uint32_t loc[8], sum = 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        loc[u] = S.hist[255 - 8 * l - u];
+        sum += loc[u];
+      }
+      uint32_t incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (l >= o) incl += v;
+      }
+      const uint32_t excl = incl - sum;
+      if (above + excl < need && need <= above + incl) {
+        uint32_t c = above + excl;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (c + loc[u] >= need) {
+            S.scal[0] = 255u - 8u * l - u;
+            S.scal[1] = c;
+            S.scal[2] = loc[u];
+            break;
+          }
+          c += loc[u];
+        }
+      }
+    }
+    G.sync();
+    const uint32_t digit = S.scal[0];
+    above = S.scal[1];
+    const uint32_t h = S.scal[2];
+    prefix = (prefix << 8) | digit;
+    if (above + h <= max_keep || shift == 0) return prefix << shift;
+  }
+  return prefix;
+}
+
+// Inclusive warp scan of v.
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
+  const int l = lane_id();
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xFFFFFFFFu, v, o);
+    if (l >= o) v += t;
+  }
+  return v;
+}
+
+// Block-level exclusive offsets of per-thread counts: returns this thread's
+// offset; *total gets the group total.  Two syncs.
+template <int NT>
+__device__ __forceinline__ uint32_t group_offsets(uint32_t cnt, uint32_t* total, SelSmem& S, const Group<NT>& G) {
+  const uint32_t incl = warp_incl_scan(cnt);
+  const int w = G.tid >> 5;
+  if ((G.tid & 31) == 31) S.warp_tot[w] = incl;
+  G.sync();
+  uint32_t off = 0, tot = 0;
+#pragma unroll
+  for (int i = 0; i < NT / 32; ++i) {
+    const uint32_t t = S.warp_tot[i];
+    if (i < w) off += t;
+    tot += t;
+  }
+  *total = tot;
+  return off + incl - cnt;
+}
+
+// Stream-compact the entries >= T of src[0..n) into dst[0..m) (dst may be
+// src: every chunk is fully read before any of its survivors is written, and
+// survivors never move forward).  Returns m.
+template <int NT, int V = 4>
+__device__ uint32_t compact_ge(const uint64_t* src, uint64_t* dst, uint32_t n, uint64_t T, SelSmem& S,
+                               const Group<NT>& G) {
+  uint32_t base = 0;
+  for (uint32_t c0 = 0; c0 < n; c0 += NT * V) {
+    uint64_t x[V];
+    uint32_t keep = 0, cnt = 0;
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      const uint32_t i = c0 + v * NT + G.tid;
+      x[v] = (i < n) ? src[i] : 0ull;
+      const bool k = (i < n) && (x[v] >= T);
+      keep |= (k ? 1u : 0u) << v;
+      cnt += k ? 1u : 0u;
+    }
+    uint32_t total;
+    uint32_t pos = base + group_offsets<NT>(cnt, &total, S, G);
+#pragma unroll
+    for (int v = 0; v < V; ++v)
+      if (keep & (1u << v)) dst[pos++] = x[v];
+    base += total;
+    G.sync();
+  }
+  return base;
+}
+
+// Count entries of buf[0..n) with index <= t (all threads get the total).
+template <int NT>
+__device__ uint32_t count_idx_le(const uint64_t* buf, uint32_t n, uint32_t t, SelSmem& S, const Group<NT>& G) {
+  uint32_t c = 0;
+  for (uint32_t i = G.tid; i < n; i += NT) c += (entry_idx(buf[i]) <= t) ? 1u : 0u;
+  uint32_t total;
+  group_offsets<NT>(c, &total, S, G);
+  G.sync();
+  return total;
+}
+
+// Write the indices (and optionally scores) of the entries of buf[0..n) that
+// satisfy  idx <= t_max && entry > cut  to row[0..) in arbitrary order; pad
+// the rest of row[0..width) with -1.  Returns the number written.
+template <int NT>
+__device__ uint32_t emit_row(const uint64_t* buf, uint32_t n, uint32_t t_max, uint64_t cut, int32_t* row,
+                             float* row_scores, uint32_t width, SelSmem& S, const Group<NT>& G) {
+  uint32_t base = 0;
+  constexpr int V = 4;
+  for (uint32_t c0 = 0; c0 < n; c0 += NT * V) {
+    uint64_t x[V];
+    uint32_t keep = 0, cnt = 0;
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      const uint32_t i = c0 + v * NT + G.tid;
+      x[v] = (i < n) ? buf[i] : 0ull;
+      const bool k = (i < n) && (entry_idx(x[v]) <= t_max) && (x[v] > cut);
+      keep |= (k ? 1u : 0u) << v;
+      cnt += k ? 1u : 0u;
+    }
+    uint32_t total;
+    uint32_t pos = base + group_offsets<NT>(cnt, &total, S, G);
+#pragma unroll
+    for (int v = 0; v < V; ++v)
+      if ((keep & (1u << v)) && pos < width) {
+        row[pos] = (int32_t)entry_idx(x[v]);
+        if (row_scores) row_scores[pos] = entry_score(x[v]);
+        ++pos;
+      }
+    base += total;
+    G.sync();
+  }
+  const uint32_t m = base < width ? base : width;
+  for (uint32_t i = m + G.tid; i < width; i += NT) {
+    row[i] = -1;
+    if (row_scores) row_scores[i] = -__int_as_float(0x7f800000);
+  }
+  return m;
+}
+
+// Eq. (6) emit for one group after its exact top-(k+g-1) sits in buf[0..m):
+// member t keeps the k best of { entries with index <= t }.  Removing the
+// r <= g-1 entries above t leaves at least k; the ones to drop beyond the
+// k best are the lowest eligible entries, all among the m-k lowest of buf.
+template <int NT>
+__device__ void emit_reuse(uint64_t* buf, uint32_t m, int topk, int64_t t_first, int nmem, int64_t out_row0,
+                           int32_t* out_idx, float* out_sc, SelSmem& S, uint64_t* bot, uint32_t* nbot,
+                           const Group<NT>& G) {
+  uint32_t nb = 0;
+  if (m > (uint32_t)topk) {
+    const uint64_t Tk = radix_threshold<NT>(buf, m, topk, topk, S, G);
+    if (G.tid == 0) *nbot = 0;
+    G.sync();
+    for (uint32_t i = G.tid; i < m; i += NT) {
+      const uint64_t x = buf[i];
+      if (x < Tk) {
+        const uint32_t p = atomicAdd(nbot, 1u);
+        if (p < 16) bot[p] = x;
+      }
+    }
+    G.sync();
+    nb = *nbot;
+    if (G.tid == 0) {  // ascending insertion sort of at most g-1 entries
+      for (uint32_t i = 1; i < nb && i < 16; ++i) {
+        const uint64_t v = bot[i];
+        int j = (int)i - 1;
+        while (j >= 0 && bot[j] > v) {
+          bot[j + 1] = bot[j];
+          --j;
+        }
+        bot[j + 1] = v;
+      }
+    }
+    G.sync();
+  }
+  for (int r = 0; r < nmem; ++r) {
+    const int64_t t = t_first + r;
+    uint64_t cut = 0;
+    if (nb > 0) {
+      const uint32_t elig = count_idx_le<NT>(buf, m, (uint32_t)t, S, G);
+      if (elig > (uint32_t)topk) {
+        const uint32_t mdrop = elig - topk;
+        uint32_t c = 0;
+        for (uint32_t u = 0; u < nb && u < 16; ++u)
+          if (entry_idx(bot[u]) <= (uint32_t)t && ++c == mdrop) {
+            cut = bot[u];
+            break;
+          }
+      }
+    }
+    const int64_t row = out_row0 + r;
+    emit_row<NT>(buf, m, (uint32_t)t, cut, out_idx + row * topk, out_sc ? out_sc + row * topk : nullptr,
+                 (uint32_t)topk, S, G);
+  }
+}
+
+}  // namespace pivot
