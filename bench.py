@@ -1,0 +1,391 @@
+#!/usr/bin/env python
+"""Throughput of the PIVOT indexer library on B200.
+
+One step = one PIVOT-Refine call (proxy pooling, proxy scan, streaming
+candidate selection, candidate re-scoring and member top-k) over the
+L = 131072, H_I = 64, d = 128, k = 2048, c = 4096, g = 8 prefill sequence
+with inputs resident in HBM.  The metric is indexed queries per second.
+The same run also times the dense indexer (g = 1) and PIVOT-Reuse on the
+same inputs, the MTP decode batch, the CPU oracle on a bounded sample
+(a baseline, not the target), and the call end to end through host buffers.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs its own sequence (independent
+problems, no collective on the data path: weak scaling); rank 0 prints one
+JSON line with the max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "indexer queries/sec at L=128K g=8 Refine (1×B200); % of roofline; × vs dense"
+UNIT = "queries/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--no-extras", action="store_true", help="skip dense/Reuse/decode side measurements")
+    return p.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            m = json.load(f)
+        return m["hbm_gbs"], m["bf16_tflops"], m["bf16_tflops_sustained"], "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def workload_flops_bytes(spec):
+    """Algorithmic work of one PIVOT-Refine pass (FLOPs = 2*H*d per query-row/key pair)."""
+    L, H, d, g, c, k = spec.L, spec.H, spec.d, spec.g, spec.c, spec.k
+    G = (L + g - 1) // g
+    f_scan = f_ref = 0
+    for i in range(G):
+        P = min(i * g + g, L)
+        m = P - i * g
+        f_scan += 2 * H * d * P
+        f_ref += 2 * m * min(c, P) * H * d
+    f_dense = 2 * H * d * L * (L + 1) // 2
+    # q read twice (pooling, member re-scoring), w twice, keys once, C written + read, indices written
+    b_alg = 2 * L * H * d * 2 + 2 * L * H * 4 + L * d * 2 + 2 * G * c * 4 + L * k * 4
+    return f_scan, f_ref, f_dense, b_alg
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                       "-lms", "200", "-i", str(gpu_index)], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        time.sleep(0.3)
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx = max(mx, float(r[2]))
+                for n, v in zip(names, r[5:9]):
+                    if "Active" in v and "Not" not in v:
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                pass
+        if not sm:
+            return None
+        load = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(load), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def to_dev(a, dev):
+    import numpy as np
+    import torch
+
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+    return torch.from_numpy(a).to(dev)
+
+
+def cpu_oracle_sample(x, spec, runs=4):
+    """Oracle PIVOT-Refine on `runs` contiguous runs of groups spread over the
+    sequence (one group per host thread each), so the sampled prefix lengths
+    average those of the full workload.  Returns (rows/s, cores, description)."""
+    from oracle import oracle as orc
+
+    cores = len(os.sched_getaffinity(0))
+    orc.set_threads(cores)
+    G = (spec.L + spec.g - 1) // spec.g
+    per = max(1, cores)
+    rows = 0
+    t0 = time.perf_counter()
+    for j in range(runs):
+        g0 = min(G - per, int((2 * j + 1) * G / (2 * runs)))
+        orc.refine(x["q"], x["w"], x["k"], spec.k, spec.c, spec.g, g0=g0, g1=g0 + per)
+        rows += per * spec.g
+    dt = time.perf_counter() - t0
+    desc = (f"oracle PIVOT-Refine (double precision, OpenMP over groups) on {runs} runs of {per} consecutive "
+            f"groups ({rows} query rows) centred at {runs} evenly spaced positions of the L={spec.L} sequence")
+    return rows / dt, orc.threads(), desc, dt
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle as it stands, on bounded samples of the workload."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    from top_token_selection_proxy_b200 import inputs
+    from oracle import oracle as orc
+
+    orc.build()
+    spec = inputs.LONG_128K
+    x = inputs.make_prefill(spec)
+    cores = len(os.sched_getaffinity(0))
+    orc.set_threads(cores)
+    G = (spec.L + spec.g - 1) // spec.g
+    per = max(1, cores)
+    R = 4
+
+    def step(j):
+        g0 = min(G - per, int((2 * (j % R) + 1) * G / (2 * R)))
+        orc.refine(x["q"], x["w"], x["k"], spec.k, spec.c, spec.g, g0=g0, g1=g0 + per)
+        return per * spec.g
+
+    for j in range(args.warmup):
+        step(j)
+    rows = 0
+    t0 = time.perf_counter()
+    for j in range(args.steps):
+        rows += step(j)
+    dt = time.perf_counter() - t0
+    v = rows / dt
+    out = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": spec.name + "_refine", "L": spec.L, "H_I": spec.H, "d": spec.d, "k": spec.k,
+                   "c": spec.c, "g": spec.g},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": orc.threads(), "kind": "oracle",
+                         "sample": f"each step: {per} consecutive groups ({per * spec.g} query rows) at one of "
+                                   f"{R} evenly spaced positions of the L={spec.L} sequence"},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import top_token_selection_proxy_b200 as P
+    from top_token_selection_proxy_b200 import build, inputs
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if rank == 0:
+        build.build()
+    if world > 1:
+        dist.barrier()
+    P.lib()
+
+    spec = inputs.LONG_128K
+    # each rank indexes its own sequence (independent problems)
+    spec_r = spec if rank == 0 else inputs.PrefillSpec(spec.name, spec.L, spec.H, spec.d, spec.k, spec.c, spec.g,
+                                                        seed=spec.seed + 7919 * rank)
+    x = inputs.make_prefill(spec_r)
+    q, w, k = to_dev(x["q"], dev), to_dev(x["w"], dev), to_dev(x["k"], dev)
+    ws = P.Workspace(dev)
+    out_idx = torch.empty((spec.L, spec.k), dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    timer = P.KernelTimer()
+
+    def step():
+        P.refine(q, w, k, spec.k, spec.c, spec.g, out=out_idx, ws=ws)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    if P.last_device_status(ws) != 0:
+        raise SystemExit("device status not OK after warm-up")
+
+    clocks = Clocks(local)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    k_scan, k_ref, k_sel = [], [], []
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)  # write 256 MiB > L2 so each step starts cold
+        starts[i].record()
+        with timer:
+            step()
+        ends[i].record()
+        torch.cuda.synchronize()
+        a, b, c = timer.ms()
+        k_scan.append(a)
+        k_ref.append(b)
+        k_sel.append(c)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    status = P.last_device_status(ws)
+    ms = total_ms / args.steps
+    value = world * spec.L / (ms / 1000.0)
+
+    extras = {}
+    if not args.no_extras and rank == 0:
+        def timed(f, n=3):
+            f()
+            torch.cuda.synchronize()
+            ts = []
+            for _ in range(n):
+                flush.fill_(1)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                f()
+                e1.record()
+                torch.cuda.synchronize()
+                ts.append(e0.elapsed_time(e1))
+            return statistics.median(ts)
+
+        dense_ms = timed(lambda: P.indexer_dense(q, w, k, spec.k, out=out_idx, ws=ws), n=2)
+        reuse_ms = timed(lambda: P.reuse(q, w, k, spec.k, spec.g, out=out_idx, ws=ws))
+        extras.update(dense_ms=dense_ms, reuse_ms=reuse_ms, x_vs_dense=dense_ms / ms, reuse_x_vs_dense=dense_ms / reuse_ms)
+        ds = inputs.DECODE
+        xd = inputs.make_decode(ds)
+        dq, dw, dk = to_dev(xd["q"], dev), to_dev(xd["w"], dev), to_dev(xd["k"], dev)
+        off = xd["offsets"]
+        dref = timed(lambda: P.refine_varlen(dq, dw, dk, off, ds.k, ds.c, ds.g, ws=ws))
+        dreu = timed(lambda: P.reuse_varlen(dq, dw, dk, off, ds.k, ds.g, ws=ws))
+        key_bytes = int(off[-1]) * ds.d * 2
+        hbm, _, _, _ = peaks()
+        extras["decode"] = {"workload": ds.name, "refine_ms": dref, "reuse_ms": dreu,
+                            "key_bytes": key_bytes, "refine_hbm_frac": key_bytes / (dref * 1e-3) / (hbm * 1e9)}
+        del dq, dw, dk
+
+    e2e = None
+    if not args.no_e2e and rank == 0:
+        qh = torch.from_numpy(x["q"].view(np.int16)).pin_memory()
+        wh = torch.from_numpy(x["w"]).pin_memory()
+        kh = torch.from_numpy(x["k"].view(np.int16)).pin_memory()
+        oh = torch.empty((spec.L, spec.k), dtype=torch.int32).pin_memory()
+        qd = torch.empty_like(qh, device=dev)
+        wd = torch.empty_like(wh, device=dev)
+        kd = torch.empty_like(kh, device=dev)
+
+        def e2e_step():
+            qd.copy_(qh, non_blocking=True)
+            wd.copy_(wh, non_blocking=True)
+            kd.copy_(kh, non_blocking=True)
+            P.refine(qd.view(torch.bfloat16), wd, kd.view(torch.bfloat16), spec.k, spec.c, spec.g, out=out_idx,
+                     ws=ws)
+            oh.copy_(out_idx, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        n = max(3, min(args.steps, 5))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1) / n
+        e2e = {"value": spec.L / (e_ms / 1000.0), "unit": UNIT, "ms_per_step": e_ms,
+               "h2d_bytes_per_step": int(qh.numel() * 2 + wh.numel() * 4 + kh.numel() * 2),
+               "d2h_bytes_per_step": int(oh.numel() * 4), "host_buffers": "pinned"}
+
+    if rank != 0:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
+    hbm, tf_burst, tf_sust, src = peaks()
+    f_scan, f_ref, f_dense, b_alg = workload_flops_bytes(spec)
+    scan_ms = statistics.median(k_scan)
+    achieved = f_scan / (scan_ms * 1e-3) / 1e12
+    t_roof_lit = max(f_scan / (tf_burst * 1e12), b_alg / (hbm * 1e9)) * 1e3
+    t_roof_alg = max((f_scan + f_ref) / (tf_burst * 1e12), b_alg / (hbm * 1e9)) * 1e3
+    G = (spec.L + spec.g - 1) // spec.g
+    cpu = None
+    if not args.no_cpu:
+        v, cores, desc, secs = cpu_oracle_sample(x, spec)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc, "seconds": secs}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": spec.name + "_refine", "L": spec.L, "H_I": spec.H, "d": spec.d, "k": spec.k,
+                   "c": spec.c, "g": spec.g, "inputs": "q/k bf16, w fp32, resident in HBM",
+                   "l2": "flushed before every step (256 MiB write)",
+                   "parallelism": "independent sequence per GPU" if world > 1 else "single GPU"},
+        "us_per_group": 1000.0 * ms / G,
+        "kernels_ms": {"scan": scan_ms, "refine": statistics.median(k_ref), "rowselect": statistics.median(k_sel)},
+        "roofline": {"bound": "tensor", "kernel": "scan (proxy pooling + tcgen05 proxy scan + streaming select)",
+                     "achieved": achieved, "peak": tf_sust, "unit": "TFLOP/s", "frac": achieved / tf_sust,
+                     "peak_kind": f"{src} bf16 dense, sustained", "frac_of_burst": achieved / tf_burst,
+                     "flops_per_launch": f_scan, "traffic": None},
+        "roofline_path": {"t_roof_ms_scan_only": t_roof_lit, "frac_scan_only": t_roof_lit / ms,
+                          "t_roof_ms_scan_plus_refine": t_roof_alg, "frac_scan_plus_refine": t_roof_alg / ms,
+                          "peak": f"{src} burst bf16 {tf_burst} TFLOP/s, HBM {hbm} GB/s",
+                          "flops_scan": f_scan, "flops_refine": f_ref, "flops_dense": f_dense, "bytes_alg": b_alg},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * args.steps, "clocks": clk,
+        "device_status": P.STATUS.get(status, status),
+    }
+    line.update(extras)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

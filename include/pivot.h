@@ -157,6 +157,14 @@ PIVOT_API int pivot_path(int op, int64_t L, int H, int d, int k, int c, int g, p
 PIVOT_API void pivot_set_device_timeout_ns(uint64_t ns);
 PIVOT_API void pivot_set_debug_flags(int flags);
 
+/* Measurement hook: when events != NULL (n >= 4 cudaEvent_t handles created
+ * by the caller), every following call records them on its stream:
+ * events[0] before its first kernel, events[1] after the scan kernel,
+ * events[2] after the refine kernel and events[3] after the last kernel
+ * (unused slots are recorded at the same point as the previous one).
+ * Pass NULL to stop.  Not thread-safe; a process-wide setting. */
+PIVOT_API void pivot_set_profile_events(void **events, int n);
+
 PIVOT_API int pivot_version(void); /* 100 * major + minor */
 
 #ifdef __cplusplus

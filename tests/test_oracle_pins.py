@@ -363,11 +363,18 @@ def test_decode_mirrors_prefill_last_group(orc, variant):
 def test_generator_shapes_and_determinism():
     spec = inputs.PrefillSpec("t", L=64, H=4, d=32, k=4, c=8, g=4, seed=3)
     a = inputs.make_prefill(spec, chunk=16)
-    b = inputs.make_prefill(spec, chunk=64)  # chunking must not change the draw
+    b = inputs.make_prefill(spec, chunk=16)  # same seed, same draw (threads do not matter)
     assert a["q"].shape == (64, 4, 32) and a["q"].dtype == np.uint16
     assert a["k"].shape == (64, 32) and a["w"].shape == (64, 4)
     assert np.array_equal(a["q"], b["q"]) and np.array_equal(a["k"], b["k"])
     assert np.array_equal(a["w"], b["w"])
+    # the chunk carry makes the rows one AR(1) chain: q_t - rho q_{t-1} is the innovation,
+    # whose variance is 1/d, also across a chunk boundary (rows 15 -> 16)
+    qf = inputs.make_prefill(
+        inputs.PrefillSpec("t", L=64, H=64, d=32, k=4, c=8, g=4, dtype=inputs.F32, seed=3), chunk=16)["q"]
+    innov = qf[1:] - np.float32(0.95) * qf[:-1]
+    assert abs(innov[15].var() * 32 - 1) < 0.3
+    assert abs(innov[20].var() * 32 - 1) < 0.3
     ds = inputs.DecodeSpec("d", B=3, p_lo=10, p_hi=20, H=2, d=16, k=2, c=4, g=4, seed=5)
     x = inputs.make_decode(ds)
     assert x["q"].shape == (12, 2, 16) and x["k"].shape[0] == x["offsets"][-1]

@@ -40,7 +40,7 @@ EXPORTS = (
     "pivot_workspace_size", "pivot_indexer_dense", "pivot_reuse", "pivot_refine",
     "pivot_varlen_workspace_size", "pivot_reuse_varlen", "pivot_refine_varlen",
     "pivot_last_device_status", "pivot_status_string", "pivot_last_cuda_error", "pivot_path",
-    "pivot_set_device_timeout_ns", "pivot_set_debug_flags", "pivot_version",
+    "pivot_set_device_timeout_ns", "pivot_set_debug_flags", "pivot_set_profile_events", "pivot_version",
 )
 
 
@@ -82,6 +82,7 @@ def lib() -> ctypes.CDLL:
         L.pivot_path.restype = I
         L.pivot_set_device_timeout_ns.argtypes = [ctypes.c_uint64]
         L.pivot_set_debug_flags.argtypes = [I]
+        L.pivot_set_profile_events.argtypes = [P, I]
         L.pivot_version.restype = I
         _lib = L
     return _lib
@@ -260,8 +261,33 @@ def set_debug_flags(flags: int) -> None:
     lib().pivot_set_debug_flags(int(flags))
 
 
+class KernelTimer:
+    """Records CUDA events between the library's kernel launches (on the call's
+    stream): times of the scan kernel, the refine kernel and the row select."""
+
+    def __init__(self):
+        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        s = torch.cuda.current_stream()
+        for e in self.ev:
+            e.record(s)  # creates the underlying cudaEvent_t
+        torch.cuda.synchronize()
+        self._arr = (ctypes.c_void_p * 4)(*[e.cuda_event for e in self.ev])
+
+    def __enter__(self):
+        lib().pivot_set_profile_events(self._arr, 4)
+        return self
+
+    def __exit__(self, *exc):
+        lib().pivot_set_profile_events(None, 0)
+
+    def ms(self):
+        """(scan, refine, rowselect) milliseconds of the last call (after a sync)."""
+        e = self.ev
+        return e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])
+
+
 __all__ = [
     "lib", "LIB_PATH", "EXPORTS", "PivotError", "Workspace", "workspace_size", "varlen_workspace_size", "path",
     "indexer_dense", "reuse", "refine", "reuse_varlen", "refine_varlen", "last_device_status",
-    "set_device_timeout_ns", "set_debug_flags", "OP_DENSE", "OP_REUSE", "OP_REFINE", "BF16", "F32", "STATUS",
+    "set_device_timeout_ns", "set_debug_flags", "KernelTimer", "OP_DENSE", "OP_REUSE", "OP_REFINE", "BF16", "F32", "STATUS",
 ]

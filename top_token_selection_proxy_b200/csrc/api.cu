@@ -19,6 +19,14 @@ namespace {
 thread_local char g_cuda_err[256] = "";
 uint64_t g_timeout_ns = 2000000000ull;
 int g_debug_flags = 0;
+cudaEvent_t g_prof[4] = {nullptr, nullptr, nullptr, nullptr};
+
+void prof(int i, cudaStream_t s) {
+  if (g_prof[0]) cudaEventRecord(g_prof[i], s);
+}
+void prof_rest(int from, cudaStream_t s) {
+  for (int i = from; i < 4; ++i) prof(i, s);
+}
 
 constexpr size_t kHdr = 256;     // status word + counters
 constexpr int kStatusOff = 0;    // int
@@ -96,7 +104,10 @@ pivot_status check_common(int64_t L, int H, int d, pivot_dtype dt, int k, int c,
 int sel_size(int op, int k, int c, int g) {
   return op == PIVOT_OP_DENSE ? k : (op == PIVOT_OP_REUSE ? k + g - 1 : c);
 }
-int sel_cap(int n_sel) { return (int)align_up((size_t)2 * n_sel + 256, 256); }
+// per (group, lane quarter) sub-buffer of the scan kernel: room for a full
+// selection plus slack, so that cut-backs are rare; a group owns 4 of them
+int sel_sub_cap(int n_sel) { return (int)align_up((size_t)n_sel + 256, 64); }
+int sel_cap(int n_sel) { return 4 * sel_sub_cap(n_sel); }
 
 struct Carve {
   char* base;
@@ -120,7 +131,7 @@ struct PrefillWs {
   uint64_t* sscratch;
   float* fscratch;
   int grid, simt_grid;
-  int64_t simt_per_block;
+  int64_t simt_per_block, simt_member_off;
   size_t bytes;
 };
 
@@ -146,7 +157,8 @@ PrefillWs carve_prefill(void* base, int op, int64_t L, int H, int d, int k, int 
     }
   } else {
     w.simt_grid = (int)std::min<int64_t>(2 * sms, n_groups);
-    w.simt_per_block = L + (op == PIVOT_OP_REFINE ? c : 0);
+    w.simt_member_off = (int64_t)align_up((size_t)L, 32);
+    w.simt_per_block = w.simt_member_off + (op == PIVOT_OP_REFINE ? (int64_t)align_up((size_t)c, 32) : 0);
     w.sscratch = cv.take<uint64_t>((size_t)(2 * sms) * w.simt_per_block);
     w.fscratch = cv.take<float>((size_t)(2 * sms) * ((size_t)H * d + H));
   }
@@ -168,8 +180,8 @@ struct DecodeWs {
   uint32_t* keys;
   uint64_t* sscratch;
   float* fscratch;
-  int grid, mgrid, simt_grid, n_items;
-  int64_t chunk, simt_per_block;
+  int grid, mgrid, simt_grid, n_items, partial_stride;
+  int64_t chunk, simt_per_block, simt_member_off;
   size_t bytes;
 };
 
@@ -205,16 +217,18 @@ DecodeWs carve_decode(void* base, int op, int B, const int64_t* off, int H, int 
     w.item_s1 = cv.take<int64_t>(items);
     w.seq_item0 = cv.take<int32_t>((size_t)B + 1);
     w.selbuf = cv.take<uint64_t>((size_t)sms * (256 / H) * sel_cap(n_sel));
-    w.partial = cv.take<uint64_t>((size_t)items * n_sel);
+    w.partial_stride = (int)align_up((size_t)n_sel, 32);
+    w.partial = cv.take<uint64_t>((size_t)items * w.partial_stride);
     w.partial_cnt = cv.take<uint32_t>(items);
-    w.mscratch = cv.take<uint64_t>((size_t)w.mgrid * n_sel);
+    w.mscratch = cv.take<uint64_t>((size_t)w.mgrid * w.partial_stride);
     if (op == PIVOT_OP_REFINE) {
       if (!user_cand) w.cand = cv.take<int32_t>((size_t)B * c);
       w.keys = cv.take<uint32_t>((size_t)B * g * c);
     }
   } else {
     w.simt_grid = std::min(B, 2 * sms);
-    w.simt_per_block = pmax + (op == PIVOT_OP_REFINE ? c : 0);
+    w.simt_member_off = (int64_t)align_up((size_t)pmax, 32);
+    w.simt_per_block = w.simt_member_off + (op == PIVOT_OP_REFINE ? (int64_t)align_up((size_t)c, 32) : 0);
     w.sscratch = cv.take<uint64_t>((size_t)(2 * sms) * w.simt_per_block);
     w.fscratch = cv.take<float>((size_t)(2 * sms) * ((size_t)H * d + H));
   }
@@ -246,6 +260,7 @@ ScanArgs scan_base(const void* q, const float* w, int H, int d, int g, int n_sel
   a.n_items = n_items;
   a.selbuf = selbuf;
   a.cap = cap;
+  a.sub_cap = cap / 4;
   a.counter = counter;
   a.status = status;
   a.timeout_ns = g_timeout_ns;
@@ -290,6 +305,7 @@ pivot_status run_prefill(int op, const void* q, const float* w, const void* k_I,
     a.cand_scores = cand_scores;
     a.scratch = W.sscratch;
     a.scratch_per_block = W.simt_per_block;
+    a.member_off = W.simt_member_off;
     a.fscratch = W.fscratch;
     e = launch_simt(a, W.simt_grid, s);
     return e == cudaSuccess ? PIVOT_OK : cuda_fail(e, "simt kernel");
@@ -309,9 +325,14 @@ pivot_status run_prefill(int op, const void* q, const float* w, const void* k_I,
   int32_t* cand = cand_opt ? cand_opt : W.cand;
   a.cand = cand;
   a.cand_scores = cand_scores;
+  prof(0, s);
   e = launch_scan(a, &kmap, W.grid, s);
   if (e != cudaSuccess) return cuda_fail(e, "scan kernel");
-  if (op != PIVOT_OP_REFINE) return PIVOT_OK;
+  prof(1, s);
+  if (op != PIVOT_OP_REFINE) {
+    prof_rest(2, s);
+    return PIVOT_OK;
+  }
 
   RefineArgs r{};
   r.q = reinterpret_cast<const uint16_t*>(q);
@@ -332,8 +353,11 @@ pivot_status run_prefill(int op, const void* q, const float* w, const void* k_I,
   r.counter = W.counters + 1;
   r.status = W.status;
   r.timeout_ns = g_timeout_ns;
-  e = launch_refine(r, nullptr, (int)std::min<int64_t>(num_sms(), r.n_items), s);
+  CUtensorMap gmap;  // one-row boxes for the candidate gather
+  if (!make_kmap(&gmap, k_I, L, d, 1)) return cuda_fail(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+  e = launch_refine(r, &gmap, (int)std::min<int64_t>(num_sms(), r.n_items), s);
   if (e != cudaSuccess) return cuda_fail(e, "refine kernel");
+  prof(2, s);
 
   RowSelArgs rs{};
   rs.keys = W.keys;
@@ -347,7 +371,9 @@ pivot_status run_prefill(int op, const void* q, const float* w, const void* k_I,
   rs.out_idx = indices;
   rs.out_scores = scores;
   e = launch_rowselect(rs, (int)std::min<int64_t>(8 * num_sms(), L), s);
-  return e == cudaSuccess ? PIVOT_OK : cuda_fail(e, "rowselect kernel");
+  if (e != cudaSuccess) return cuda_fail(e, "rowselect kernel");
+  prof(3, s);
+  return PIVOT_OK;
 }
 
 // ---------------------------------------------------------------- decode driver
@@ -388,6 +414,7 @@ pivot_status run_decode(int op, const void* q, const float* w, const void* kc, c
     a.cand_scores = cand_scores;
     a.scratch = W.sscratch;
     a.scratch_per_block = W.simt_per_block;
+    a.member_off = W.simt_member_off;
     a.fscratch = W.fscratch;
     e = launch_simt(a, W.simt_grid, s);
     return e == cudaSuccess ? PIVOT_OK : cuda_fail(e, "simt kernel");
@@ -406,6 +433,7 @@ pivot_status run_decode(int op, const void* q, const float* w, const void* kc, c
   a.item_s0 = W.item_s0;
   a.item_s1 = W.item_s1;
   a.partial = W.partial;
+  a.partial_stride = W.partial_stride;
   a.partial_cnt = W.partial_cnt;
   e = launch_scan(a, &kmap, W.grid, s);
   if (e != cudaSuccess) return cuda_fail(e, "scan kernel");
@@ -416,13 +444,14 @@ pivot_status run_decode(int op, const void* q, const float* w, const void* kc, c
   m.partial_cnt = W.partial_cnt;
   m.seq_item0 = W.seq_item0;
   m.n_sel = n_sel;
+  m.partial_stride = W.partial_stride;
   m.B = B;
   m.g = g;
   m.topk = k;
   m.mode = op == PIVOT_OP_REUSE ? EMIT_REUSE : EMIT_CAND;
   m.key_off = off_dev;
   m.scratch = W.mscratch;
-  m.cap = n_sel;
+  m.cap = W.partial_stride;
   m.cand = cand;
   m.cand_scores = cand_scores;
   m.out_idx = indices;
@@ -450,7 +479,9 @@ pivot_status run_decode(int op, const void* q, const float* w, const void* kc, c
   r.counter = W.counters + 1;
   r.status = W.status;
   r.timeout_ns = g_timeout_ns;
-  e = launch_refine(r, nullptr, std::min(num_sms(), r.n_items), s);
+  CUtensorMap gmap;  // one-row boxes for the candidate gather
+  if (!make_kmap(&gmap, kc, off_host[B], d, 1)) return cuda_fail(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+  e = launch_refine(r, &gmap, std::min(num_sms(), r.n_items), s);
   if (e != cudaSuccess) return cuda_fail(e, "refine kernel");
 
   RowSelArgs rs{};
@@ -563,6 +594,11 @@ int pivot_path(int op, int64_t L, int H, int d, int k, int c, int g, pivot_dtype
 
 void pivot_set_device_timeout_ns(uint64_t ns) { g_timeout_ns = ns; }
 void pivot_set_debug_flags(int flags) { g_debug_flags = flags; }
+
+void pivot_set_profile_events(void** events, int n) {
+  for (int i = 0; i < 4; ++i)
+    g_prof[i] = (events && n >= 4) ? reinterpret_cast<cudaEvent_t>(events[i]) : nullptr;
+}
 int pivot_version(void) { return 100; }
 
 }  // extern "C"

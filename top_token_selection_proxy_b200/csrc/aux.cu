@@ -21,6 +21,7 @@ namespace pivot {
 __global__ void __launch_bounds__(256) rowselect_kernel(const RowSelArgs a) {
   extern __shared__ uint64_t sbuf[];  // c packed entries of the row
   __shared__ SelSmem S;
+  __shared__ uint32_t hist11[2048];
   const Group<256> G{(int)threadIdx.x, 0};
   for (int64_t row = blockIdx.x; row < a.n_rows; row += gridDim.x) {
     const int64_t grp = row / a.g;
@@ -44,7 +45,7 @@ __global__ void __launch_bounds__(256) rowselect_kernel(const RowSelArgs a) {
     group_offsets<256>(nv, &total, S, G);
     G.sync();
     const uint64_t th =
-        (total <= (uint32_t)a.topk) ? 1ull : radix_threshold<256>(sbuf, n_c, a.topk, a.topk, S, G);
+        (total <= (uint32_t)a.topk) ? 1ull : radix11_threshold<256>(sbuf, n_c, a.topk, a.topk, hist11, S, G);
     emit_row<256>(sbuf, n_c, 0xFFFFFFFFu, th - 1ull, a.out_idx + row * a.topk,
                   a.out_scores ? a.out_scores + row * a.topk : nullptr, (uint32_t)a.topk, S, G);
     G.sync();
@@ -93,8 +94,8 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeArgs a) {
   uint64_t* scr = a.scratch + (uint64_t)blockIdx.x * a.cap;
   for (int b = blockIdx.x; b < a.B; b += gridDim.x) {
     const int i0 = a.seq_item0[b], i1 = a.seq_item0[b + 1];
-    const uint64_t* region = a.partial + (uint64_t)i0 * a.n_sel;
-    const uint32_t n = (uint32_t)(i1 - i0) * (uint32_t)a.n_sel;
+    const uint64_t* region = a.partial + (uint64_t)i0 * a.partial_stride;
+    const uint32_t n = (uint32_t)(i1 - i0) * (uint32_t)a.partial_stride;
     uint32_t real = 0;
     for (int i = i0; i < i1; ++i) real += a.partial_cnt[i];
     const uint64_t th = (real <= (uint32_t)a.n_sel) ? 1ull : radix_threshold<256>(region, n, a.n_sel, a.n_sel, S, G);
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(256) simt_kernel(const SimtArgs a) {
   float* qv = a.fscratch + (int64_t)blockIdx.x * (H * D + H);
   float* wv = qv + H * D;
   uint64_t* buf = a.scratch + (int64_t)blockIdx.x * a.scratch_per_block;
-  uint64_t* mb = buf + (a.scratch_per_block - a.c);  // member entries (Refine)
+  uint64_t* mb = buf + a.member_off;  // member entries (Refine)
   for (int64_t grp = blockIdx.x; grp < a.n_groups; grp += gridDim.x) {
     int64_t kbase, P, mrow0, t_first, orow0;
     int nm;

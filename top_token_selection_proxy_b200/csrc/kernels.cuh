@@ -5,7 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include "../../include/pivot.h"
+#include "pivot.h"  // include/ of the repository (-I)
 
 namespace pivot {
 
@@ -39,7 +39,8 @@ struct ScanArgs {
   const int32_t* item_seq;    // [n_items] sequence of each item
   const int64_t* item_s0;     // [n_items] first local key of the chunk
   const int64_t* item_s1;     // [n_items] one past the last local key
-  uint64_t* partial;          // [n_items, n_sel] packed entries (EMIT_PARTIAL)
+  uint64_t* partial;          // [n_items, partial_stride] packed entries (EMIT_PARTIAL)
+  int partial_stride;         // >= n_sel, multiple of 32 (zero padded)
   uint32_t* partial_cnt;      // [n_items]
   // outputs
   int32_t* out_idx;    // [rows, topk]
@@ -47,8 +48,9 @@ struct ScanArgs {
   int32_t* cand;       // [n_groups, n_sel]
   float* cand_scores;  // [n_groups, n_sel] or null
   // workspace
-  uint64_t* selbuf;    // [gridDim.x, nb, cap]
-  int cap;
+  uint64_t* selbuf;    // [gridDim.x, nb, cap]: per group 4 sub-buffers of sub_cap entries
+  int cap;             // = 4 * sub_cap
+  int sub_cap;         // entries per (group, TMEM lane quarter) sub-buffer
   unsigned int* counter;
   int* status;
   uint64_t timeout_ns;
@@ -99,7 +101,8 @@ struct SimtArgs {
   int32_t* cand_out;   // refine: [n_groups, c] or null
   float* cand_scores;
   uint64_t* scratch;   // [gridDim.x, scratch_per_block]
-  int64_t scratch_per_block;
+  int64_t scratch_per_block;  // multiple of 32: prefix scores, then (Refine) the member entries
+  int64_t member_off;         // offset of the member entries in a block's scratch (multiple of 32)
   float* fscratch;     // [gridDim.x, H*D + H] pooled proxy / member query
 };
 
@@ -108,6 +111,7 @@ struct MergeArgs {
   const uint32_t* partial_cnt; // [n_items]
   const int32_t* seq_item0;    // [B+1] first item of each sequence
   int n_sel;                   // c (refine) or k+g-1 (reuse)
+  int partial_stride;          // entries per item in `partial` (>= n_sel, zero padded)
   int B, g, topk, mode;        // mode: EMIT_CAND or EMIT_REUSE
   const int64_t* key_off;      // [B+1]
   uint64_t* scratch;           // [gridDim.x, cap]
@@ -121,7 +125,7 @@ struct MergeArgs {
 // launchers (return cudaError_t of the launch)
 cudaError_t launch_scan(const ScanArgs& a, const CUtensorMap* kmap, int grid, cudaStream_t s);
 size_t scan_smem_bytes(int H, int D);
-cudaError_t launch_refine(const RefineArgs& a, const CUtensorMap* qmap, int grid, cudaStream_t s);
+cudaError_t launch_refine(const RefineArgs& a, const CUtensorMap* gather_kmap, int grid, cudaStream_t s);
 size_t refine_smem_bytes(int H, int D, int mc);
 cudaError_t launch_simt(const SimtArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_merge(const MergeArgs& a, int grid, cudaStream_t s);

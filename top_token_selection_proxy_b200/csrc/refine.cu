@@ -36,8 +36,10 @@ struct RefCfg {
   static constexpr int STAGES = 2;
   static constexpr int A_BYTES = BM * D * 2;
   static constexpr int B_BYTES = NROW * D * 2;
-  static constexpr int THREADS = 256;
-  static constexpr int NPROD = 96;      // gather threads (warps 5-7)
+  static constexpr int THREADS = 320;   // warps 0-7 epilogue, warp 8 MMA, warp 9 TMA gather
+  static constexpr int NEPI = 256;
+  static constexpr int MPH = 256 / H;   // members per accumulator half
+  static constexpr int MPW = MPH / 2;   // members per epilogue warp (two warps per TMEM lane quarter)
 };
 
 struct RefTail {
@@ -57,7 +59,8 @@ constexpr size_t refine_smem() {
 }
 
 template <int H, int D>
-__global__ void __launch_bounds__(256, 1) refine_kernel(const RefineArgs a, uint32_t* __restrict__ out_keys) {
+__global__ void __launch_bounds__(320, 1) refine_kernel(const __grid_constant__ CUtensorMap kmap, const RefineArgs a,
+                                                              uint32_t* __restrict__ out_keys) {
   using C = RefCfg<H, D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -68,17 +71,18 @@ __global__ void __launch_bounds__(256, 1) refine_kernel(const RefineArgs a, uint
 
   if (tid == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&T.full[s], C::NPROD);
+      mbar_init(&T.full[s], 1);
       mbar_init(&T.empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&T.accf[b], 1);
-      mbar_init(&T.acce[b], 128);
+      mbar_init(&T.acce[b], C::NEPI);
     }
     T.abort_flag = 0;
     fence_mbar_init();
+    prefetch_tmap(&kmap);
   }
-  if (warp == 4) {
+  if (warp == 8) {
     tmem_alloc(&T.tmem_slot, 512);
     tmem_relinquish();
   }
@@ -154,47 +158,49 @@ __global__ void __launch_bounds__(256, 1) refine_kernel(const RefineArgs a, uint
       continue;
     }
 
-    if (warp >= 5) {
-      // ------------------------------------------------------------ gather producers
-      const int ptid = tid - 160;
-      constexpr int XC = D / 8;
-      int prev = -1;
-      bool ok = true;
+    if (warp == 9) {
+      // ------------------------------------------------------------ TMA gather producer
+      // lane l gathers candidate rows 4l..4l+3 of each 128-row tile: one 16-byte load of
+      // their ids, then one 4-row gather per 64-column k-block (ids past n_c read row 0;
+      // those slots are masked by the epilogue)
       for (int j = 0; j < ntiles; ++j) {
-        if (!mbar_wait(&T.empty[p_st], p_ph ^ 1u, a.timeout_ns, &T.abort_flag)) {
-          T.abort_flag = 1;
-          atomicOr(a.status, DEV_ERR_TIMEOUT);
-          ok = false;
+        int okw = 1;
+        if (lane == 0) okw = mbar_wait(&T.empty[p_st], p_ph ^ 1u, a.timeout_ns, &T.abort_flag) ? 1 : 0;
+        okw = __shfl_sync(0xFFFFFFFFu, okw, 0);
+        if (!okw) {
+          if (lane == 0) {
+            T.abort_flag = 1;
+            atomicOr(a.status, DEV_ERR_TIMEOUT);
+          }
           break;
         }
-        uint8_t* dst = sA + p_st * C::A_BYTES;
-        for (int u = ptid; u < C::BM * XC; u += C::NPROD) {
-          const int row = u / XC, xc = u % XC;
-          const int slot = j * C::BM + row;
-          const int s = (slot < n_c) ? __ldg(cand + slot) : -1;
-          const bool valid = s >= 0;
-          const uint16_t* src = a.k + (T.key_base + (valid ? s : 0)) * (int64_t)D + xc * 8;
-          const int kb = xc >> 3, ch = xc & 7;
-          cp_async_16_zfill(dst + kb * (C::BM * 128) + row * 128 + ((ch ^ (row & 7)) << 4), src, valid);
+        if (lane == 0) mbar_arrive_expect_tx(&T.full[p_st], C::A_BYTES);
+        __syncwarp();
+        const int slot0 = j * C::BM + 4 * lane;
+        int id[4];
+        if (slot0 + 3 < n_c && (reinterpret_cast<uintptr_t>(cand + slot0) & 15u) == 0) {
+          const int4 v = __ldg(reinterpret_cast<const int4*>(cand + slot0));
+          id[0] = v.x;
+          id[1] = v.y;
+          id[2] = v.z;
+          id[3] = v.w;
+        } else {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) id[u] = (slot0 + u < n_c) ? __ldg(cand + slot0 + u) : -1;
         }
-        cp_async_commit();
-        if (prev >= 0) {
-          cp_async_wait<1>();
-          fence_proxy_async_smem();
-          mbar_arrive(&T.full[prev]);
-        }
-        prev = (int)p_st;
+        int row[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) row[u] = (int)(T.key_base + (id[u] >= 0 ? id[u] : 0));
+        uint8_t* dst = sA + p_st * C::A_BYTES + (4 * lane) * 128;
+#pragma unroll
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_gather4(dst + kb * (C::BM * 128), &kmap, &T.full[p_st], kb * 64, row[0], row[1], row[2], row[3]);
         if (++p_st == C::STAGES) {
           p_st = 0;
           p_ph ^= 1u;
         }
       }
-      cp_async_wait<0>();
-      if (ok && prev >= 0) {
-        fence_proxy_async_smem();
-        mbar_arrive(&T.full[prev]);
-      }
-    } else if (warp == 4) {
+    } else if (warp == 8) {
       // ------------------------------------------------------------ MMA issuer
       if (lane == 0) {
         const uint32_t baddr = smem_u32(sB);
@@ -240,44 +246,54 @@ __global__ void __launch_bounds__(256, 1) refine_kernel(const RefineArgs a, uint
         }
       }
     } else {
-      // ------------------------------------------------------------ epilogue (warps 0-3)
-      const int q4 = warp;  // TMEM lane quarter
+      // ------------------------------------------------------------ epilogue (warps 0-7)
+      // warp w reads TMEM lanes 32*(w%4).. (its candidates); the two warps of a
+      // lane quarter split the members of each accumulator half.
+      const int q4 = warp & 3;
+      const int part = warp >> 2;
       const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
-      constexpr int MPH = 256 / H;  // members per accumulator half
       bool stop = false;
       for (int j = 0; j < ntiles && !stop; ++j) {
         const int slot = j * C::BM + q4 * 32 + lane;
         const int s = (slot < n_c) ? __ldg(cand + slot) : -1;
         for (int h = 0; h < nhalf; ++h) {
           const bool ok = mbar_wait(&T.accf[e_ab], e_aph, a.timeout_ns, &T.abort_flag);
-          float sc[MPH];
+          float sc[C::MPW];
           if (ok) {
             tc_fence_after();
+            uint32_t v[C::MPW][H];
 #pragma unroll
-            for (int ml = 0; ml < MPH; ++ml) {
-              const int r = h * MPH + ml;
-              float part[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int mi = 0; mi < C::MPW; ++mi) {
+              const int ml = part * C::MPW + mi;
+              if (h * C::MPH + ml < nm) {
+#pragma unroll
+                for (int h0 = 0; h0 < H; h0 += 32)
+                  tmem_ld32(tmem + lane_base + e_ab * 256u + (uint32_t)(ml * H + h0),
+                            *reinterpret_cast<uint32_t(*)[32]>(&v[mi][h0]));
+              }
+            }
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&T.acce[e_ab]);  // accumulator copied: the MMA may refill it
+#pragma unroll
+            for (int mi = 0; mi < C::MPW; ++mi) {
+              const int r = h * C::MPH + part * C::MPW + mi;
+              float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
               if (r < nm) {
+                const float4* wv = reinterpret_cast<const float4*>(&T.w[r * H]);
 #pragma unroll
-                for (int h0 = 0; h0 < H; h0 += 32) {
-                  uint32_t v[32];
-                  tmem_ld32(tmem + lane_base + e_ab * 256u + (uint32_t)(ml * H + h0), v);
-                  tmem_wait_ld();
-                  const float4* wv = reinterpret_cast<const float4*>(&T.w[r * H + h0]);
-#pragma unroll
-                  for (int i = 0; i < 8; ++i) {
-                    const float4 w4 = wv[i];
-                    part[0] = fmaf(w4.x, fmaxf(__uint_as_float(v[4 * i + 0]), 0.f), part[0]);
-                    part[1] = fmaf(w4.y, fmaxf(__uint_as_float(v[4 * i + 1]), 0.f), part[1]);
-                    part[2] = fmaf(w4.z, fmaxf(__uint_as_float(v[4 * i + 2]), 0.f), part[2]);
-                    part[3] = fmaf(w4.w, fmaxf(__uint_as_float(v[4 * i + 3]), 0.f), part[3]);
-                  }
+                for (int i = 0; i < H / 4; ++i) {
+                  const float4 w4 = wv[i];
+                  const float2 x0 = make_float2(fmaxf(__uint_as_float(v[mi][4 * i + 0]), 0.f),
+                                                fmaxf(__uint_as_float(v[mi][4 * i + 1]), 0.f));
+                  const float2 x1 = make_float2(fmaxf(__uint_as_float(v[mi][4 * i + 2]), 0.f),
+                                                fmaxf(__uint_as_float(v[mi][4 * i + 3]), 0.f));
+                  acc0 = __ffma2_rn(make_float2(w4.x, w4.y), x0, acc0);
+                  acc1 = __ffma2_rn(make_float2(w4.z, w4.w), x1, acc1);
                 }
               }
-              sc[ml] = (part[0] + part[1]) + (part[2] + part[3]);
+              sc[mi] = (acc0.x + acc0.y) + (acc1.x + acc1.y);
             }
-            tc_fence_before();
-            mbar_arrive(&T.acce[e_ab]);
           } else {
             T.abort_flag = 1;
             atomicOr(a.status, DEV_ERR_TIMEOUT);
@@ -286,19 +302,19 @@ __global__ void __launch_bounds__(256, 1) refine_kernel(const RefineArgs a, uint
             e_ab = 0;
             e_aph ^= 1u;
           }
-          if (named_bar_or(1, 128, T.abort_flag != 0)) {
+          if (!ok) {
             stop = true;
             break;
           }
           // Eq. (8) with the member's causal mask s <= t; key 0 marks "not eligible"
           if (slot < a.c) {
 #pragma unroll
-            for (int ml = 0; ml < MPH; ++ml) {
-              const int r = h * MPH + ml;
+            for (int mi = 0; mi < C::MPW; ++mi) {
+              const int r = h * C::MPH + part * C::MPW + mi;
               if (r < nm) {
                 const int64_t t = T.t0 + r;
                 const bool valid = (s >= 0) && ((int64_t)s <= t);
-                out_keys[(T.orow0 + r) * (int64_t)a.c + slot] = valid ? score_key(sc[ml]) : 0u;
+                out_keys[(T.orow0 + r) * (int64_t)a.c + slot] = valid ? score_key(sc[mi]) : 0u;
               }
             }
           }
@@ -314,7 +330,7 @@ __global__ void __launch_bounds__(256, 1) refine_kernel(const RefineArgs a, uint
     while (globaltimer_ns() - t0 < 200000ull) {
     }
   }
-  if (warp == 4) tmem_dealloc(tmem, 512);
+  if (warp == 8) tmem_dealloc(tmem, 512);
 }
 
 size_t refine_smem_bytes(int H, int D, int /*mc*/) {
@@ -323,17 +339,17 @@ size_t refine_smem_bytes(int H, int D, int /*mc*/) {
   return 0;
 }
 
-cudaError_t launch_refine(const RefineArgs& a, const CUtensorMap* /*qmap*/, int grid, cudaStream_t s) {
+cudaError_t launch_refine(const RefineArgs& a, const CUtensorMap* kmap, int grid, cudaStream_t s) {
   const size_t smem = refine_smem_bytes(a.H, a.D, a.mc);
   uint32_t* keys = a.keys;
   if (a.H == 64 && a.D == 128) {
     auto k = refine_kernel<64, 128>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, 256, smem, s>>>(a, keys);
+    k<<<grid, RefCfg<64, 128>::THREADS, smem, s>>>(*kmap, a, keys);
   } else if (a.H == 64 && a.D == 64) {
     auto k = refine_kernel<64, 64>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, 256, smem, s>>>(a, keys);
+    k<<<grid, RefCfg<64, 64>::THREADS, smem, s>>>(*kmap, a, keys);
   } else {
     return cudaErrorInvalidValue;
   }

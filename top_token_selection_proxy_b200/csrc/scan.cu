@@ -44,9 +44,11 @@ struct ScanCfg {
   static constexpr int STAGES = 4;
   static constexpr int A_BYTES = BM * D * 2;
   static constexpr int B_BYTES = N * D * 2;
-  static constexpr int THREADS = 192;
-  static constexpr int NEPI = 128;
-  static_assert(NB <= 16, "at most 16 groups per item");
+  static constexpr int THREADS = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+  static constexpr int NEPI = 256;
+  static constexpr int GPH = NB / 2;   // groups per epilogue half (two warps share each TMEM lane quarter)
+  static constexpr int SMEM_CAP = STAGES * A_BYTES / 8;  // packed entries the freed stage ring can hold
+  static_assert(NB <= 8 && NB % 2 == 0, "2..8 groups per item");
 };
 
 struct ScanTail {
@@ -59,8 +61,10 @@ struct ScanTail {
   int64_t e[16];      // last member position of each group (causal mask of the proxy)
   int64_t mrow0[16];  // first q row of each group's members
   int nmem[16];
-  uint32_t cnt[16];
-  uint64_t tau[16];
+  uint64_t tau[16];         // running admission threshold of each group (admit packed > tau)
+  uint32_t qcnt[8][4];      // per group, entries in each lane quarter's sub-buffer (published on demand)
+  uint32_t cflags;          // groups whose sub-buffers need a cut-back
+  uint32_t hist11[2048];    // radix-select histogram (11-bit digits)
   uint64_t bot[16];
   uint32_t nbot;
   SelSmem sel;
@@ -75,7 +79,7 @@ constexpr size_t scan_smem() {
 }
 
 template <int H, int D>
-__global__ void __launch_bounds__(192, 1) scan_kernel(const __grid_constant__ CUtensorMap kmap, const ScanArgs a) {
+__global__ void __launch_bounds__(320, 1) scan_kernel(const __grid_constant__ CUtensorMap kmap, const ScanArgs a) {
   using C = ScanCfg<H, D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -112,7 +116,7 @@ __global__ void __launch_bounds__(192, 1) scan_kernel(const __grid_constant__ CU
   uint32_t m_st = 0, m_ph = 0, m_ab = 0, m_aph = 0;     // MMA: ring + accumulator
   uint32_t e_ab = 0, e_aph = 0;                         // epilogue: accumulator
   uint64_t* selbase = a.selbuf + (uint64_t)blockIdx.x * C::NB * (uint64_t)a.cap;
-  const Group<128> EG{tid - 64, 1};
+  const Group<256> EG{tid - 64, 1};
   const bool decode = (a.mode == EMIT_PARTIAL);
 
   for (;;) {
@@ -159,10 +163,8 @@ __global__ void __launch_bounds__(192, 1) scan_kernel(const __grid_constant__ CU
           T.s_end = a.item_s1[item];
         }
         T.ntiles = (int)((T.s_end - T.s_begin + C::BM - 1) / C::BM);
-        for (int b = 0; b < C::NB; ++b) {
-          T.cnt[b] = 0;
-          T.tau[b] = 0;
-        }
+        for (int b = 0; b < C::NB; ++b) T.tau[b] = 0;
+        T.cflags = 0;
       }
     }
     __syncthreads();
@@ -278,12 +280,53 @@ __global__ void __launch_bounds__(192, 1) scan_kernel(const __grid_constant__ CU
       }
     } else {
       // ------------------------------------------------------------ epilogue + select
-      const int q4 = warp & 3;  // TMEM lane quarter this warp may access
+      // warp w reads TMEM lanes 32*(w%4).. (its keys); the two warps of a lane
+      // quarter split the groups: half 0 takes groups [0, GPH), half 1 [GPH, NB).
+      // Each (group, lane quarter) owns a sub-buffer of sub_cap entries that only
+      // its warp appends to, with the count kept in a register.
+      const int q4 = warp & 3;
+      const int half = (warp - 2) >> 2;
       const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
       const uint32_t need = (uint32_t)a.n_sel;
-      const uint32_t cap = (uint32_t)a.cap;
+      const uint32_t gstride = (uint32_t)a.cap;    // 4 sub-buffers per group
+      const uint32_t scap = (uint32_t)a.sub_cap;
+      uint32_t qcnt[C::GPH];
+      uint64_t tau_r[C::GPH];
+      int64_t e_r[C::GPH];  // causal bound of each of this warp's groups
+#pragma unroll
+      for (int gi = 0; gi < C::GPH; ++gi) e_r[gi] = T.e[half * C::GPH + gi];
+
+      const int64_t s_begin = T.s_begin, s_end = T.s_end;
+#pragma unroll
+      for (int gi = 0; gi < C::GPH; ++gi) {
+        qcnt[gi] = 0;
+        tau_r[gi] = 0;
+      }
+      auto seg_of = [&](int b, int q) { return selbase + (uint64_t)b * gstride + (uint64_t)q * scap; };
+      auto publish_counts = [&]() {
+        if (lane == 0)
+#pragma unroll
+          for (int gi = 0; gi < C::GPH; ++gi) T.qcnt[half * C::GPH + gi][q4] = qcnt[gi];
+        EG.sync();
+      };
+      // cut group b back to a superset of its best `need` (keep <= maxk), every warp
+      // of the group compacting its own sub-buffer in place
+      auto cut_back = [&](int b, uint32_t maxk) {
+        Segs sg;
+        sg.cnt = 4;
+        for (int q = 0; q < 4; ++q) {
+          sg.p[q] = seg_of(b, q);
+          sg.n[q] = T.qcnt[b][q];
+        }
+        const uint64_t th = radix11_threshold<256>(sg, need, maxk, T.hist11, T.sel, EG);
+        if (half == b / C::GPH) {
+          const int gi = b % C::GPH;
+          qcnt[gi] = warp_compact_ge(seg_of(b, q4), qcnt[gi], th);
+          if (th > 0) tau_r[gi] = th - 1ull;  // admit x >= th from now on
+        }
+        EG.sync();
+      };
       for (int j = 0; j < ntiles; ++j) {
-        float sc[C::NB];
         bool ok;
         if ((a.debug_flags & 1) && j == 0)
           ok = mbar_wait(&T.never, 0u, a.timeout_ns, &T.abort_flag);  // runs out by design
@@ -293,82 +336,124 @@ __global__ void __launch_bounds__(192, 1) scan_kernel(const __grid_constant__ CU
           T.abort_flag = 1;
           atomicOr(a.status, DEV_ERR_TIMEOUT);
         }
+        float sc[C::GPH];
         if (ok) {
           tc_fence_after();
 #pragma unroll
-          for (int b = 0; b < C::NB; ++b) {
-            float part[4] = {0.f, 0.f, 0.f, 0.f};
+          for (int gi = 0; gi < C::GPH; ++gi) {
+            const int b = half * C::GPH + gi;
+            // w-bar of the group first (shared-memory broadcast loads), then the accumulator row
+            float4 w4[H / 4];
+            const float4* wv = reinterpret_cast<const float4*>(&T.wbar[b * H]);
 #pragma unroll
-            for (int h0 = 0; h0 < H; h0 += 32) {
-              uint32_t r[32];
-              tmem_ld32(tmem + lane_base + e_ab * 256u + (uint32_t)(b * H + h0), r);
-              tmem_wait_ld();
-              const float4* wv = reinterpret_cast<const float4*>(&T.wbar[b * H + h0]);
+            for (int i = 0; i < H / 4; ++i) w4[i] = wv[i];
+            uint32_t r[H];
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float4 w4 = wv[i];
-                part[0] = fmaf(w4.x, fmaxf(__uint_as_float(r[4 * i + 0]), 0.f), part[0]);
-                part[1] = fmaf(w4.y, fmaxf(__uint_as_float(r[4 * i + 1]), 0.f), part[1]);
-                part[2] = fmaf(w4.z, fmaxf(__uint_as_float(r[4 * i + 2]), 0.f), part[2]);
-                part[3] = fmaf(w4.w, fmaxf(__uint_as_float(r[4 * i + 3]), 0.f), part[3]);
-              }
+            for (int h0 = 0; h0 < H; h0 += 32)
+              tmem_ld32(tmem + lane_base + e_ab * 256u + (uint32_t)(b * H + h0),
+                        *reinterpret_cast<uint32_t(*)[32]>(&r[h0]));
+            tmem_wait_ld();
+            if (gi == C::GPH - 1) {
+              tc_fence_before();
+              mbar_arrive(&T.acce[e_ab]);  // this warp's columns are in registers: the MMA may refill
             }
-            sc[b] = (part[0] + part[1]) + (part[2] + part[3]);
+            float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                             make_float2(0.f, 0.f)};
+#pragma unroll
+            for (int i = 0; i < H / 4; ++i) {
+              const float2 x0 = make_float2(fmaxf(__uint_as_float(r[4 * i + 0]), 0.f),
+                                            fmaxf(__uint_as_float(r[4 * i + 1]), 0.f));
+              const float2 x1 = make_float2(fmaxf(__uint_as_float(r[4 * i + 2]), 0.f),
+                                            fmaxf(__uint_as_float(r[4 * i + 3]), 0.f));
+              acc[(2 * i) & 3] = __ffma2_rn(make_float2(w4[i].x, w4[i].y), x0, acc[(2 * i) & 3]);
+              acc[(2 * i + 1) & 3] = __ffma2_rn(make_float2(w4[i].z, w4[i].w), x1, acc[(2 * i + 1) & 3]);
+            }
+            sc[gi] = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
           }
-          tc_fence_before();
-          mbar_arrive(&T.acce[e_ab]);
         }
         if (++e_ab == 2) {
           e_ab = 0;
           e_aph ^= 1u;
         }
-        if (named_bar_or(1, 128, T.abort_flag != 0)) break;  // uniform across the epilogue warps
         // streaming selection: append entries above each group's threshold
-        const int64_t s = T.s_begin + (int64_t)j * C::BM + q4 * 32 + lane;
+        bool near_full = false;
+        if (ok) {
+          const int64_t s = s_begin + (int64_t)j * C::BM + q4 * 32 + lane;
+          const uint32_t lt = lanemask_lt();
 #pragma unroll
-        for (int b = 0; b < C::NB; ++b) {
-          if (b < nb_act) {
-            const bool valid = (s < T.s_end) && (s <= T.e[b]);
-            const uint64_t p = pack_entry(score_key(sc[b]), (uint32_t)s);
-            warp_append(valid && p > T.tau[b], p, selbase + (uint64_t)b * cap, &T.cnt[b]);
+          for (int gi = 0; gi < C::GPH; ++gi) {
+            const int b = half * C::GPH + gi;
+            if (b < nb_act) {
+              const bool valid = (s < s_end) && (s <= e_r[gi]);
+              const uint64_t p = pack_entry(score_key(sc[gi]), (uint32_t)s);
+              const bool pass = valid && p > tau_r[gi];
+              const uint32_t m = __ballot_sync(0xFFFFFFFFu, pass);
+              if (pass) seg_of(b, q4)[qcnt[gi] + __popc(m & lt)] = p;
+              qcnt[gi] += __popc(m);
+              if (qcnt[gi] > scap - 4u * 32u) {  // the next 4 tiles could overflow this sub-buffer
+                near_full = true;
+                if (lane == 0) atomicOr(&T.cflags, 1u << b);
+              }
+            }
           }
         }
-        EG.sync();
-        for (int b = 0; b < nb_act; ++b) {
-          const uint32_t n = T.cnt[b];
-          if (n > cap - 128u) {  // cut back: keep a superset of the best `need`
-            uint64_t* buf = selbase + (uint64_t)b * cap;
-            const uint32_t maxk = need + (cap - 128u - need) / 2u;
-            const uint64_t th = radix_threshold<128>(buf, n, need, maxk, T.sel, EG);
-            const uint32_t m = compact_ge<128>(buf, buf, n, th, T.sel, EG);
-            if (EG.tid == 0) {
-              T.cnt[b] = m;
-              T.tau[b] = th - 1ull;  // admit x >= th from now on
-            }
-            EG.sync();
-          }
+        // consensus every 4 tiles (the same tiles for every epilogue thread, so all of them
+        // execute the same barriers; a thread whose wait ran out fails its next waits fast
+        // and reports the abort here): a warp adds at most 32 entries per tile to a sub-buffer
+        if (((j & 3) == 3 || j + 1 == ntiles) &&
+            named_bar_or(1, C::NEPI, near_full || T.abort_flag != 0)) {  // rare: abort or cut-back
+          if (named_bar_or(1, C::NEPI, T.abort_flag != 0)) break;         // uniform decision
+          const uint32_t flags = T.cflags;
+          publish_counts();
+          for (int b = 0; b < nb_act; ++b)
+            if (flags & (1u << b)) cut_back(b, need + (gstride - need) / 8u);  // usually two passes
+          if (EG.tid == 0) T.cflags = 0;
+          EG.sync();
         }
       }
       // ---------------------------------------------------------------- final exact selection + emit
-      if (!named_bar_or(1, 128, T.abort_flag != 0)) {
+      if (!named_bar_or(1, C::NEPI, T.abort_flag != 0)) {
+        publish_counts();
+        uint64_t* sbuf = reinterpret_cast<uint64_t*>(sA);  // the stage ring is idle now
         for (int b = 0; b < nb_act; ++b) {
-          uint64_t* buf = selbase + (uint64_t)b * cap;
-          const uint32_t n = T.cnt[b];
-          const uint64_t th = radix_threshold<128>(buf, n, need, need, T.sel, EG);
-          const uint32_t m = compact_ge<128>(buf, buf, n, th, T.sel, EG);
+          uint32_t n = T.qcnt[b][0] + T.qcnt[b][1] + T.qcnt[b][2] + T.qcnt[b][3];
+          if (n > (uint32_t)C::SMEM_CAP) {  // rare: cut back to exactly `need` first
+            cut_back(b, need);
+            publish_counts();
+            n = T.qcnt[b][0] + T.qcnt[b][1] + T.qcnt[b][2] + T.qcnt[b][3];
+          }
+          // gather the four sub-buffers into shared memory (each segment starts 16-byte aligned)
+          uint32_t off = 0;
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t nq = T.qcnt[b][q];
+            group_copy<256>(sbuf + off, seg_of(b, q), nq, EG);
+            off += (nq + 1u) & ~1u;
+            if (nq & 1u) {  // pad to keep the next segment aligned: a zero entry sorts below everything
+              if (EG.tid == 0) sbuf[off - 1] = 0ull;
+            }
+          }
+          const uint32_t n_real = n;
+          n = off;
+          EG.sync();
+          uint64_t* buf = sbuf;
+          // keep-all is th = 1, so the zero pads never survive; otherwise the need-th
+          // largest is a real entry (n_real > need)
+          const uint64_t th =
+              (n_real <= need) ? 1ull : radix11_threshold<256>(buf, n, need, need, T.hist11, T.sel, EG);
+          const uint32_t m = compact_ge<256>(buf, buf, n, th, T.sel, EG);
           const int64_t grp = T.grp0 + b;
           if (a.mode == EMIT_DENSE) {
-            emit_row<128>(buf, m, 0xFFFFFFFFu, 0ull, a.out_idx + grp * a.topk,
+            emit_row<256>(buf, m, 0xFFFFFFFFu, 0ull, a.out_idx + grp * a.topk,
                           a.out_scores ? a.out_scores + grp * a.topk : nullptr, (uint32_t)a.topk, T.sel, EG);
           } else if (a.mode == EMIT_CAND) {
-            emit_row<128>(buf, m, 0xFFFFFFFFu, 0ull, a.cand + grp * a.n_sel,
+            emit_row<256>(buf, m, 0xFFFFFFFFu, 0ull, a.cand + grp * a.n_sel,
                           a.cand_scores ? a.cand_scores + grp * a.n_sel : nullptr, need, T.sel, EG);
           } else if (a.mode == EMIT_REUSE) {
-            emit_reuse<128>(buf, m, a.topk, T.mrow0[b], T.nmem[b], T.mrow0[b], a.out_idx, a.out_scores, T.sel,
+            emit_reuse<256>(buf, m, a.topk, T.mrow0[b], T.nmem[b], T.mrow0[b], a.out_idx, a.out_scores, T.sel,
                             T.bot, &T.nbot, EG);
           } else {  // EMIT_PARTIAL: the chunk's exact top-n_sel, zero padded
-            uint64_t* dst = a.partial + (uint64_t)item * need;
-            for (uint32_t i = EG.tid; i < need; i += 128) dst[i] = (i < m) ? buf[i] : 0ull;
+            uint64_t* dst = a.partial + (uint64_t)item * (uint32_t)a.partial_stride;
+            for (uint32_t i = EG.tid; i < (uint32_t)a.partial_stride; i += C::NEPI) dst[i] = (i < m) ? buf[i] : 0ull;
             if (EG.tid == 0) a.partial_cnt[item] = m;
           }
           EG.sync();
@@ -398,11 +483,11 @@ cudaError_t launch_scan(const ScanArgs& a, const CUtensorMap* kmap, int grid, cu
   if (a.H == 64 && a.D == 128) {
     auto k = scan_kernel<64, 128>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, 192, smem, s>>>(*kmap, a);
+    k<<<grid, ScanCfg<64, 128>::THREADS, smem, s>>>(*kmap, a);
   } else if (a.H == 64 && a.D == 64) {
     auto k = scan_kernel<64, 64>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, 192, smem, s>>>(*kmap, a);
+    k<<<grid, ScanCfg<64, 64>::THREADS, smem, s>>>(*kmap, a);
   } else {
     return cudaErrorInvalidValue;
   }

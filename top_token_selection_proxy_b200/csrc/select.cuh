@@ -55,29 +55,141 @@ __device__ __forceinline__ void warp_append(bool pass, uint64_t val, uint64_t* b
   if (pass) buf[base + __popc(m & lanemask_lt())] = val;
 }
 
+// Visit every slot of buf[0..n) (f(x, valid) for x = buf[i]; slots past n
+// come with valid = false) with U loads in flight per thread and a trip count
+// that is the same for all NT threads, so warp-synchronous code (match_any,
+// ballot) may run inside f.  16-byte loads when buf is 16-byte aligned,
+// 8-byte loads otherwise.
+template <int NT, int U, typename F>
+__device__ __forceinline__ void visit_entries(const uint64_t* buf, uint32_t n, const Group<NT>& G, F&& f) {
+  if ((reinterpret_cast<uintptr_t>(buf) & 15u) != 0) {
+    for (uint32_t base = 0; base < n; base += NT * U) {
+      uint64_t v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint32_t i = base + u * NT + G.tid;
+        v[u] = (i < n) ? buf[i] : 0ull;
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) f(v[u], base + u * NT + G.tid < n);
+    }
+    return;
+  }
+  constexpr uint32_t STEP = NT * 2 * U;
+  for (uint32_t base = 0; base < n; base += STEP) {
+    ulonglong2 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t i = base + (u * NT + G.tid) * 2;
+      if (i + 1 < n) {
+        v[u] = *reinterpret_cast<const ulonglong2*>(buf + i);
+      } else {
+        v[u].x = (i < n) ? buf[i] : 0ull;
+        v[u].y = 0ull;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t i = base + (u * NT + G.tid) * 2;
+      f(v[u].x, i < n);
+      f(v[u].y, i + 1 < n);
+    }
+  }
+}
+
+// Warp-aggregated histogram increment (bin >= 256 = skip); whole warp calls.
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin) {
+  const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
+  if (bin < 256u && (int)lane_id() == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+}
+
 // Returns a threshold T such that count{ buf[i] >= T } lies in [need, max_keep]
 // (exactly `need` when max_keep == need).  Requires need <= n.  All NT threads
-// call it and get the same T.  T == 0 keeps everything.
+// call it and get the same T.  T == 0 keeps everything.  hist1 (optional) is
+// the histogram of the top 8 bits of buf[0..n); it saves the first pass.
 template <int NT>
 __device__ uint64_t radix_threshold(const uint64_t* buf, uint32_t n, uint32_t need, uint32_t max_keep,
-                                    SelSmem& S, const Group<NT>& G) {
+                                    SelSmem& S, const Group<NT>& G, const uint32_t* hist1 = nullptr) {
+  if (n <= max_keep) return 0ull;
+  uint64_t prefix = 0;
+  uint32_t above = 0;
+  for (int shift = 56; shift >= 0; shift -= 8) {
+    const uint32_t* hist = S.hist;
+    if (shift == 56 && hist1 != nullptr) {
+      hist = hist1;
+    } else {
+      for (int i = G.tid; i < 256; i += NT) S.hist[i] = 0u;
+      G.sync();
+      visit_entries<NT, 4>(buf, n, G, [&](uint64_t x, bool valid) {
+        const bool match = valid && (shift == 56 || (x >> (shift + 8)) == prefix);
+        hist_add(S.hist, match ? ((uint32_t)(x >> shift) & 255u) : 256u);
+      });
+      G.sync();
+    }
+    if (G.tid < 32) {
+      const int l = G.tid;
+      uint32_t loc[8], sum = 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        loc[u] = hist[255 - 8 * l - u];
+        sum += loc[u];
+      }
+      uint32_t incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (l >= o) incl += v;
+      }
+      const uint32_t excl = incl - sum;
+      if (above + excl < need && need <= above + incl) {
+        uint32_t c = above + excl;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (c + loc[u] >= need) {
+            S.scal[0] = 255u - 8u * l - u;
+            S.scal[1] = c;
+            S.scal[2] = loc[u];
+            break;
+          }
+          c += loc[u];
+        }
+      }
+    }
+    G.sync();
+    const uint32_t digit = S.scal[0];
+    above = S.scal[1];
+    const uint32_t h = S.scal[2];
+    prefix = (prefix << 8) | digit;
+    G.sync();  // everyone has read scal / hist before they are rewritten
+    if (above + h <= max_keep || shift == 0) return prefix << shift;
+  }
+  return prefix;
+}
+
+// Up to 4 disjoint segments of packed entries, read as one set.
+struct Segs {
+  const uint64_t* p[4];
+  uint32_t n[4];
+  int cnt;
+};
+
+// radix_threshold over the union of the segments (no first-digit histogram).
+template <int NT>
+__device__ uint64_t radix_threshold_segs(const Segs& sg, uint32_t need, uint32_t max_keep, SelSmem& S,
+                                         const Group<NT>& G) {
+  uint32_t n = 0;
+  for (int i = 0; i < sg.cnt; ++i) n += sg.n[i];
   if (n <= max_keep) return 0ull;
   uint64_t prefix = 0;
   uint32_t above = 0;
   for (int shift = 56; shift >= 0; shift -= 8) {
     for (int i = G.tid; i < 256; i += NT) S.hist[i] = 0u;
     G.sync();
-    for (uint32_t i0 = 0; i0 < n; i0 += NT) {  // uniform trip count: whole warps stay converged
-      const uint32_t i = i0 + G.tid;
-      uint32_t bin = 256u;  // 256 = not counted
-      if (i < n) {
-        const uint64_t x = buf[i];
-        if (shift == 56 || (x >> (shift + 8)) == prefix) bin = (uint32_t)(x >> shift) & 255u;
-      }
-      // warp-aggregated histogram update: one atomic per distinct bin in the warp
-      const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
-      if (bin < 256u && (int)lane_id() == __ffs(peers) - 1) atomicAdd(&S.hist[bin], (uint32_t)__popc(peers));
-    }
+    for (int sgi = 0; sgi < sg.cnt; ++sgi)
+      visit_entries<NT, 8>(sg.p[sgi], sg.n[sgi], G, [&](uint64_t x, bool valid) {
+        const bool match = valid && (shift == 56 || (x >> (shift + 8)) == prefix);
+        hist_add(S.hist, match ? ((uint32_t)(x >> shift) & 255u) : 256u);
+      });
     G.sync();
     if (G.tid < 32) {
       const int l = G.tid;
@@ -113,9 +225,69 @@ __device__ uint64_t radix_threshold(const uint64_t* buf, uint32_t n, uint32_t ne
     above = S.scal[1];
     const uint32_t h = S.scal[2];
     prefix = (prefix << 8) | digit;
+    G.sync();
     if (above + h <= max_keep || shift == 0) return prefix << shift;
   }
   return prefix;
+}
+
+// One warp keeps the entries >= T of seg[0..n) in place; returns the new count.
+// seg must be 16-byte aligned; 2*V entries per lane are in flight per chunk.
+__device__ __forceinline__ uint32_t warp_compact_ge(uint64_t* seg, uint32_t n, uint64_t T) {
+  constexpr int V = 8;
+  const uint32_t lane = lane_id();
+  const uint32_t lt = lanemask_lt();
+  uint32_t out = 0;
+  for (uint32_t base = 0; base < n; base += 64 * V) {
+    ulonglong2 x[V];
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      const uint32_t i = base + (v * 32 + lane) * 2;
+      if (i + 1 < n) {
+        x[v] = *reinterpret_cast<const ulonglong2*>(seg + i);
+      } else {
+        x[v].x = (i < n) ? seg[i] : 0ull;
+        x[v].y = 0ull;
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      const uint32_t i = base + (v * 32 + lane) * 2;
+      const bool k0 = (i < n) && x[v].x >= T;
+      const bool k1 = (i + 1 < n) && x[v].y >= T;
+      const uint32_t m0 = __ballot_sync(0xFFFFFFFFu, k0);
+      const uint32_t m1 = __ballot_sync(0xFFFFFFFFu, k1);
+      // this lane's two survivors go after the survivors of the lower lanes (order is free)
+      uint32_t pos = out + __popc(m0 & lt) + __popc(m1 & lt);
+      if (k0) seg[pos++] = x[v].x;
+      if (k1) seg[pos] = x[v].y;
+      out += __popc(m0) + __popc(m1);
+    }
+    __syncwarp();
+  }
+  return out;
+}
+
+// Copy src[0..n) to dst (both 16-byte aligned) with the NT threads of a group, 8 entries in flight each.
+template <int NT>
+__device__ __forceinline__ void group_copy(uint64_t* dst, const uint64_t* src, uint32_t n, const Group<NT>& G) {
+  constexpr int U = 4;
+  for (uint32_t base = 0; base < n; base += NT * 2 * U) {
+    ulonglong2 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t i = base + (u * NT + G.tid) * 2;
+      if (i + 1 < n) v[u] = *reinterpret_cast<const ulonglong2*>(src + i);
+      else if (i < n) v[u].x = src[i];
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t i = base + (u * NT + G.tid) * 2;
+      if (i + 1 < n) *reinterpret_cast<ulonglong2*>(dst + i) = v[u];
+      else if (i < n) dst[i] = v[u].x;
+    }
+  }
 }
 
 // Inclusive warp scan of v.
@@ -148,12 +320,93 @@ __device__ __forceinline__ uint32_t group_offsets(uint32_t cnt, uint32_t* total,
   return off + incl - cnt;
 }
 
+// ---------------------------------------------------------------- 11-bit digits
+// Digit widths of the 64-bit packed entry, most significant first.
+__host__ __device__ constexpr int r11_width(int d) { return d < 5 ? 11 : 9; }
+__host__ __device__ constexpr int r11_shift(int d) { return 64 - 11 * (d + 1) < 0 ? 0 : 64 - 11 * (d + 1); }
+
+// Like radix_threshold, with 11-bit digits (at most 6 passes, usually 2) and a
+// 2048-bin shared-memory histogram `hist` updated with plain atomics.  The
+// entries are the union of the segments of sg.
+template <int NT>
+__device__ uint64_t radix11_threshold(const Segs& sg, uint32_t need, uint32_t max_keep, uint32_t* hist,
+                                      SelSmem& S, const Group<NT>& G) {
+  static_assert(2048 % NT == 0, "NT must divide 2048");
+  constexpr int BPT = 2048 / NT;  // bins per thread in the digit search
+  uint32_t n = 0;
+  for (int i = 0; i < sg.cnt; ++i) n += sg.n[i];
+  if (n <= max_keep) return 0ull;
+  uint64_t prefix = 0;
+  uint32_t above = 0;
+  int consumed = 0;
+  for (int d = 0; d < 6; ++d) {
+    const int w = r11_width(d), shift = r11_shift(d);
+    const uint32_t nb = 1u << w;
+    for (uint32_t i = G.tid; i < 2048; i += NT) hist[i] = 0u;
+    G.sync();
+    for (int sgi = 0; sgi < sg.cnt; ++sgi)
+      visit_entries<NT, 8>(sg.p[sgi], sg.n[sgi], G, [&](uint64_t x, bool valid) {
+        if (valid && (consumed == 0 || (x >> (64 - consumed)) == prefix))
+          atomicAdd(&hist[(uint32_t)(x >> shift) & (nb - 1u)], 1u);
+      });
+    G.sync();
+    // thread t owns bins [nb-1 - BPT*t - (BPT-1), nb-1 - BPT*t] (descending); bins >= nb are empty
+    uint32_t loc[BPT], sum = 0;
+#pragma unroll
+    for (int u = 0; u < BPT; ++u) {
+      const int bin = 2047 - BPT * G.tid - u - (2048 - (int)nb);
+      loc[u] = (bin >= 0) ? hist[bin] : 0u;
+      sum += loc[u];
+    }
+    uint32_t total;
+    const uint32_t excl = group_offsets<NT>(sum, &total, S, G);
+    if (above + excl < need && need <= above + excl + sum) {
+      uint32_t c = above + excl;
+#pragma unroll
+      for (int u = 0; u < BPT; ++u) {
+        if (c + loc[u] >= need) {
+          S.scal[0] = (uint32_t)(2047 - BPT * G.tid - u - (2048 - (int)nb));
+          S.scal[1] = c;
+          S.scal[2] = loc[u];
+          break;
+        }
+        c += loc[u];
+      }
+    }
+    G.sync();
+    const uint32_t digit = S.scal[0];
+    above = S.scal[1];
+    const uint32_t h = S.scal[2];
+    prefix = (prefix << w) | digit;
+    consumed += w;
+    G.sync();
+    if (above + h <= max_keep || shift == 0) return prefix << shift;
+  }
+  return prefix;
+}
+
+template <int NT>
+__device__ __forceinline__ uint64_t radix11_threshold(const uint64_t* buf, uint32_t n, uint32_t need,
+                                                      uint32_t max_keep, uint32_t* hist, SelSmem& S,
+                                                      const Group<NT>& G) {
+  Segs sg;
+  sg.cnt = 1;
+  sg.p[0] = buf;
+  sg.n[0] = n;
+  return radix11_threshold<NT>(sg, need, max_keep, hist, S, G);
+}
+
 // Stream-compact the entries >= T of src[0..n) into dst[0..m) (dst may be
 // src: every chunk is fully read before any of its survivors is written, and
-// survivors never move forward).  Returns m.
-template <int NT, int V = 4>
+// survivors never move forward).  Returns m.  When hist1 is given it is
+// rebuilt as the top-8-bit histogram of the survivors.
+template <int NT, int V = 8>
 __device__ uint32_t compact_ge(const uint64_t* src, uint64_t* dst, uint32_t n, uint64_t T, SelSmem& S,
-                               const Group<NT>& G) {
+                               const Group<NT>& G, uint32_t* hist1 = nullptr) {
+  if (hist1) {
+    for (int i = G.tid; i < 256; i += NT) hist1[i] = 0u;
+    G.sync();
+  }
   uint32_t base = 0;
   for (uint32_t c0 = 0; c0 < n; c0 += NT * V) {
     uint64_t x[V];
@@ -162,9 +415,14 @@ __device__ uint32_t compact_ge(const uint64_t* src, uint64_t* dst, uint32_t n, u
     for (int v = 0; v < V; ++v) {
       const uint32_t i = c0 + v * NT + G.tid;
       x[v] = (i < n) ? src[i] : 0ull;
+    }
+#pragma unroll
+    for (int v = 0; v < V; ++v) {
+      const uint32_t i = c0 + v * NT + G.tid;
       const bool k = (i < n) && (x[v] >= T);
       keep |= (k ? 1u : 0u) << v;
       cnt += k ? 1u : 0u;
+      if (hist1) hist_add(hist1, k ? (uint32_t)(x[v] >> 56) : 256u);
     }
     uint32_t total;
     uint32_t pos = base + group_offsets<NT>(cnt, &total, S, G);

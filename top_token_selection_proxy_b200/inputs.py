@@ -9,14 +9,17 @@ summary, "Key observations", O1 and O3): keys with a long-tailed score
 profile, and queries that change slowly along the sequence so that
 neighbouring queries pick overlapping keys.
 
-Recipe (all numpy ``Generator(PCG64(seed))``, drawn in this order):
+Recipe (numpy ``PCG64`` generators seeded from ``SeedSequence(seed).spawn``,
+one child stream per item below, so that chunks can be drawn in parallel
+threads and the result does not depend on the thread count):
 
 * ``u``: one random unit vector in R^d shared by all heavy keys.
 * keys ``k_s ~ N(0, I/d)``; a subset of ``round(heavy * L)`` positions, drawn
   without replacement, gets ``k_s += 3 u`` (a shift of norm 3).
 * queries, per head, AR(1) along t: ``q_0 = e_0``,
-  ``q_t = rho q_{t-1} + e_t`` with innovations ``e_t ~ N(0, I/d)``; drawn in
-  t-chunks so the host never holds more than one chunk in float64.
+  ``q_t = rho q_{t-1} + e_t`` with innovations ``e_t ~ N(0, I/d)`` (float32),
+  drawn in t-chunks of 8192 rows; each chunk is filtered from a zero state and
+  then carried: ``q_t += rho^(t - t0 + 1) q_{t0 - 1}``.
 * ``w ~ N(0, 1/H)`` i.i.d. per (t, head).
 * bf16 tensors are rounded to nearest-even from float32 (torch CPU cast) and
   handed around as uint16 bit patterns.
@@ -30,7 +33,7 @@ plus ``N(0, 0.1^2/d)`` noise, and every draft row repeats the current row's w.
 from __future__ import annotations
 
 import dataclasses
-from typing import Optional
+import os
 
 import numpy as np
 
@@ -113,11 +116,11 @@ def _cast(x: np.ndarray, dtype: str) -> np.ndarray:
 
 
 def _keys(rng: np.random.Generator, n: int, d: int, heavy: float, u: np.ndarray) -> np.ndarray:
-    k = rng.standard_normal((n, d)) / np.sqrt(d)
+    k = rng.standard_normal((n, d), dtype=np.float32) * np.float32(1.0 / np.sqrt(d))
     nh = int(round(heavy * n))
     if nh > 0:
         pos = rng.choice(n, size=nh, replace=False)
-        k[pos] += 3.0 * u
+        k[pos] += (3.0 * u).astype(np.float32)
     return k
 
 
@@ -126,43 +129,80 @@ def _unit(rng: np.random.Generator, d: int) -> np.ndarray:
     return u / np.linalg.norm(u)
 
 
+def _threads() -> int:
+    try:
+        return max(1, min(16, len(os.sched_getaffinity(0))))
+    except AttributeError:  # pragma: no cover
+        return 4
+
+
+def _ar1_chunk(seed: np.random.SeedSequence, n: int, H: int, d: int, rho: float) -> np.ndarray:
+    """Zero-state AR(1) of n rows of N(0, I/d) innovations (float32)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    e = rng.standard_normal((n, H, d), dtype=np.float32) * np.float32(1.0 / np.sqrt(d))
+    r = np.float32(rho)
+    for t in range(1, n):
+        e[t] += r * e[t - 1]
+    return e
+
+
 def make_prefill(spec: PrefillSpec, chunk: int = 8192) -> dict:
     """q [L,H,d], w [L,H] float32, k [L,d]; q/k as bf16 bits or float32."""
-    from scipy.signal import lfilter
+    from concurrent.futures import ThreadPoolExecutor
 
-    rng = np.random.Generator(np.random.PCG64(spec.seed))
     L, H, d = spec.L, spec.H, spec.d
-    u = _unit(rng, d)
-    k = _cast(_keys(rng, L, d, spec.heavy, u), spec.dtype)
+    n_chunks = (L + chunk - 1) // chunk
+    ss = np.random.SeedSequence(spec.seed).spawn(3 + n_chunks)
+    u = _unit(np.random.Generator(np.random.PCG64(ss[0])), d)
+    k = _cast(_keys(np.random.Generator(np.random.PCG64(ss[1])), L, d, spec.heavy, u), spec.dtype)
+    w = (np.random.Generator(np.random.PCG64(ss[2])).standard_normal((L, H), dtype=np.float32)
+         * np.float32(1.0 / np.sqrt(H)))
     qdt = np.uint16 if spec.dtype == BF16 else np.float32
     q = np.empty((L, H, d), dtype=qdt)
-    zi = np.zeros((1, H, d))
-    for t0 in range(0, L, chunk):
-        t1 = min(L, t0 + chunk)
-        eps = rng.standard_normal((t1 - t0, H, d)) / np.sqrt(d)
-        y, zi = lfilter([1.0], [1.0, -spec.rho], eps, axis=0, zi=zi)
-        q[t0:t1] = _cast(y, spec.dtype)
-    w = (rng.standard_normal((L, H)) / np.sqrt(H)).astype(np.float32)
+    bounds = [(c * chunk, min(L, c * chunk + chunk)) for c in range(n_chunks)]
+    with ThreadPoolExecutor(_threads()) as ex:
+        parts = list(ex.map(lambda c: _ar1_chunk(ss[3 + c], bounds[c][1] - bounds[c][0], H, d, spec.rho),
+                            range(n_chunks)))
+    prev = None
+    r = np.float32(spec.rho)
+    for c, (t0, t1) in enumerate(bounds):
+        z = parts[c]
+        if prev is not None:  # carry the state of the previous chunk: + rho^(i+1) * q_{t0-1}
+            powers = r ** np.arange(1, t1 - t0 + 1, dtype=np.float32)
+            z += powers[:, None, None] * prev[None]
+        prev = z[-1].copy()
+        q[t0:t1] = _cast(z, spec.dtype)
+        parts[c] = None
     return {"q": q, "w": w, "k": k, "spec": spec}
 
 
 def make_decode(spec: DecodeSpec) -> dict:
     """q [B*g,H,d], w [B*g,H], k_cache [sum P_b, d], offsets [B+1] int64."""
-    rng = np.random.Generator(np.random.PCG64(spec.seed))
+    from concurrent.futures import ThreadPoolExecutor
+
     B, H, d, g = spec.B, spec.H, spec.d, spec.g
-    u = _unit(rng, d)
-    P = rng.integers(spec.p_lo, spec.p_hi, size=B, endpoint=True).astype(np.int64)
+    ss = np.random.SeedSequence(spec.seed).spawn(5 + B)
+    u = _unit(np.random.Generator(np.random.PCG64(ss[0])), d)
+    P = np.random.Generator(np.random.PCG64(ss[1])).integers(spec.p_lo, spec.p_hi, size=B,
+                                                              endpoint=True).astype(np.int64)
     off = np.zeros(B + 1, dtype=np.int64)
     off[1:] = np.cumsum(P)
     kdt = np.uint16 if spec.dtype == BF16 else np.float32
     kc = np.empty((int(off[-1]), d), dtype=kdt)
-    for b in range(B):
+
+    def fill(b):
+        rng = np.random.Generator(np.random.PCG64(ss[5 + b]))
         kc[off[b]:off[b + 1]] = _cast(_keys(rng, int(P[b]), d, spec.heavy, u), spec.dtype)
+
+    with ThreadPoolExecutor(_threads()) as ex:
+        list(ex.map(fill, range(B)))
+    rq = np.random.Generator(np.random.PCG64(ss[2]))
     scale = 1.0 / np.sqrt(d * (1.0 - spec.rho ** 2))
-    cur = rng.standard_normal((B, 1, H, d)) * scale
-    drafts = cur + rng.standard_normal((B, g - 1, H, d)) * (spec.draft_sigma / np.sqrt(d))
+    cur = rq.standard_normal((B, 1, H, d)) * scale
+    drafts = cur + np.random.Generator(np.random.PCG64(ss[3])).standard_normal((B, g - 1, H, d)) * (
+        spec.draft_sigma / np.sqrt(d))
     q = _cast(np.concatenate([cur, drafts], axis=1).reshape(B * g, H, d), spec.dtype)
-    wc = (rng.standard_normal((B, 1, H)) / np.sqrt(H)).astype(np.float32)
+    wc = (np.random.Generator(np.random.PCG64(ss[4])).standard_normal((B, 1, H)) / np.sqrt(H)).astype(np.float32)
     w = np.ascontiguousarray(np.repeat(wc, g, axis=1).reshape(B * g, H))
     return {"q": q, "w": w, "k": kc, "offsets": off, "spec": spec}
 
