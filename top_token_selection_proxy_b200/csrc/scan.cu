@@ -406,7 +406,9 @@ __global__ void __launch_bounds__(320, 1) scan_kernel(const __grid_constant__ CU
           const uint32_t flags = T.cflags;
           publish_counts();
           for (int b = 0; b < nb_act; ++b)
-            if (flags & (1u << b)) cut_back(b, need + (gstride - need) / 8u);  // usually two passes
+            // keep at most sub_cap - 128 in total (>= need + 128 since sub_cap >= need + 256):
+            // then every sub-buffer has room for the 4 tiles until the next consensus
+            if (flags & (1u << b)) cut_back(b, scap - 128u);
           if (EG.tid == 0) T.cflags = 0;
           EG.sync();
         }
