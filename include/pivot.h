@@ -165,6 +165,28 @@ PIVOT_API void pivot_set_debug_flags(int flags);
  * Pass NULL to stop.  Not thread-safe; a process-wide setting. */
 PIVOT_API void pivot_set_profile_events(void **events, int n);
 
+/* PIVOT-Reuse without a workspace (the pages describing PIVOT have no
+ * counterpart of this; it is an integration convenience).  For callers that
+ * cannot allocate device memory, e.g. whose device memory belongs to a pool
+ * or memory planner they do not control, so they can neither call cudaMalloc
+ * nor hand over a workspace.  Computes exactly what pivot_reuse computes,
+ * with the same arguments minus the workspace, on the tensor-core scan
+ * kernel; its scratch (status word, work counter, candidate buffers) is a
+ * fixed static device array of 8 MiB + 256 B that every process loading this
+ * library holds on every device it uses until exit.
+ * Limits: bf16 q/k, H = 64, d in {64, 128}, g <= 16 and k + g - 1 <= 256;
+ * larger sizes return PIVOT_ERR_UNSUPPORTED_SHAPE without launching.
+ * The first call on a device looks the array's device address up (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's
+ * contents: calls that overlap on the GPU (other streams, other host
+ * threads) race and give undefined results, so order them.  Device-side
+ * wait timeouts of this variant are not reported (there is no workspace for
+ * pivot_last_device_status to read).  Allocates nothing. */
+PIVOT_API pivot_status pivot_reuse_noalloc(const void *q_I, const float *w_I, const void *k_I, int64_t L, int H,
+                                           int d, pivot_dtype dt, int k, int g, int32_t *indices, float *scores_opt,
+                                           pivot_stream_t stream);
+
 PIVOT_API int pivot_version(void); /* 100 * major + minor */
 
 #ifdef __cplusplus

@@ -41,6 +41,7 @@ EXPORTS = (
     "pivot_varlen_workspace_size", "pivot_reuse_varlen", "pivot_refine_varlen",
     "pivot_last_device_status", "pivot_status_string", "pivot_last_cuda_error", "pivot_path",
     "pivot_set_device_timeout_ns", "pivot_set_debug_flags", "pivot_set_profile_events", "pivot_version",
+    "pivot_reuse_noalloc",
 )
 
 
