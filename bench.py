@@ -44,7 +44,33 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--no-extras", action="store_true", help="skip dense/Reuse/decode side measurements")
+    p.add_argument("--profile-case", type=int, default=0, metavar="L",
+                   help="profiling run: two PIVOT-Refine calls at sequence length L (H_I=64, d=128, k=2048, "
+                        "c=4096, g=8) and exit; no timing, no JSON")
     return p.parse_args()
+
+
+def run_profile_case(L):
+    """Small case for ncu captures: a warm-up call, then the captured call."""
+    import numpy as np
+    import torch
+
+    import top_token_selection_proxy_b200 as P
+    from top_token_selection_proxy_b200 import build, inputs
+
+    build.build()
+    spec = inputs.PrefillSpec(f"profile_L{L}", L=L, H=64, d=128, k=2048, c=4096, g=8, seed=5)
+    x = inputs.make_prefill(spec)
+    dev = torch.device("cuda", 0)
+    q, w, k = to_dev(x["q"], dev), to_dev(x["w"], dev), to_dev(x["k"], dev)
+    ws = P.Workspace(dev)
+    for _ in range(2):
+        P.refine(q, w, k, spec.k, spec.c, spec.g, ws=ws)
+    torch.cuda.synchronize()
+    st = P.last_device_status(ws)
+    print(f"profile case L={L}: status {P.STATUS.get(st, st)}")
+    if st != 0:
+        raise SystemExit(1)
 
 
 def peaks():
@@ -136,7 +162,7 @@ def to_dev(a, dev):
     return torch.from_numpy(a).to(dev)
 
 
-def cpu_oracle_sample(x, spec, runs=4):
+def cpu_oracle_sample(x, spec, runs=24):
     """Oracle PIVOT-Refine on `runs` contiguous runs of groups spread over the
     sequence (one group per host thread each), so the sampled prefix lengths
     average those of the full workload.  Returns (rows/s, cores, description)."""
@@ -204,6 +230,9 @@ def run_reference(args):
 
 def main():
     args = parse()
+    if args.profile_case:
+        run_profile_case(args.profile_case)
+        return
     if args.impl == "reference":
         run_reference(args)
         return
