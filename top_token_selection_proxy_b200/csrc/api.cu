@@ -353,9 +353,10 @@ pivot_status run_prefill(int op, const void* q, const float* w, const void* k_I,
   r.counter = W.counters + 1;
   r.status = W.status;
   r.timeout_ns = g_timeout_ns;
-  CUtensorMap gmap;  // one-row boxes for the candidate gather
-  if (!make_kmap(&gmap, k_I, L, d, 1)) return cuda_fail(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
-  e = launch_refine(r, &gmap, (int)std::min<int64_t>(num_sms(), r.n_items), s);
+  CUtensorMap gmap, qmap;  // one-row boxes for the candidate gather; 256-row boxes of q rows
+  if (!make_kmap(&gmap, k_I, L, d, 1) || !make_kmap(&qmap, q, L * H, d, 256))
+    return cuda_fail(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+  e = launch_refine(r, &gmap, &qmap, (int)std::min<int64_t>(num_sms(), r.n_items), s);
   if (e != cudaSuccess) return cuda_fail(e, "refine kernel");
   prof(2, s);
 
@@ -479,9 +480,10 @@ pivot_status run_decode(int op, const void* q, const float* w, const void* kc, c
   r.counter = W.counters + 1;
   r.status = W.status;
   r.timeout_ns = g_timeout_ns;
-  CUtensorMap gmap;  // one-row boxes for the candidate gather
-  if (!make_kmap(&gmap, kc, off_host[B], d, 1)) return cuda_fail(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
-  e = launch_refine(r, &gmap, std::min(num_sms(), r.n_items), s);
+  CUtensorMap gmap, qmap;  // one-row boxes for the candidate gather; 256-row boxes of q rows
+  if (!make_kmap(&gmap, kc, off_host[B], d, 1) || !make_kmap(&qmap, q, (int64_t)B * g * H, d, 256))
+    return cuda_fail(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+  e = launch_refine(r, &gmap, &qmap, std::min(num_sms(), r.n_items), s);
   if (e != cudaSuccess) return cuda_fail(e, "refine kernel");
 
   RowSelArgs rs{};

@@ -125,7 +125,8 @@ struct MergeArgs {
 // launchers (return cudaError_t of the launch)
 cudaError_t launch_scan(const ScanArgs& a, const CUtensorMap* kmap, int grid, cudaStream_t s);
 size_t scan_smem_bytes(int H, int D);
-cudaError_t launch_refine(const RefineArgs& a, const CUtensorMap* gather_kmap, int grid, cudaStream_t s);
+cudaError_t launch_refine(const RefineArgs& a, const CUtensorMap* gather_kmap, const CUtensorMap* qmap, int grid,
+                          cudaStream_t s);
 size_t refine_smem_bytes(int H, int D, int mc);
 cudaError_t launch_simt(const SimtArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_merge(const MergeArgs& a, int grid, cudaStream_t s);

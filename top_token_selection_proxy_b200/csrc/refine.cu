@@ -33,7 +33,7 @@ struct RefCfg {
   static constexpr int MC = NROW / H;   // members per item
   static constexpr int KB = D / 64;
   static constexpr int BM = 128;
-  static constexpr int STAGES = 2;
+  static constexpr int STAGES = 3;
   static constexpr int A_BYTES = BM * D * 2;
   static constexpr int B_BYTES = NROW * D * 2;
   static constexpr int THREADS = 320;   // warps 0-7 epilogue, warp 8 MMA, warp 9 TMA gather
@@ -43,7 +43,8 @@ struct RefCfg {
 };
 
 struct RefTail {
-  uint64_t full[2], empty[2], accf[2], acce[2];
+  uint64_t full[3], empty[3], accf[2], acce[2];
+  uint64_t bfull;  // members' q rows (B operand) landed
   uint32_t tmem_slot;
   int item, nm, ntiles, nhalf, n_c;
   volatile int abort_flag;
@@ -55,15 +56,22 @@ static_assert(offsetof(RefTail, w) % 16 == 0, "w must be 16-byte aligned");
 template <int H, int D>
 constexpr size_t refine_smem() {
   using C = RefCfg<H, D>;
-  return 1024 + C::B_BYTES + C::STAGES * C::A_BYTES + sizeof(RefTail);
+  return C::B_BYTES + C::STAGES * C::A_BYTES + sizeof(RefTail);  // base must be 1024-aligned (checked)
 }
 
 template <int H, int D>
-__global__ void __launch_bounds__(320, 1) refine_kernel(const __grid_constant__ CUtensorMap kmap, const RefineArgs a,
+__global__ void __launch_bounds__(320, 1) refine_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                              const __grid_constant__ CUtensorMap qmap, const RefineArgs a,
                                                               uint32_t* __restrict__ out_keys) {
   using C = RefCfg<H, D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // the 128-byte-swizzled operands need a 1024-byte aligned base; there is no
+  // room for alignment slack next to a 3-stage ring, so refuse to run otherwise
+  if ((smem_u32(smem_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicOr(a.status, DEV_ERR_BOUNDS);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint8_t* sB = smem;
   uint8_t* sA = smem + C::B_BYTES;
   RefTail& T = *reinterpret_cast<RefTail*>(smem + C::B_BYTES + C::STAGES * C::A_BYTES);
@@ -78,9 +86,11 @@ __global__ void __launch_bounds__(320, 1) refine_kernel(const __grid_constant__ 
       mbar_init(&T.accf[b], 1);
       mbar_init(&T.acce[b], C::NEPI);
     }
+    mbar_init(&T.bfull, 1);
     T.abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&kmap);
+    prefetch_tmap(&qmap);
   }
   if (warp == 8) {
     tmem_alloc(&T.tmem_slot, 512);
@@ -94,6 +104,7 @@ __global__ void __launch_bounds__(320, 1) refine_kernel(const __grid_constant__ 
   uint32_t p_st = 0, p_ph = 0;
   uint32_t m_st = 0, m_ph = 0, m_ab = 0, m_aph = 0;
   uint32_t e_ab = 0, e_aph = 0;
+  uint32_t b_ph = 0;  // phase of bfull (one completion per item)
   const int chunks = (a.g + C::MC - 1) / C::MC;
   const bool decode = (a.key_off != nullptr);
 
@@ -137,33 +148,51 @@ __global__ void __launch_bounds__(320, 1) refine_kernel(const __grid_constant__ 
     const int nm = T.nm, ntiles = T.ntiles, nhalf = T.nhalf, n_c = T.n_c;
     const int32_t* cand = a.cand + T.grp * (int64_t)a.c;
 
-    // ---------------------------------------------------------------- members' q rows -> B, w -> smem
-    {
-      constexpr int XC = D / 8;
-      const int units = nm * H * XC;
-      for (int u = tid; u < units; u += C::THREADS) {
-        const int xc = u % XC;
-        const int n = u / XC;  // = member * H + head
-        const uint4 v =
-            __ldg(reinterpret_cast<const uint4*>(a.q + (T.qrow0 * H + n) * (int64_t)D) + xc);
-        const int kb = xc >> 3, ch = xc & 7;
-        *reinterpret_cast<uint4*>(sB + kb * (C::NROW * 128) + n * 128 + ((ch ^ (n & 7)) << 4)) = v;
-      }
-      for (int u = tid; u < nm * H; u += C::THREADS) T.w[u] = __ldg(a.w + T.qrow0 * H + u);
+    // ---------------------------------------------------------------- members' q rows -> B (TMA), w -> smem
+    // B rows n = member * H + head are rows qrow0*H + n of q viewed as [rows*H, D]; boxes of
+    // 256 rows x 64 columns (rows past the item's members are loaded but not multiplied)
+    if (tid == 0 && nm > 0 && ntiles > 0) {
+      const int nhb = (nm * H + 255) / 256;
+      mbar_arrive_expect_tx(&T.bfull, (uint32_t)(nhb * C::KB * 256 * 128));
+      for (int hb = 0; hb < nhb; ++hb)
+        for (int kb = 0; kb < C::KB; ++kb)
+          tma_load_2d(sB + kb * (C::NROW * 128) + hb * 256 * 128, &qmap, &T.bfull, kb * 64,
+                      (int)(T.qrow0 * H + hb * 256));
     }
+    for (int u = tid; u < nm * H; u += C::THREADS) T.w[u] = __ldg(a.w + T.qrow0 * H + u);
     fence_proxy_async_smem();
     __syncthreads();
     if (nm == 0 || ntiles == 0) {
       __syncthreads();
       continue;
     }
+    const uint32_t b_ph_item = b_ph;
+    b_ph ^= 1u;
+    (void)b_ph_item;
 
     if (warp == 9) {
       // ------------------------------------------------------------ TMA gather producer
       // lane l gathers candidate rows 4l..4l+3 of each 128-row tile: one 16-byte load of
       // their ids, then one 4-row gather per 64-column k-block (ids past n_c read row 0;
       // those slots are masked by the epilogue)
+      auto load_ids = [&](int j, int (&id)[4]) {
+        const int slot0 = j * C::BM + 4 * lane;
+        if (slot0 + 3 < n_c && (reinterpret_cast<uintptr_t>(cand + slot0) & 15u) == 0) {
+          const int4 v = __ldg(reinterpret_cast<const int4*>(cand + slot0));
+          id[0] = v.x;
+          id[1] = v.y;
+          id[2] = v.z;
+          id[3] = v.w;
+        } else {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) id[u] = (slot0 + u < n_c) ? __ldg(cand + slot0 + u) : -1;
+        }
+      };
+      int idn[4];
+      load_ids(0, idn);  // ids of the next tile are loaded one tile ahead
       for (int j = 0; j < ntiles; ++j) {
+        int id[4] = {idn[0], idn[1], idn[2], idn[3]};
+        if (j + 1 < ntiles) load_ids(j + 1, idn);
         int okw = 1;
         if (lane == 0) okw = mbar_wait(&T.empty[p_st], p_ph ^ 1u, a.timeout_ns, &T.abort_flag) ? 1 : 0;
         okw = __shfl_sync(0xFFFFFFFFu, okw, 0);
@@ -176,18 +205,6 @@ __global__ void __launch_bounds__(320, 1) refine_kernel(const __grid_constant__ 
         }
         if (lane == 0) mbar_arrive_expect_tx(&T.full[p_st], C::A_BYTES);
         __syncwarp();
-        const int slot0 = j * C::BM + 4 * lane;
-        int id[4];
-        if (slot0 + 3 < n_c && (reinterpret_cast<uintptr_t>(cand + slot0) & 15u) == 0) {
-          const int4 v = __ldg(reinterpret_cast<const int4*>(cand + slot0));
-          id[0] = v.x;
-          id[1] = v.y;
-          id[2] = v.z;
-          id[3] = v.w;
-        } else {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) id[u] = (slot0 + u < n_c) ? __ldg(cand + slot0 + u) : -1;
-        }
         int row[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) row[u] = (int)(T.key_base + (id[u] >= 0 ? id[u] : 0));
@@ -204,7 +221,12 @@ __global__ void __launch_bounds__(320, 1) refine_kernel(const __grid_constant__ 
       // ------------------------------------------------------------ MMA issuer
       if (lane == 0) {
         const uint32_t baddr = smem_u32(sB);
-        for (int j = 0; j < ntiles; ++j) {
+        const bool bok = mbar_wait(&T.bfull, b_ph ^ 1u, a.timeout_ns, &T.abort_flag);  // this item's phase
+        if (!bok) {
+          T.abort_flag = 1;
+          atomicOr(a.status, DEV_ERR_TIMEOUT);
+        }
+        for (int j = 0; j < ntiles && bok; ++j) {
           if (!mbar_wait(&T.full[m_st], m_ph, a.timeout_ns, &T.abort_flag)) {
             T.abort_flag = 1;
             atomicOr(a.status, DEV_ERR_TIMEOUT);
@@ -339,17 +361,18 @@ size_t refine_smem_bytes(int H, int D, int /*mc*/) {
   return 0;
 }
 
-cudaError_t launch_refine(const RefineArgs& a, const CUtensorMap* kmap, int grid, cudaStream_t s) {
+cudaError_t launch_refine(const RefineArgs& a, const CUtensorMap* kmap, const CUtensorMap* qmap, int grid,
+                          cudaStream_t s) {
   const size_t smem = refine_smem_bytes(a.H, a.D, a.mc);
   uint32_t* keys = a.keys;
   if (a.H == 64 && a.D == 128) {
     auto k = refine_kernel<64, 128>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, RefCfg<64, 128>::THREADS, smem, s>>>(*kmap, a, keys);
+    k<<<grid, RefCfg<64, 128>::THREADS, smem, s>>>(*kmap, *qmap, a, keys);
   } else if (a.H == 64 && a.D == 64) {
     auto k = refine_kernel<64, 64>;
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k<<<grid, RefCfg<64, 64>::THREADS, smem, s>>>(*kmap, a, keys);
+    k<<<grid, RefCfg<64, 64>::THREADS, smem, s>>>(*kmap, *qmap, a, keys);
   } else {
     return cudaErrorInvalidValue;
   }
