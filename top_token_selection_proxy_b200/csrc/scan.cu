@@ -44,11 +44,10 @@ struct ScanCfg {
   static constexpr int STAGES = 4;
   static constexpr int A_BYTES = BM * D * 2;
   static constexpr int B_BYTES = N * D * 2;
-  static constexpr int THREADS = 320;  // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
-  static constexpr int NEPI = 256;
-  static constexpr int GPH = NB / 2;   // groups per epilogue half (two warps share each TMEM lane quarter)
+  static constexpr int THREADS = 64 + 128 * NB;  // warp 0 TMA, warp 1 MMA, 4 epilogue warps per group
+  static constexpr int NEPI = 128 * NB;          // one warp per (group, TMEM lane quarter)
   static constexpr int SMEM_CAP = STAGES * A_BYTES / 8;  // packed entries the freed stage ring can hold
-  static_assert(NB <= 8 && NB % 2 == 0, "2..8 groups per item");
+  static_assert(NB == 4, "four groups per item (H = 64)");
 };
 
 struct ScanTail {
@@ -79,7 +78,7 @@ constexpr size_t scan_smem() {
 }
 
 template <int H, int D>
-__global__ void __launch_bounds__(320, 1) scan_kernel(const __grid_constant__ CUtensorMap kmap, const ScanArgs a) {
+__global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CUtensorMap kmap, const ScanArgs a) {
   using C = ScanCfg<H, D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -116,7 +115,7 @@ __global__ void __launch_bounds__(320, 1) scan_kernel(const __grid_constant__ CU
   uint32_t m_st = 0, m_ph = 0, m_ab = 0, m_aph = 0;     // MMA: ring + accumulator
   uint32_t e_ab = 0, e_aph = 0;                         // epilogue: accumulator
   uint64_t* selbase = a.selbuf + (uint64_t)blockIdx.x * C::NB * (uint64_t)a.cap;
-  const Group<256> EG{tid - 64, 1};
+  const Group<C::NEPI> EG{tid - 64, 1};
   const bool decode = (a.mode == EMIT_PARTIAL);
 
   for (;;) {
@@ -280,33 +279,22 @@ __global__ void __launch_bounds__(320, 1) scan_kernel(const __grid_constant__ CU
       }
     } else {
       // ------------------------------------------------------------ epilogue + select
-      // warp w reads TMEM lanes 32*(w%4).. (its keys); the two warps of a lane
-      // quarter split the groups: half 0 takes groups [0, GPH), half 1 [GPH, NB).
-      // Each (group, lane quarter) owns a sub-buffer of sub_cap entries that only
-      // its warp appends to, with the count kept in a register.
+      // warp w reads TMEM lanes 32*(w%4).. (its keys) and handles one group: warps
+      // 2-5 group 0, 6-9 group 1, ...  Each (group, lane quarter) owns a sub-buffer of
+      // sub_cap entries that only its warp appends to, with the count in a register.
       const int q4 = warp & 3;
-      const int half = (warp - 2) >> 2;
+      const int grp_w = (warp - 2) >> 2;  // this warp's group within the item
       const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
       const uint32_t need = (uint32_t)a.n_sel;
       const uint32_t gstride = (uint32_t)a.cap;    // 4 sub-buffers per group
       const uint32_t scap = (uint32_t)a.sub_cap;
-      uint32_t qcnt[C::GPH];
-      uint64_t tau_r[C::GPH];
-      int64_t e_r[C::GPH];  // causal bound of each of this warp's groups
-#pragma unroll
-      for (int gi = 0; gi < C::GPH; ++gi) e_r[gi] = T.e[half * C::GPH + gi];
-
+      uint32_t qcnt = 0;
+      uint64_t tau_r = 0;
+      const int64_t e_r = T.e[grp_w];  // causal bound of this warp's group
       const int64_t s_begin = T.s_begin, s_end = T.s_end;
-#pragma unroll
-      for (int gi = 0; gi < C::GPH; ++gi) {
-        qcnt[gi] = 0;
-        tau_r[gi] = 0;
-      }
       auto seg_of = [&](int b, int q) { return selbase + (uint64_t)b * gstride + (uint64_t)q * scap; };
       auto publish_counts = [&]() {
-        if (lane == 0)
-#pragma unroll
-          for (int gi = 0; gi < C::GPH; ++gi) T.qcnt[half * C::GPH + gi][q4] = qcnt[gi];
+        if (lane == 0) T.qcnt[grp_w][q4] = qcnt;
         EG.sync();
       };
       // cut group b back to a superset of its best `need` (keep <= maxk), every warp
@@ -318,11 +306,10 @@ __global__ void __launch_bounds__(320, 1) scan_kernel(const __grid_constant__ CU
           sg.p[q] = seg_of(b, q);
           sg.n[q] = T.qcnt[b][q];
         }
-        const uint64_t th = radix11_threshold<256>(sg, need, maxk, T.hist11, T.sel, EG);
-        if (half == b / C::GPH) {
-          const int gi = b % C::GPH;
-          qcnt[gi] = warp_compact_ge(seg_of(b, q4), qcnt[gi], th);
-          if (th > 0) tau_r[gi] = th - 1ull;  // admit x >= th from now on
+        const uint64_t th = radix11_threshold<C::NEPI>(sg, need, maxk, T.hist11, T.sel, EG);
+        if (grp_w == b) {
+          qcnt = warp_compact_ge(seg_of(b, q4), qcnt, th);
+          if (th > 0) tau_r = th - 1ull;  // admit x >= th from now on
         }
         EG.sync();
       };
@@ -336,65 +323,51 @@ __global__ void __launch_bounds__(320, 1) scan_kernel(const __grid_constant__ CU
           T.abort_flag = 1;
           atomicOr(a.status, DEV_ERR_TIMEOUT);
         }
-        float sc[C::GPH];
+        float sc = 0.f;
         if (ok) {
           tc_fence_after();
+          const float4* wv = reinterpret_cast<const float4*>(&T.wbar[grp_w * H]);
+          float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                           make_float2(0.f, 0.f)};
 #pragma unroll
-          for (int gi = 0; gi < C::GPH; ++gi) {
-            const int b = half * C::GPH + gi;
-            // w-bar of the group first (shared-memory broadcast loads), then the accumulator row
-            float4 w4[H / 4];
-            const float4* wv = reinterpret_cast<const float4*>(&T.wbar[b * H]);
-#pragma unroll
-            for (int i = 0; i < H / 4; ++i) w4[i] = wv[i];
-            uint32_t r[H];
-#pragma unroll
-            for (int h0 = 0; h0 < H; h0 += 32)
-              tmem_ld32(tmem + lane_base + e_ab * 256u + (uint32_t)(b * H + h0),
-                        *reinterpret_cast<uint32_t(*)[32]>(&r[h0]));
+          for (int h0 = 0; h0 < H; h0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(tmem + lane_base + e_ab * 256u + (uint32_t)(grp_w * H + h0), r);
             tmem_wait_ld();
-            if (gi == C::GPH - 1) {
+            if (h0 + 32 == H) {
               tc_fence_before();
               mbar_arrive(&T.acce[e_ab]);  // this warp's columns are in registers: the MMA may refill
             }
-            float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                             make_float2(0.f, 0.f)};
 #pragma unroll
-            for (int i = 0; i < H / 4; ++i) {
+            for (int i = 0; i < 8; ++i) {
+              const float4 w4 = wv[h0 / 4 + i];
               const float2 x0 = make_float2(fmaxf(__uint_as_float(r[4 * i + 0]), 0.f),
                                             fmaxf(__uint_as_float(r[4 * i + 1]), 0.f));
               const float2 x1 = make_float2(fmaxf(__uint_as_float(r[4 * i + 2]), 0.f),
                                             fmaxf(__uint_as_float(r[4 * i + 3]), 0.f));
-              acc[(2 * i) & 3] = __ffma2_rn(make_float2(w4[i].x, w4[i].y), x0, acc[(2 * i) & 3]);
-              acc[(2 * i + 1) & 3] = __ffma2_rn(make_float2(w4[i].z, w4[i].w), x1, acc[(2 * i + 1) & 3]);
+              acc[(2 * i) & 3] = __ffma2_rn(make_float2(w4.x, w4.y), x0, acc[(2 * i) & 3]);
+              acc[(2 * i + 1) & 3] = __ffma2_rn(make_float2(w4.z, w4.w), x1, acc[(2 * i + 1) & 3]);
             }
-            sc[gi] = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
           }
+          sc = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
         }
         if (++e_ab == 2) {
           e_ab = 0;
           e_aph ^= 1u;
         }
-        // streaming selection: append entries above each group's threshold
+        // streaming selection: append entries above the group's threshold
         bool near_full = false;
-        if (ok) {
+        if (ok && grp_w < nb_act) {
           const int64_t s = s_begin + (int64_t)j * C::BM + q4 * 32 + lane;
-          const uint32_t lt = lanemask_lt();
-#pragma unroll
-          for (int gi = 0; gi < C::GPH; ++gi) {
-            const int b = half * C::GPH + gi;
-            if (b < nb_act) {
-              const bool valid = (s < s_end) && (s <= e_r[gi]);
-              const uint64_t p = pack_entry(score_key(sc[gi]), (uint32_t)s);
-              const bool pass = valid && p > tau_r[gi];
-              const uint32_t m = __ballot_sync(0xFFFFFFFFu, pass);
-              if (pass) seg_of(b, q4)[qcnt[gi] + __popc(m & lt)] = p;
-              qcnt[gi] += __popc(m);
-              if (qcnt[gi] > scap - 4u * 32u) {  // the next 4 tiles could overflow this sub-buffer
-                near_full = true;
-                if (lane == 0) atomicOr(&T.cflags, 1u << b);
-              }
-            }
+          const bool valid = (s < s_end) && (s <= e_r);
+          const uint64_t p = pack_entry(score_key(sc), (uint32_t)s);
+          const bool pass = valid && p > tau_r;
+          const uint32_t m = __ballot_sync(0xFFFFFFFFu, pass);
+          if (pass) seg_of(grp_w, q4)[qcnt + __popc(m & lanemask_lt())] = p;
+          qcnt += __popc(m);
+          if (qcnt > scap - 4u * 32u) {  // the next 4 tiles could overflow this sub-buffer
+            near_full = true;
+            if (lane == 0) atomicOr(&T.cflags, 1u << grp_w);
           }
         }
         // consensus every 4 tiles (the same tiles for every epilogue thread, so all of them
@@ -428,7 +401,7 @@ __global__ void __launch_bounds__(320, 1) scan_kernel(const __grid_constant__ CU
           uint32_t off = 0;
           for (int q = 0; q < 4; ++q) {
             const uint32_t nq = T.qcnt[b][q];
-            group_copy<256>(sbuf + off, seg_of(b, q), nq, EG);
+            group_copy<C::NEPI>(sbuf + off, seg_of(b, q), nq, EG);
             off += (nq + 1u) & ~1u;
             if (nq & 1u) {  // pad to keep the next segment aligned: a zero entry sorts below everything
               if (EG.tid == 0) sbuf[off - 1] = 0ull;
@@ -441,17 +414,17 @@ __global__ void __launch_bounds__(320, 1) scan_kernel(const __grid_constant__ CU
           // keep-all is th = 1, so the zero pads never survive; otherwise the need-th
           // largest is a real entry (n_real > need)
           const uint64_t th =
-              (n_real <= need) ? 1ull : radix11_threshold<256>(buf, n, need, need, T.hist11, T.sel, EG);
-          const uint32_t m = compact_ge<256>(buf, buf, n, th, T.sel, EG);
+              (n_real <= need) ? 1ull : radix11_threshold<C::NEPI>(buf, n, need, need, T.hist11, T.sel, EG);
+          const uint32_t m = compact_ge<C::NEPI>(buf, buf, n, th, T.sel, EG);
           const int64_t grp = T.grp0 + b;
           if (a.mode == EMIT_DENSE) {
-            emit_row<256>(buf, m, 0xFFFFFFFFu, 0ull, a.out_idx + grp * a.topk,
+            emit_row<C::NEPI>(buf, m, 0xFFFFFFFFu, 0ull, a.out_idx + grp * a.topk,
                           a.out_scores ? a.out_scores + grp * a.topk : nullptr, (uint32_t)a.topk, T.sel, EG);
           } else if (a.mode == EMIT_CAND) {
-            emit_row<256>(buf, m, 0xFFFFFFFFu, 0ull, a.cand + grp * a.n_sel,
+            emit_row<C::NEPI>(buf, m, 0xFFFFFFFFu, 0ull, a.cand + grp * a.n_sel,
                           a.cand_scores ? a.cand_scores + grp * a.n_sel : nullptr, need, T.sel, EG);
           } else if (a.mode == EMIT_REUSE) {
-            emit_reuse<256>(buf, m, a.topk, T.mrow0[b], T.nmem[b], T.mrow0[b], a.out_idx, a.out_scores, T.sel,
+            emit_reuse<C::NEPI>(buf, m, a.topk, T.mrow0[b], T.nmem[b], T.mrow0[b], a.out_idx, a.out_scores, T.sel,
                             T.bot, &T.nbot, EG);
           } else {  // EMIT_PARTIAL: the chunk's exact top-n_sel, zero padded
             uint64_t* dst = a.partial + (uint64_t)item * (uint32_t)a.partial_stride;
