@@ -29,7 +29,7 @@ __device__ __forceinline__ uint64_t pack_entry(uint32_t key, uint32_t idx) {
 __device__ __forceinline__ uint32_t entry_idx(uint64_t p) { return 0xFFFFFFFFu - (uint32_t)p; }
 __device__ __forceinline__ float entry_score(uint64_t p) { return key_score((uint32_t)(p >> 32)); }
 
-struct SelSmem {
+struct alignas(16) SelSmem {  // hist is also reused as uint64 scratch (emit_reuse)
   uint32_t hist[256];
   uint32_t warp_tot[32];
   uint32_t scal[4];
@@ -396,6 +396,67 @@ __device__ __forceinline__ uint64_t radix11_threshold(const uint64_t* buf, uint3
   return radix11_threshold<NT>(sg, need, max_keep, hist, S, G);
 }
 
+// Like radix11_threshold, for entries known to lie in [lo, hi]: each pass
+// histograms (x - lo) >> shift into up to 2048 bins with shift chosen so the
+// bins tile the current range, then narrows the range to the bin holding the
+// need-th largest.  A tight [lo, hi] spreads the entries over all bins (little
+// atomic contention) and usually settles within one pass.
+template <int NT>
+__device__ uint64_t radix_range_threshold(const Segs& sg, uint64_t lo, uint64_t hi, uint32_t need,
+                                          uint32_t max_keep, uint32_t* hist, SelSmem& S, const Group<NT>& G) {
+  static_assert(2048 % NT == 0 || NT % 2048 == 0, "NT must divide 2048 or be a multiple");
+  constexpr int BPT = (2048 / NT) > 0 ? (2048 / NT) : 1;
+  uint32_t n = 0;
+  for (int i = 0; i < sg.cnt; ++i) n += sg.n[i];
+  if (n <= max_keep) return 0ull;
+  uint32_t above = 0;
+  for (int pass = 0; pass < 8; ++pass) {
+    const uint64_t span = hi - lo;  // entries of interest are in [lo, hi]
+    const int bits = span == 0 ? 0 : 64 - __clzll(span);
+    const int shift = bits > 11 ? bits - 11 : 0;
+    for (uint32_t i = G.tid; i < 2048; i += NT) hist[i] = 0u;
+    G.sync();
+    for (int sgi = 0; sgi < sg.cnt; ++sgi)
+      visit_entries<NT, 8>(sg.p[sgi], sg.n[sgi], G, [&](uint64_t x, bool valid) {
+        if (valid && x >= lo && x <= hi) atomicAdd(&hist[(uint32_t)((x - lo) >> shift)], 1u);
+      });
+    G.sync();
+    uint32_t loc[BPT], sum = 0;
+#pragma unroll
+    for (int u = 0; u < BPT; ++u) {
+      const int bin = 2047 - BPT * G.tid - u;
+      loc[u] = (bin >= 0 && G.tid * BPT + u < 2048) ? hist[bin] : 0u;
+      sum += loc[u];
+    }
+    uint32_t total;
+    const uint32_t excl = group_offsets<NT>(sum, &total, S, G);
+    if (above + excl < need && need <= above + excl + sum) {
+      uint32_t c = above + excl;
+#pragma unroll
+      for (int u = 0; u < BPT; ++u) {
+        if (c + loc[u] >= need) {
+          S.scal[0] = (uint32_t)(2047 - BPT * G.tid - u);
+          S.scal[1] = c;
+          S.scal[2] = loc[u];
+          break;
+        }
+        c += loc[u];
+      }
+    }
+    G.sync();
+    const uint32_t bin = S.scal[0];
+    above = S.scal[1];
+    const uint32_t h = S.scal[2];
+    G.sync();
+    const uint64_t blo = lo + ((uint64_t)bin << shift);
+    const uint64_t bhi = (shift == 0) ? blo : (blo + (((uint64_t)1 << shift) - 1ull));
+    if (above + h <= max_keep || shift == 0) return blo;  // keep x >= blo
+    lo = blo;
+    hi = bhi < hi ? bhi : hi;
+  }
+  return lo;
+}
+
 // Stream-compact the entries >= T of src[0..n) into dst[0..m) (dst may be
 // src: every chunk is fully read before any of its survivors is written, and
 // survivors never move forward).  Returns m.  When hist1 is given it is
@@ -489,10 +550,14 @@ __device__ uint32_t emit_row(const uint64_t* buf, uint32_t n, uint32_t t_max, ui
 // member t keeps the k best of { entries with index <= t }.  Removing the
 // r <= g-1 entries above t leaves at least k; the ones to drop beyond the
 // k best are the lowest eligible entries, all among the m-k lowest of buf.
+// One counting pass (each entry's first eligible member) and one emission
+// pass that writes every entry to each member row it belongs to (row order
+// is free; rows are padded with -1 to width topk).  nmem <= 16.
 template <int NT>
 __device__ void emit_reuse(uint64_t* buf, uint32_t m, int topk, int64_t t_first, int nmem, int64_t out_row0,
                            int32_t* out_idx, float* out_sc, SelSmem& S, uint64_t* bot, uint32_t* nbot,
                            const Group<NT>& G) {
+  // bottom entries (the m - topk lowest, at most 15), sorted ascending
   uint32_t nb = 0;
   if (m > (uint32_t)topk) {
     const uint64_t Tk = radix_threshold<NT>(buf, m, topk, topk, S, G);
@@ -507,7 +572,7 @@ __device__ void emit_reuse(uint64_t* buf, uint32_t m, int topk, int64_t t_first,
     }
     G.sync();
     nb = *nbot;
-    if (G.tid == 0) {  // ascending insertion sort of at most g-1 entries
+    if (G.tid == 0) {
       for (uint32_t i = 1; i < nb && i < 16; ++i) {
         const uint64_t v = bot[i];
         int j = (int)i - 1;
@@ -520,25 +585,78 @@ __device__ void emit_reuse(uint64_t* buf, uint32_t m, int topk, int64_t t_first,
     }
     G.sync();
   }
-  for (int r = 0; r < nmem; ++r) {
-    const int64_t t = t_first + r;
-    uint64_t cut = 0;
-    if (nb > 0) {
-      const uint32_t elig = count_idx_le<NT>(buf, m, (uint32_t)t, S, G);
-      if (elig > (uint32_t)topk) {
-        const uint32_t mdrop = elig - topk;
-        uint32_t c = 0;
-        for (uint32_t u = 0; u < nb && u < 16; ++u)
-          if (entry_idx(bot[u]) <= (uint32_t)t && ++c == mdrop) {
-            cut = bot[u];
-            break;
-          }
+  // eligible count of every member: entry i is eligible for members r >= first(i)
+  for (int i = G.tid; i < 16; i += NT) S.hist[i] = 0u;
+  G.sync();
+  for (uint32_t i0 = 0; i0 < m; i0 += NT) {
+    const uint32_t i = i0 + G.tid;
+    uint32_t r0 = 16u;
+    if (i < m) {
+      const int64_t s = entry_idx(buf[i]);
+      r0 = (uint32_t)(s <= t_first ? 0 : (s - t_first));
+    }
+    hist_add(S.hist, r0 < 16u ? r0 : 256u);
+  }
+  G.sync();
+  // per member: its cut (drop the lowest eligible beyond k) and its row counter
+  uint64_t* cut = reinterpret_cast<uint64_t*>(&S.hist[32]);  // 16 x uint64 after the 16 counts
+  uint32_t* rowc = &S.hist[64];
+  if (G.tid < nmem) {
+    const int r = G.tid;
+    uint32_t elig = 0;
+    for (int u = 0; u <= r; ++u) elig += S.hist[u];
+    uint64_t c = 0;
+    if (nb > 0 && elig > (uint32_t)topk) {
+      const uint32_t mdrop = elig - topk;
+      const int64_t t = t_first + r;
+      uint32_t cc = 0;
+      for (uint32_t u = 0; u < nb && u < 16; ++u)
+        if ((int64_t)entry_idx(bot[u]) <= t && ++cc == mdrop) {
+          c = bot[u];
+          break;
+        }
+    }
+    cut[r] = c;
+    rowc[r] = 0u;
+  }
+  G.sync();
+  const uint32_t lt = lanemask_lt();
+  for (uint32_t i0 = 0; i0 < m; i0 += NT) {
+    const uint32_t i = i0 + G.tid;
+    uint64_t x = 0;
+    int64_t s = 0;
+    if (i < m) {
+      x = buf[i];
+      s = entry_idx(x);
+    }
+    for (int r = 0; r < nmem; ++r) {
+      const bool in = (i < m) && s <= t_first + r && x > cut[r];
+      const uint32_t msk = __ballot_sync(0xFFFFFFFFu, in);
+      if (msk == 0u) continue;
+      const int leader = __ffs(msk) - 1;
+      uint32_t base = 0;
+      if ((int)lane_id() == leader) base = atomicAdd(&rowc[r], (uint32_t)__popc(msk));
+      base = __shfl_sync(0xFFFFFFFFu, base, leader);
+      if (in) {
+        const uint32_t pos = base + __popc(msk & lt);
+        if (pos < (uint32_t)topk) {
+          const int64_t row = out_row0 + r;
+          out_idx[row * topk + pos] = (int32_t)s;
+          if (out_sc) out_sc[row * topk + pos] = entry_score(x);
+        }
       }
     }
-    const int64_t row = out_row0 + r;
-    emit_row<NT>(buf, m, (uint32_t)t, cut, out_idx + row * topk, out_sc ? out_sc + row * topk : nullptr,
-                 (uint32_t)topk, S, G);
   }
+  G.sync();
+  for (int r = 0; r < nmem; ++r) {  // pad
+    const uint32_t cnt = rowc[r] < (uint32_t)topk ? rowc[r] : (uint32_t)topk;
+    const int64_t row = out_row0 + r;
+    for (uint32_t p = cnt + G.tid; p < (uint32_t)topk; p += NT) {
+      out_idx[row * topk + p] = -1;
+      if (out_sc) out_sc[row * topk + p] = -__int_as_float(0x7f800000);
+    }
+  }
+  G.sync();
 }
 
 }  // namespace pivot
