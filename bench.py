@@ -34,6 +34,34 @@ METRIC = "indexer queries/sec at L=128K g=8 Refine (1×B200); % of roofline; × 
 UNIT = "queries/s"
 L2_FLUSH_BYTES = 256 << 20
 
+# DRAM bytes (read + write) of one scan launch on this workload, from a 1-pass
+# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum); valid only while
+# the sources the scan kernel is built from hash to `sources_sha256`.
+SCAN_TRAFFIC = {
+    "bytes": 3.35e9 + 4.12e9,
+    "sources": ("scan.cu", "select.cuh", "ptx.cuh", "kernels.cuh"),
+    "sources_sha256": "6a8f91ad0a02e7c42a55fce3e70fc52245b026b4000edcf72cfb20936590727a",
+    "profile": "profiles/dram_traffic_prefill_L131072_g8_refine.md",
+}
+
+
+def scan_sources_sha256():
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in SCAN_TRAFFIC["sources"]:
+        with open(os.path.join(ROOT, "top_token_selection_proxy_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def scan_traffic():
+    """Measured DRAM bytes per scan launch, or None once the kernel changed since the capture."""
+    try:
+        return SCAN_TRAFFIC["bytes"] if scan_sources_sha256() == SCAN_TRAFFIC["sources_sha256"] else None
+    except OSError:
+        return None
+
 
 def parse():
     p = argparse.ArgumentParser()
@@ -399,9 +427,10 @@ def main():
         "us_per_group": 1000.0 * ms / G,
         "kernels_ms": {"scan": scan_ms, "refine": statistics.median(k_ref), "rowselect": statistics.median(k_sel)},
         "roofline": {"bound": "tensor", "kernel": "scan (proxy pooling + tcgen05 proxy scan + streaming select)",
-                     "achieved": achieved, "peak": tf_sust, "unit": "TFLOP/s", "frac": achieved / tf_sust,
-                     "peak_kind": f"{src} bf16 dense, sustained", "frac_of_burst": achieved / tf_burst,
-                     "flops_per_launch": f_scan, "traffic": None},
+                     "achieved": achieved, "peak": tf_burst, "unit": "TFLOP/s", "frac": achieved / tf_burst,
+                     "peak_kind": f"{src} bf16 dense, burst", "frac_of_sustained": achieved / tf_sust,
+                     "flops_per_launch": f_scan, "traffic": scan_traffic(),
+                     "traffic_source": SCAN_TRAFFIC["profile"]},
         "roofline_path": {"t_roof_ms_scan_only": t_roof_lit, "frac_scan_only": t_roof_lit / ms,
                           "t_roof_ms_scan_plus_refine": t_roof_alg, "frac_scan_plus_refine": t_roof_alg / ms,
                           "peak": f"{src} burst bf16 {tf_burst} TFLOP/s, HBM {hbm} GB/s",
