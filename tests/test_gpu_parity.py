@@ -121,6 +121,24 @@ def full_check(orc, x, res, topk, c, g, groups=None, dense_rows=None):
 # ---------------------------------------------------------------- small workloads, every row
 
 
+@pytest.mark.parametrize("c_sel,topk", [(100, 37), (130, 64)])
+def test_refine_unaligned_candidates_and_odd_c(orc, c_sel, topk):
+    """C written to a 4-byte-offset buffer, c not a multiple of 4: the member
+    top-k takes its scalar-load path; every group is checked."""
+    x = inputs.random_prefill(1337, 64, 128, inputs.BF16, seed=777)
+    q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
+    g = 8
+    G = (1337 + g - 1) // g
+    backing = torch.empty(G * c_sel + 1, dtype=torch.int32, device=q.device)
+    cand_buf = backing[1:].view(G, c_sel)
+    assert cand_buf.data_ptr() % 16 != 0
+    r_idx, r_sc, r_c, r_cs = P.refine(q, w, k, topk, c_sel, g, scores=True, cand=cand_buf)
+    torch.cuda.synchronize()
+    assert r_c.data_ptr() == cand_buf.data_ptr()
+    fails = check_refine(orc, x, host(r_idx), host(r_sc), host(r_c), host(r_cs), range(G), topk, c_sel, g)
+    assert not fails, summarize(fails)
+
+
 def test_tiny_config_every_group(orc):
     s = inputs.TINY
     x = inputs.make_prefill(s)

@@ -193,15 +193,24 @@ def reuse(q, w, k, topk: int, g: int, *, scores: bool = False, out=None, ws: Opt
     return idx, sc
 
 
-def refine(q, w, k, topk: int, c: int, g: int, *, scores: bool = False, cand: bool = False, out=None,
+def refine(q, w, k, topk: int, c: int, g: int, *, scores: bool = False, cand=False, out=None,
            ws: Optional[Workspace] = None, stream=None):
-    """Eq. (4),(5),(7)-(9): PIVOT-Refine.  Returns (indices, member scores|None, C|None, C scores|None)."""
+    """Eq. (4),(5),(7)-(9): PIVOT-Refine.  Returns (indices, member scores|None, C|None, C scores|None).
+
+    `cand` is False, True (allocate C) or a contiguous int32 [G, c] device tensor
+    that receives C (any 4-byte aligned address)."""
     L, H, d, dt = _prefill_common(q, w, k)
     G = (L + g - 1) // g
     idx = out if out is not None else torch.empty((L, topk), dtype=torch.int32, device=q.device)
     sc = torch.empty((L, topk), dtype=torch.float32, device=q.device) if scores else None
-    cd = torch.empty((G, c), dtype=torch.int32, device=q.device) if cand else None
-    cs = torch.empty((G, c), dtype=torch.float32, device=q.device) if (cand and scores) else None
+    if isinstance(cand, torch.Tensor):
+        if cand.dtype != torch.int32 or tuple(cand.shape) != (G, c) or not cand.is_contiguous() \
+                or cand.device != q.device:
+            raise ValueError("cand must be a contiguous int32 [G, c] tensor on q's device")
+        cd = cand
+    else:
+        cd = torch.empty((G, c), dtype=torch.int32, device=q.device) if cand else None
+    cs = torch.empty((G, c), dtype=torch.float32, device=q.device) if (cd is not None and scores) else None
     nbytes = workspace_size(OP_REFINE, L, H, d, topk, c, g, dt)
     W = _ws_for(ws, q.device).get(nbytes)
     _check(lib().pivot_refine(_ptr(q), _ptr(w), _ptr(k), L, H, d, dt, topk, c, g, _ptr(idx), _ptr(sc), _ptr(cd),

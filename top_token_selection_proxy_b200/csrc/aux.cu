@@ -21,7 +21,7 @@ namespace pivot {
 __global__ void __launch_bounds__(256) rowselect_kernel(const RowSelArgs a) {
   extern __shared__ uint64_t sbuf[];  // c packed entries of the row
   __shared__ SelSmem S;
-  __shared__ uint32_t hist11[2048];
+  __shared__ uint32_t hist11[kHist11Words];
   const Group<256> G{(int)threadIdx.x, 0};
   for (int64_t row = blockIdx.x; row < a.n_rows; row += gridDim.x) {
     const int64_t grp = row / a.g;

@@ -63,7 +63,7 @@ struct ScanTail {
   uint64_t tau[16];         // running admission threshold of each group (admit packed > tau)
   uint32_t qcnt[8][4];      // per group, entries in each lane quarter's sub-buffer (published on demand)
   uint32_t cflags;          // groups whose sub-buffers need a cut-back
-  uint32_t hist11[2048];    // radix-select histogram (11-bit digits)
+  uint32_t hist11[kHist11Words];    // radix-select histogram (11-bit digits)
   uint64_t bot[16];
   uint32_t nbot;
   SelSmem sel;

@@ -323,10 +323,17 @@ __device__ __forceinline__ uint32_t group_offsets(uint32_t cnt, uint32_t* total,
 // ---------------------------------------------------------------- 11-bit digits
 // Digit widths of the 64-bit packed entry, most significant first.
 __host__ __device__ constexpr int r11_width(int d) { return d < 5 ? 11 : 9; }
+
+// The 2048-bin histogram is stored with one pad word after every 32 bins, so
+// the digit search (thread t reads bins BPT*t .. BPT*t + BPT-1, BPT = 4 or 8)
+// hits 32 distinct banks per warp instead of 32 / BPT.
+constexpr int kHist11Words = 2048 + 64;
+__device__ __forceinline__ uint32_t h11(uint32_t bin) { return bin + (bin >> 5); }
 __host__ __device__ constexpr int r11_shift(int d) { return 64 - 11 * (d + 1) < 0 ? 0 : 64 - 11 * (d + 1); }
 
 // Like radix_threshold, with 11-bit digits (at most 6 passes, usually 2) and a
-// 2048-bin shared-memory histogram `hist` updated with plain atomics.  The
+// 2048-bin shared-memory histogram `hist` (kHist11Words words, padded layout)
+// updated with plain atomics.  The
 // entries are the union of the segments of sg.
 template <int NT>
 __device__ uint64_t radix11_threshold(const Segs& sg, uint32_t need, uint32_t max_keep, uint32_t* hist,
@@ -342,12 +349,12 @@ __device__ uint64_t radix11_threshold(const Segs& sg, uint32_t need, uint32_t ma
   for (int d = 0; d < 6; ++d) {
     const int w = r11_width(d), shift = r11_shift(d);
     const uint32_t nb = 1u << w;
-    for (uint32_t i = G.tid; i < 2048; i += NT) hist[i] = 0u;
+    for (uint32_t i = G.tid; i < (uint32_t)kHist11Words; i += NT) hist[i] = 0u;
     G.sync();
     for (int sgi = 0; sgi < sg.cnt; ++sgi)
       visit_entries<NT, 8>(sg.p[sgi], sg.n[sgi], G, [&](uint64_t x, bool valid) {
         if (valid && (consumed == 0 || (x >> (64 - consumed)) == prefix))
-          atomicAdd(&hist[(uint32_t)(x >> shift) & (nb - 1u)], 1u);
+          atomicAdd(&hist[h11((uint32_t)(x >> shift) & (nb - 1u))], 1u);
       });
     G.sync();
     // thread t owns bins [nb-1 - BPT*t - (BPT-1), nb-1 - BPT*t] (descending); bins >= nb are empty
@@ -355,7 +362,7 @@ __device__ uint64_t radix11_threshold(const Segs& sg, uint32_t need, uint32_t ma
 #pragma unroll
     for (int u = 0; u < BPT; ++u) {
       const int bin = 2047 - BPT * G.tid - u - (2048 - (int)nb);
-      loc[u] = (bin >= 0) ? hist[bin] : 0u;
+      loc[u] = (bin >= 0) ? hist[h11((uint32_t)bin)] : 0u;
       sum += loc[u];
     }
     uint32_t total;
@@ -394,67 +401,6 @@ __device__ __forceinline__ uint64_t radix11_threshold(const uint64_t* buf, uint3
   sg.p[0] = buf;
   sg.n[0] = n;
   return radix11_threshold<NT>(sg, need, max_keep, hist, S, G);
-}
-
-// Like radix11_threshold, for entries known to lie in [lo, hi]: each pass
-// histograms (x - lo) >> shift into up to 2048 bins with shift chosen so the
-// bins tile the current range, then narrows the range to the bin holding the
-// need-th largest.  A tight [lo, hi] spreads the entries over all bins (little
-// atomic contention) and usually settles within one pass.
-template <int NT>
-__device__ uint64_t radix_range_threshold(const Segs& sg, uint64_t lo, uint64_t hi, uint32_t need,
-                                          uint32_t max_keep, uint32_t* hist, SelSmem& S, const Group<NT>& G) {
-  static_assert(2048 % NT == 0 || NT % 2048 == 0, "NT must divide 2048 or be a multiple");
-  constexpr int BPT = (2048 / NT) > 0 ? (2048 / NT) : 1;
-  uint32_t n = 0;
-  for (int i = 0; i < sg.cnt; ++i) n += sg.n[i];
-  if (n <= max_keep) return 0ull;
-  uint32_t above = 0;
-  for (int pass = 0; pass < 8; ++pass) {
-    const uint64_t span = hi - lo;  // entries of interest are in [lo, hi]
-    const int bits = span == 0 ? 0 : 64 - __clzll(span);
-    const int shift = bits > 11 ? bits - 11 : 0;
-    for (uint32_t i = G.tid; i < 2048; i += NT) hist[i] = 0u;
-    G.sync();
-    for (int sgi = 0; sgi < sg.cnt; ++sgi)
-      visit_entries<NT, 8>(sg.p[sgi], sg.n[sgi], G, [&](uint64_t x, bool valid) {
-        if (valid && x >= lo && x <= hi) atomicAdd(&hist[(uint32_t)((x - lo) >> shift)], 1u);
-      });
-    G.sync();
-    uint32_t loc[BPT], sum = 0;
-#pragma unroll
-    for (int u = 0; u < BPT; ++u) {
-      const int bin = 2047 - BPT * G.tid - u;
-      loc[u] = (bin >= 0 && G.tid * BPT + u < 2048) ? hist[bin] : 0u;
-      sum += loc[u];
-    }
-    uint32_t total;
-    const uint32_t excl = group_offsets<NT>(sum, &total, S, G);
-    if (above + excl < need && need <= above + excl + sum) {
-      uint32_t c = above + excl;
-#pragma unroll
-      for (int u = 0; u < BPT; ++u) {
-        if (c + loc[u] >= need) {
-          S.scal[0] = (uint32_t)(2047 - BPT * G.tid - u);
-          S.scal[1] = c;
-          S.scal[2] = loc[u];
-          break;
-        }
-        c += loc[u];
-      }
-    }
-    G.sync();
-    const uint32_t bin = S.scal[0];
-    above = S.scal[1];
-    const uint32_t h = S.scal[2];
-    G.sync();
-    const uint64_t blo = lo + ((uint64_t)bin << shift);
-    const uint64_t bhi = (shift == 0) ? blo : (blo + (((uint64_t)1 << shift) - 1ull));
-    if (above + h <= max_keep || shift == 0) return blo;  // keep x >= blo
-    lo = blo;
-    hi = bhi < hi ? bhi : hi;
-  }
-  return lo;
 }
 
 // Stream-compact the entries >= T of src[0..n) into dst[0..m) (dst may be
