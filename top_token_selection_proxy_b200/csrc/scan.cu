@@ -67,9 +67,12 @@ struct ScanTail {
   uint64_t bot[16];
   uint32_t nbot;
   SelSmem sel;
-  alignas(16) float wbar[256];  // read as float4
+  // w-bar of the item's groups, permuted for the epilogue: row (b, m) holds heads
+  // 8j + 2m, 8j + 2m + 1 (j = 0..7) of group b in 16 floats, rows 20 floats apart
+  // so the 4 rows a warp reads sit in distinct banks
+  alignas(16) float wperm[16 * 20];
 };
-static_assert(offsetof(ScanTail, wbar) % 16 == 0, "wbar must be 16-byte aligned");
+static_assert(offsetof(ScanTail, wperm) % 16 == 0, "wperm must be 16-byte aligned");
 
 template <int H, int D>
 constexpr size_t scan_smem() {
@@ -215,7 +218,8 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
         const int64_t r0 = T.mrow0[b];
         float s = 0.f;
         for (int mm = 0; mm < nm; ++mm) s += __ldg(a.w + (r0 + mm) * H + hj);
-        T.wbar[u] = nm > 1 ? __fdiv_rn(s, (float)nm) : s;
+        const int jj = hj >> 3, m = (hj >> 1) & 3;
+        T.wperm[(b * 4 + m) * 20 + 2 * jj + (hj & 1)] = nm > 1 ? __fdiv_rn(s, (float)nm) : s;
       }
     }
     fence_proxy_async_smem();
@@ -284,7 +288,9 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
       // sub_cap entries that only its warp appends to, with the count in a register.
       const int q4 = warp & 3;
       const int grp_w = (warp - 2) >> 2;  // this warp's group within the item
-      const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+      // the key (TMEM lane within the quarter) whose score this thread ends up with
+      const int my_lane = (lane >> 2) + 8 * (lane & 1) + 16 * ((lane >> 1) & 1);
+
       const uint32_t need = (uint32_t)a.n_sel;
       const uint32_t gstride = (uint32_t)a.cap;    // 4 sub-buffers per group
       const uint32_t scap = (uint32_t)a.sub_cap;
@@ -326,30 +332,51 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
         float sc = 0.f;
         if (ok) {
           tc_fence_after();
-          const float4* wv = reinterpret_cast<const float4*>(&T.wbar[grp_w * H]);
-          float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                           make_float2(0.f, 0.f)};
+          // Eq. (5) for 4 keys x 16 heads per thread (two 16-lane slabs, 16x256b shape),
+          // then a reduce-scatter over the 4 threads of the quad: thread m ends with the
+          // full 64-head score of key m (slab m >> 1, lane kq + 8 (m & 1))
+          float2 w2[8];
 #pragma unroll
-          for (int h0 = 0; h0 < H; h0 += 32) {
-            uint32_t r[32];
-            tmem_ld32(tmem + lane_base + e_ab * 256u + (uint32_t)(grp_w * H + h0), r);
-            tmem_wait_ld();
-            if (h0 + 32 == H) {
-              tc_fence_before();
-              mbar_arrive(&T.acce[e_ab]);  // this warp's columns are in registers: the MMA may refill
-            }
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float4 w4 = wv[h0 / 4 + i];
-              const float2 x0 = make_float2(fmaxf(__uint_as_float(r[4 * i + 0]), 0.f),
-                                            fmaxf(__uint_as_float(r[4 * i + 1]), 0.f));
-              const float2 x1 = make_float2(fmaxf(__uint_as_float(r[4 * i + 2]), 0.f),
-                                            fmaxf(__uint_as_float(r[4 * i + 3]), 0.f));
-              acc[(2 * i) & 3] = __ffma2_rn(make_float2(w4.x, w4.y), x0, acc[(2 * i) & 3]);
-              acc[(2 * i + 1) & 3] = __ffma2_rn(make_float2(w4.z, w4.w), x1, acc[(2 * i + 1) & 3]);
-            }
+          for (int jj = 0; jj < 8; jj += 2) {
+            const float4 w4 = *reinterpret_cast<const float4*>(&T.wperm[(grp_w * 4 + (lane & 3)) * 20 + 2 * jj]);
+            w2[jj] = make_float2(w4.x, w4.y);
+            w2[jj + 1] = make_float2(w4.z, w4.w);
           }
-          sc = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+          float v[4];
+#pragma unroll
+          for (int slab = 0; slab < 2; ++slab) {
+            float2 a0 = make_float2(0.f, 0.f), a1 = a0, b0 = a0, b1 = a0;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              uint32_t r[16];
+              tmem_ld16x256b_x4(tmem + ((uint32_t)(q4 * 32 + slab * 16) << 16) + e_ab * 256u +
+                                    (uint32_t)(grp_w * H + 32 * half), r);
+              tmem_wait_ld();
+              if (slab == 1 && half == 1) {
+                tc_fence_before();
+                mbar_arrive(&T.acce[e_ab]);  // this warp's columns are in registers: the MMA may refill
+              }
+#pragma unroll
+              for (int jj = 0; jj < 4; jj += 2) {
+                const float2 wa = w2[4 * half + jj], wb = w2[4 * half + jj + 1];
+                a0 = __ffma2_rn(wa, make_float2(fmaxf(__uint_as_float(r[4 * jj + 0]), 0.f),
+                                                fmaxf(__uint_as_float(r[4 * jj + 1]), 0.f)), a0);
+                b0 = __ffma2_rn(wa, make_float2(fmaxf(__uint_as_float(r[4 * jj + 2]), 0.f),
+                                                fmaxf(__uint_as_float(r[4 * jj + 3]), 0.f)), b0);
+                a1 = __ffma2_rn(wb, make_float2(fmaxf(__uint_as_float(r[4 * jj + 4]), 0.f),
+                                                fmaxf(__uint_as_float(r[4 * jj + 5]), 0.f)), a1);
+                b1 = __ffma2_rn(wb, make_float2(fmaxf(__uint_as_float(r[4 * jj + 6]), 0.f),
+                                                fmaxf(__uint_as_float(r[4 * jj + 7]), 0.f)), b1);
+              }
+            }
+            v[2 * slab] = (a0.x + a0.y) + (a1.x + a1.y);
+            v[2 * slab + 1] = (b0.x + b0.y) + (b1.x + b1.y);
+          }
+          const bool x1 = (lane & 1) != 0, x2 = (lane & 2) != 0;
+          float k0 = x1 ? v[1] : v[0], k1 = x1 ? v[3] : v[2];  // keys with bit 0 == lane bit 0
+          k0 += __shfl_xor_sync(0xFFFFFFFFu, x1 ? v[0] : v[1], 1);
+          k1 += __shfl_xor_sync(0xFFFFFFFFu, x1 ? v[2] : v[3], 1);
+          sc = (x2 ? k1 : k0) + __shfl_xor_sync(0xFFFFFFFFu, x2 ? k0 : k1, 2);
         }
         if (++e_ab == 2) {
           e_ab = 0;
@@ -358,7 +385,7 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
         // streaming selection: append entries above the group's threshold
         bool near_full = false;
         if (ok && grp_w < nb_act) {
-          const int64_t s = s_begin + (int64_t)j * C::BM + q4 * 32 + lane;
+          const int64_t s = s_begin + (int64_t)j * C::BM + q4 * 32 + my_lane;
           const bool valid = (s < s_end) && (s <= e_r);
           const uint64_t p = pack_entry(score_key(sc), (uint32_t)s);
           const bool pass = valid && p > tau_r;
