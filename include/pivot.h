@@ -151,9 +151,16 @@ PIVOT_API const char *pivot_last_cuda_error(void);
 PIVOT_API int pivot_path(int op, int64_t L, int H, int d, int k, int c, int g, pivot_dtype dt);
 
 /* Bound (nanoseconds of wall-clock time) on every device-side wait; default
- * 2e9.  Test hook: flags bit 0 makes the scan kernel wait on a barrier that
- * nothing signals, so that the bound runs out and the timeout path is
- * exercised without hanging the GPU. */
+ * 2e9.  Test hooks (pivot_set_debug_flags, process-wide, 0 = normal):
+ *   bit 0 (1): the scan kernel waits on a barrier that nothing signals, so
+ *              the bound runs out and the timeout path is exercised without
+ *              hanging the GPU;
+ *   bit 1 (2): the scan visits key tiles in natural order (no sampled
+ *              threshold estimate);
+ *   bit 2 (4): the sampled estimate is taken at the sample's best entry, so
+ *              it is too high and every long work item is scanned a second
+ *              time (exercises the exact fallback).
+ * Results are identical under bits 1 and 2; only the work differs. */
 PIVOT_API void pivot_set_device_timeout_ns(uint64_t ns);
 PIVOT_API void pivot_set_debug_flags(int flags);
 

@@ -337,6 +337,38 @@ def test_decode_small_ragged(orc):
             assert len(a ^ b) <= 2, (row, len(a ^ b))
 
 
+# ---------------------------------------------------------------- scan visiting orders
+
+
+def test_sampled_order_natural_order_and_fallback_agree(orc):
+    """The scan's sampled threshold estimate (default), natural tile order (flag 2)
+    and a too-high estimate that forces every long item to be scanned again
+    (flag 4) select exactly the same sets; a few groups are also checked
+    against the oracle."""
+    L, topk, c, g = 16384, 256, 512, 8
+    x = inputs.random_prefill(L, 64, 128, inputs.BF16, seed=61, rho=0.9, heavy=0.02)
+    q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
+    runs = {}
+    try:
+        for flags in (0, 2, 4):
+            P.set_debug_flags(flags)
+            d_idx, _ = P.indexer_dense(q, w, k, topk)
+            u_idx, _ = P.reuse(q, w, k, topk, g)
+            r_idx, _, r_c, _ = P.refine(q, w, k, topk, c, g, cand=True)
+            torch.cuda.synchronize()
+            runs[flags] = [host(t) for t in (d_idx, u_idx, r_idx, r_c)]
+    finally:
+        P.set_debug_flags(0)
+    for flags in (2, 4):
+        for name, a0, a1 in zip(("dense", "reuse", "refine", "cand"), runs[0], runs[flags]):
+            assert np.array_equal(np.sort(a0, axis=1), np.sort(a1, axis=1)), \
+                f"{name}: flags {flags} differ from the sampled order"
+    G = (L + g - 1) // g
+    groups = [0, 1, G // 3, G - 2, G - 1]
+    fails = check_refine(orc, x, runs[0][2], None, runs[0][3], None, groups, topk, c, g)
+    assert not fails, summarize(fails)
+
+
 # ---------------------------------------------------------------- failure paths (no GPU fault)
 
 

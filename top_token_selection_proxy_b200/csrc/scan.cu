@@ -50,6 +50,21 @@ struct ScanCfg {
   static_assert(NB == 4, "four groups per item (H = 64)");
 };
 
+// Sample-first tile order: on the first attempt at a long item the tiles
+// 0, S, 2S, ... are scanned first (every entry admitted), the groups are cut
+// back to the best ~1.5 * n_sel * (sample share) of that sample, and the
+// remaining tiles are scanned with the resulting threshold.  The selection
+// stays exact: if fewer than n_sel entries end above the estimate, the item
+// is scanned again in natural order from an empty threshold.
+constexpr int kSampleStride = 32;
+
+// Key tile visited at step j of an item of ntiles tiles with ns sample tiles (ns = 0: natural order).
+__device__ __forceinline__ int tile_of(int j, int ns) {
+  if (ns == 0 || j < ns) return ns == 0 ? j : j * kSampleStride;
+  const int r = j - ns;  // the r-th tile that is not a sample tile
+  return (r / (kSampleStride - 1)) * kSampleStride + 1 + r % (kSampleStride - 1);
+}
+
 struct ScanTail {
   uint64_t full[4], empty[4], accf[2], acce[2];
   uint64_t never;  // a barrier nothing arrives on (forced-timeout test hook)
@@ -63,6 +78,8 @@ struct ScanTail {
   uint64_t tau[16];         // running admission threshold of each group (admit packed > tau)
   uint32_t qcnt[8][4];      // per group, entries in each lane quarter's sub-buffer (published on demand)
   uint32_t cflags;          // groups whose sub-buffers need a cut-back
+  int est[4];               // group got a sampled threshold estimate in this attempt
+  int retry;                // the attempt's estimate was too high: scan the item again
   uint32_t hist11[kHist11Words];    // radix-select histogram (11-bit digits)
   uint64_t bot[16];
   uint32_t nbot;
@@ -165,8 +182,12 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
           T.s_end = a.item_s1[item];
         }
         T.ntiles = (int)((T.s_end - T.s_begin + C::BM - 1) / C::BM);
-        for (int b = 0; b < C::NB; ++b) T.tau[b] = 0;
+        for (int b = 0; b < C::NB; ++b) {
+          T.tau[b] = 0;
+          T.est[b] = 0;
+        }
         T.cflags = 0;
+        T.retry = 0;
       }
     }
     __syncthreads();
@@ -225,6 +246,10 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
     fence_proxy_async_smem();
     __syncthreads();
 
+    for (int attempt = 0;; ++attempt) {
+    const int ns = (attempt == 0 && !(a.debug_flags & 2) && (int64_t)ntiles * C::BM >= 8 * (int64_t)a.n_sel)
+                       ? (ntiles + kSampleStride - 1) / kSampleStride
+                       : 0;
     if (warp == 0) {
       // ------------------------------------------------------------ TMA producer
       if (lane == 0) {
@@ -239,7 +264,8 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
           uint8_t* dst = sA + p_st * C::A_BYTES;
 #pragma unroll
           for (int kb = 0; kb < C::KB; ++kb)
-            tma_load_2d(dst + kb * (C::BM * 128), &kmap, &T.full[p_st], kb * 64, (int)(row0 + (int64_t)j * C::BM));
+            tma_load_2d(dst + kb * (C::BM * 128), &kmap, &T.full[p_st], kb * 64,
+                        (int)(row0 + (int64_t)tile_of(j, ns) * C::BM));
           if (++p_st == C::STAGES) {
             p_st = 0;
             p_ph ^= 1u;
@@ -305,19 +331,20 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
       };
       // cut group b back to a superset of its best `need` (keep <= maxk), every warp
       // of the group compacting its own sub-buffer in place
-      auto cut_back = [&](int b, uint32_t maxk) {
+      auto cut_back = [&](int b, uint32_t nd, uint32_t maxk) -> uint64_t {
         Segs sg;
         sg.cnt = 4;
         for (int q = 0; q < 4; ++q) {
           sg.p[q] = seg_of(b, q);
           sg.n[q] = T.qcnt[b][q];
         }
-        const uint64_t th = radix11_threshold<C::NEPI>(sg, need, maxk, T.hist11, T.sel, EG);
+        const uint64_t th = radix11_threshold<C::NEPI>(sg, nd, maxk, T.hist11, T.sel, EG);
         if (grp_w == b) {
           qcnt = warp_compact_ge(seg_of(b, q4), qcnt, th);
           if (th > 0) tau_r = th - 1ull;  // admit x >= th from now on
         }
         EG.sync();
+        return th;
       };
       for (int j = 0; j < ntiles; ++j) {
         bool ok;
@@ -385,7 +412,7 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
         // streaming selection: append entries above the group's threshold
         bool near_full = false;
         if (ok && grp_w < nb_act) {
-          const int64_t s = s_begin + (int64_t)j * C::BM + q4 * 32 + my_lane;
+          const int64_t s = s_begin + (int64_t)tile_of(j, ns) * C::BM + q4 * 32 + my_lane;
           const bool valid = (s < s_end) && (s <= e_r);
           const uint64_t p = pack_entry(score_key(sc), (uint32_t)s);
           const bool pass = valid && p > tau_r;
@@ -400,27 +427,48 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
         // consensus every 4 tiles (the same tiles for every epilogue thread, so all of them
         // execute the same barriers; a thread whose wait ran out fails its next waits fast
         // and reports the abort here): a warp adds at most 32 entries per tile to a sub-buffer
-        if (((j & 3) == 3 || j + 1 == ntiles) &&
-            named_bar_or(1, C::NEPI, near_full || T.abort_flag != 0)) {  // rare: abort or cut-back
-          if (named_bar_or(1, C::NEPI, T.abort_flag != 0)) break;         // uniform decision
+        const bool est_now = (j + 1 == ns);  // the sample is complete
+        if (((j & 3) == 3 || j + 1 == ntiles || est_now) &&
+            named_bar_or(1, C::NEPI, near_full || est_now || T.abort_flag != 0)) {  // rare
+          if (named_bar_or(1, C::NEPI, T.abort_flag != 0)) break;                   // uniform decision
           const uint32_t flags = T.cflags;
           publish_counts();
-          for (int b = 0; b < nb_act; ++b)
-            // keep at most sub_cap - 128 in total (>= need + 128 since sub_cap >= need + 256):
-            // then every sub-buffer has room for the 4 tiles until the next consensus
-            if (flags & (1u << b)) cut_back(b, scap - 128u);
+          for (int b = 0; b < nb_act; ++b) {
+            if (est_now) {
+              // keep the sample's best r0 (the sample's expected share of 1.5 * need, plus
+              // a margin); the threshold admits about 1.5 * need of the remaining keys
+              uint32_t r0 = (uint32_t)((3 * (int64_t)need * ns) / (2 * (int64_t)ntiles)) + 64u;
+              if (a.debug_flags & 4) r0 = 1;  // test hook: an estimate that is always too high
+              const uint64_t th = cut_back(b, r0, r0 + r0 / 4u);
+              if (EG.tid == 0) T.est[b] = th > 0 ? 1 : 0;
+            } else if (flags & (1u << b)) {
+              // keep at most sub_cap - 128 in total (>= need + 128 since sub_cap >= need + 256):
+              // then every sub-buffer has room for the 4 tiles until the next consensus
+              cut_back(b, need, scap - 128u);
+            }
+          }
           if (EG.tid == 0) T.cflags = 0;
           EG.sync();
         }
       }
       // ---------------------------------------------------------------- final exact selection + emit
+      if (EG.tid == 0) T.retry = 0;
       if (!named_bar_or(1, C::NEPI, T.abort_flag != 0)) {
         publish_counts();
+        // every entry left lies above the group's estimate (if it has one): with fewer
+        // than `need` of them the estimate was too high and the top-need is not complete
+        bool redo = false;
+        for (int b = 0; b < nb_act; ++b)
+          redo |= T.est[b] && (T.qcnt[b][0] + T.qcnt[b][1] + T.qcnt[b][2] + T.qcnt[b][3] < need);
+        if (redo && EG.tid == 0) {
+          T.retry = 1;
+          for (int b = 0; b < C::NB; ++b) T.est[b] = 0;
+        }
         uint64_t* sbuf = reinterpret_cast<uint64_t*>(sA);  // the stage ring is idle now
-        for (int b = 0; b < nb_act; ++b) {
+        for (int b = 0; b < (redo ? 0 : nb_act); ++b) {
           uint32_t n = T.qcnt[b][0] + T.qcnt[b][1] + T.qcnt[b][2] + T.qcnt[b][3];
           if (n > (uint32_t)C::SMEM_CAP) {  // rare: cut back to exactly `need` first
-            cut_back(b, need);
+            cut_back(b, need, need);
             publish_counts();
             n = T.qcnt[b][0] + T.qcnt[b][1] + T.qcnt[b][2] + T.qcnt[b][3];
           }
@@ -462,7 +510,11 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
         }
       }
     }
-    __syncthreads();  // item done: B, the stage ring and the select state are free
+    __syncthreads();  // attempt done: the stage ring and the select state are free
+    const bool again = T.retry != 0 && T.abort_flag == 0;
+    __syncthreads();
+    if (!again) break;
+    }  // attempts
   }
 
   __syncthreads();
