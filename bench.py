@@ -38,9 +38,9 @@ L2_FLUSH_BYTES = 256 << 20
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum); valid only while
 # the sources the scan kernel is built from hash to `sources_sha256`.
 SCAN_TRAFFIC = {
-    "bytes": 3.35e9 + 4.12e9,
+    "bytes": 2.78e9 + 1.65e9,
     "sources": ("scan.cu", "select.cuh", "ptx.cuh", "kernels.cuh"),
-    "sources_sha256": "6a8f91ad0a02e7c42a55fce3e70fc52245b026b4000edcf72cfb20936590727a",
+    "sources_sha256": "8455db8b267b93dbe025a7066c02542eedd04712edc95da759c2e550d7abcbe1",
     "profile": "profiles/dram_traffic_prefill_L131072_g8_refine.md",
 }
 

@@ -182,16 +182,6 @@ __device__ __forceinline__ void tmem_ld16x256b_x8(uint32_t taddr, uint32_t (&r)[
       : "r"(taddr));
 }
 
-// The same shape with 4 repetitions: 16 lanes x 32 columns, r[4j..4j+3] as above for j = 0..3.
-__device__ __forceinline__ void tmem_ld16x256b_x4(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-}
-
 // Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
 // 128 bytes, 8-row groups 1024 bytes apart (SBO), sm_100 descriptor version 1.
 __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {

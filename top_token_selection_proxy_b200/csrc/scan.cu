@@ -65,6 +65,26 @@ __device__ __forceinline__ int tile_of(int j, int ns) {
   return (r / (kSampleStride - 1)) * kSampleStride + 1 + r % (kSampleStride - 1);
 }
 
+// Eq. (5) partial sums of one 16x256b.x8 slab: sum over this thread's 16 heads of
+// w-bar_h * ReLU(x_h) for its two keys (lanes t/4 and t/4 + 8 of the slab).
+__device__ __forceinline__ void slab_head_sums(const uint32_t (&r)[32], const float2 (&w2)[8], float& ka,
+                                               float& kb) {
+  float2 a0 = make_float2(0.f, 0.f), a1 = a0, b0 = a0, b1 = a0;
+#pragma unroll
+  for (int jj = 0; jj < 8; jj += 2) {
+    a0 = __ffma2_rn(w2[jj], make_float2(fmaxf(__uint_as_float(r[4 * jj + 0]), 0.f),
+                                        fmaxf(__uint_as_float(r[4 * jj + 1]), 0.f)), a0);
+    b0 = __ffma2_rn(w2[jj], make_float2(fmaxf(__uint_as_float(r[4 * jj + 2]), 0.f),
+                                        fmaxf(__uint_as_float(r[4 * jj + 3]), 0.f)), b0);
+    a1 = __ffma2_rn(w2[jj + 1], make_float2(fmaxf(__uint_as_float(r[4 * jj + 4]), 0.f),
+                                            fmaxf(__uint_as_float(r[4 * jj + 5]), 0.f)), a1);
+    b1 = __ffma2_rn(w2[jj + 1], make_float2(fmaxf(__uint_as_float(r[4 * jj + 6]), 0.f),
+                                            fmaxf(__uint_as_float(r[4 * jj + 7]), 0.f)), b1);
+  }
+  ka = (a0.x + a0.y) + (a1.x + a1.y);
+  kb = (b0.x + b0.y) + (b1.x + b1.y);
+}
+
 struct ScanTail {
   uint64_t full[4], empty[4], accf[2], acce[2];
   uint64_t never;  // a barrier nothing arrives on (forced-timeout test hook)
@@ -209,13 +229,22 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
         for (int i = 0; i < 8; ++i) acc[i] = 0.f;
         const int nm = T.nmem[b];
         const int64_t r0 = T.mrow0[b];
-        for (int mm = 0; mm < nm; ++mm) {
-          const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.q + ((r0 + mm) * H + hj) * (int64_t)D) + xc);
-          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+        for (int m0 = 0; m0 < nm; m0 += 8) {  // 8 members' loads in flight, summed in member order
+          uint4 vv[8];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            acc[2 * i] += __uint_as_float(wv[i] << 16);
-            acc[2 * i + 1] += __uint_as_float(wv[i] & 0xFFFF0000u);
+          for (int u = 0; u < 8; ++u)
+            vv[u] = (m0 + u < nm) ? __ldg(reinterpret_cast<const uint4*>(a.q + ((r0 + m0 + u) * H + hj) * (int64_t)D) + xc)
+                                  : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            if (m0 + u < nm) {
+              const uint32_t wv[4] = {vv[u].x, vv[u].y, vv[u].z, vv[u].w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                acc[2 * i] += __uint_as_float(wv[i] << 16);
+                acc[2 * i + 1] += __uint_as_float(wv[i] & 0xFFFF0000u);
+              }
+            }
           }
         }
         uint32_t pk[4];
@@ -237,8 +266,13 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
         const int b = u / H, hj = u % H;
         const int nm = T.nmem[b];
         const int64_t r0 = T.mrow0[b];
+        float wl[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) wl[u] = (u < nm) ? __ldg(a.w + (r0 + u) * H + hj) : 0.f;
         float s = 0.f;
-        for (int mm = 0; mm < nm; ++mm) s += __ldg(a.w + (r0 + mm) * H + hj);
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+          if (u < nm) s += wl[u];
         const int jj = hj >> 3, m = (hj >> 1) & 3;
         T.wperm[(b * 4 + m) * 20 + 2 * jj + (hj & 1)] = nm > 1 ? __fdiv_rn(s, (float)nm) : s;
       }
@@ -372,32 +406,14 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
           float v[4];
 #pragma unroll
           for (int slab = 0; slab < 2; ++slab) {
-            float2 a0 = make_float2(0.f, 0.f), a1 = a0, b0 = a0, b1 = a0;
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              uint32_t r[16];
-              tmem_ld16x256b_x4(tmem + ((uint32_t)(q4 * 32 + slab * 16) << 16) + e_ab * 256u +
-                                    (uint32_t)(grp_w * H + 32 * half), r);
-              tmem_wait_ld();
-              if (slab == 1 && half == 1) {
-                tc_fence_before();
-                mbar_arrive(&T.acce[e_ab]);  // this warp's columns are in registers: the MMA may refill
-              }
-#pragma unroll
-              for (int jj = 0; jj < 4; jj += 2) {
-                const float2 wa = w2[4 * half + jj], wb = w2[4 * half + jj + 1];
-                a0 = __ffma2_rn(wa, make_float2(fmaxf(__uint_as_float(r[4 * jj + 0]), 0.f),
-                                                fmaxf(__uint_as_float(r[4 * jj + 1]), 0.f)), a0);
-                b0 = __ffma2_rn(wa, make_float2(fmaxf(__uint_as_float(r[4 * jj + 2]), 0.f),
-                                                fmaxf(__uint_as_float(r[4 * jj + 3]), 0.f)), b0);
-                a1 = __ffma2_rn(wb, make_float2(fmaxf(__uint_as_float(r[4 * jj + 4]), 0.f),
-                                                fmaxf(__uint_as_float(r[4 * jj + 5]), 0.f)), a1);
-                b1 = __ffma2_rn(wb, make_float2(fmaxf(__uint_as_float(r[4 * jj + 6]), 0.f),
-                                                fmaxf(__uint_as_float(r[4 * jj + 7]), 0.f)), b1);
-              }
+            uint32_t r[32];
+            tmem_ld16x256b_x8(tmem + ((uint32_t)(q4 * 32 + slab * 16) << 16) + e_ab * 256u + (uint32_t)(grp_w * H), r);
+            tmem_wait_ld();
+            if (slab == 1) {
+              tc_fence_before();
+              mbar_arrive(&T.acce[e_ab]);  // this warp's columns are in registers: the MMA may refill
             }
-            v[2 * slab] = (a0.x + a0.y) + (a1.x + a1.y);
-            v[2 * slab + 1] = (b0.x + b0.y) + (b1.x + b1.y);
+            slab_head_sums(r, w2, v[2 * slab], v[2 * slab + 1]);
           }
           const bool x1 = (lane & 1) != 0, x2 = (lane & 2) != 0;
           float k0 = x1 ? v[1] : v[0], k1 = x1 ? v[3] : v[2];  // keys with bit 0 == lane bit 0
