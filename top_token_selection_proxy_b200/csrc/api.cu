@@ -106,7 +106,7 @@ int sel_size(int op, int k, int c, int g) {
 }
 // per (group, lane quarter) sub-buffer of the scan kernel: room for a full
 // selection plus slack, so that cut-backs are rare; a group owns 4 of them
-int sel_sub_cap(int n_sel) { return (int)align_up((size_t)n_sel + 256, 64); }
+int sel_sub_cap(int n_sel) { return (int)align_up((size_t)n_sel + 384, 64); }
 int sel_cap(int n_sel) { return 4 * sel_sub_cap(n_sel); }
 
 struct Carve {

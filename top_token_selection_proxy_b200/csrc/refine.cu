@@ -10,17 +10,23 @@
 //
 // One persistent CTA per SM; a work item is (group, chunk of MC = 512/H
 // members).  Per item the members' query rows (MC*H rows x D, bf16) are the
-// MMA's B operand in shared memory (K-major, 128-byte swizzle).  Warps 5-7
-// gather 128 candidate key rows per tile with 16-byte cp.async into a
-// swizzled A tile (2-stage ring); warp 4 issues
+// MMA's B operand in shared memory (K-major, 128-byte swizzle), loaded by TMA.
+// Each 128-candidate A tile (3-stage ring) is gathered in two halves that
+// complete on the same barrier: rows 0-63 by TMA 4-row gathers (warp 17),
+// rows 64-127 by 16-byte cp.async into the same swizzled layout (warps 18-19,
+// one row per thread), so both the TMA and the load/store path have requests
+// in flight.  Warp 16 issues
 //     D[128 candidates x (members*H)] = K_gathered . Q_members^T
-// as up to two N=256 MMAs into two TMEM accumulators; warps 0-3 (one thread
-// per candidate lane) apply ReLU, weight each head by the member's own w and
-// sum the H heads per member in registers, then write the member's key row.
+// as up to two N=256 MMAs into two TMEM accumulators.  Warps 0-15 (one per
+// TMEM lane quarter and member of an accumulator half) read their member's 64
+// columns in the 16x256b shape, apply ReLU, weight each head by the member's
+// own w (16 weights per thread) and sum the heads across the thread quad, then
+// write the member's key row.
 #include <cuda_bf16.h>
 
 #include <cstddef>
 
+#include "headsum.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
 #include "select.cuh"
@@ -36,10 +42,15 @@ struct RefCfg {
   static constexpr int STAGES = 3;
   static constexpr int A_BYTES = BM * D * 2;
   static constexpr int B_BYTES = NROW * D * 2;
-  static constexpr int THREADS = 320;   // warps 0-7 epilogue, warp 8 MMA, warp 9 TMA gather
-  static constexpr int NEPI = 256;
+  // warps 0-15 epilogue (one per TMEM lane quarter and member of an accumulator
+  // half), 16 MMA, 17 TMA gather, 18-19 cp.async gather
+  static constexpr int THREADS = 640;
+  static constexpr int W_MMA = 16, W_TMA = 17, W_CPA = 18;
+  static constexpr int TMA_ROWS = 64;   // rows 0..63 of a tile by TMA gather, the rest by cp.async
+  static constexpr int NEPI = 512;
   static constexpr int MPH = 256 / H;   // members per accumulator half
-  static constexpr int MPW = MPH / 2;   // members per epilogue warp (two warps per TMEM lane quarter)
+  static_assert(MPH * 4 * 32 == NEPI, "one epilogue warp per (lane quarter, member of a half)");
+  static_assert(H == 64, "the epilogue reads 64 heads per member in the 16x256b.x8 shape");
 };
 
 struct RefTail {
@@ -49,9 +60,9 @@ struct RefTail {
   int item, nm, ntiles, nhalf, n_c;
   volatile int abort_flag;
   int64_t grp, key_base, qrow0, t0, orow0;
-  alignas(16) float w[512];  // read as float4
+  alignas(16) float wperm[8 * 4 * 20];  // members' w in the row-permuted layout of wperm_index
 };
-static_assert(offsetof(RefTail, w) % 16 == 0, "w must be 16-byte aligned");
+static_assert(offsetof(RefTail, wperm) % 16 == 0, "wperm must be 16-byte aligned");
 
 template <int H, int D>
 constexpr size_t refine_smem() {
@@ -60,7 +71,7 @@ constexpr size_t refine_smem() {
 }
 
 template <int H, int D>
-__global__ void __launch_bounds__(320, 1) refine_kernel(const __grid_constant__ CUtensorMap kmap,
+__global__ void __launch_bounds__(640, 1) refine_kernel(const __grid_constant__ CUtensorMap kmap,
                                                               const __grid_constant__ CUtensorMap qmap, const RefineArgs a,
                                                               uint32_t* __restrict__ out_keys) {
   using C = RefCfg<H, D>;
@@ -79,7 +90,7 @@ __global__ void __launch_bounds__(320, 1) refine_kernel(const __grid_constant__ 
 
   if (tid == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&T.full[s], 1);
+      mbar_init(&T.full[s], 1 + (C::BM - C::TMA_ROWS));  // TMA expect-tx arrive + one per cp.async row
       mbar_init(&T.empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -92,7 +103,7 @@ __global__ void __launch_bounds__(320, 1) refine_kernel(const __grid_constant__ 
     prefetch_tmap(&kmap);
     prefetch_tmap(&qmap);
   }
-  if (warp == 8) {
+  if (warp == C::W_MMA) {
     tmem_alloc(&T.tmem_slot, 512);
     tmem_relinquish();
   }
@@ -159,7 +170,7 @@ __global__ void __launch_bounds__(320, 1) refine_kernel(const __grid_constant__ 
           tma_load_2d(sB + kb * (C::NROW * 128) + hb * 256 * 128, &qmap, &T.bfull, kb * 64,
                       (int)(T.qrow0 * H + hb * 256));
     }
-    for (int u = tid; u < nm * H; u += C::THREADS) T.w[u] = __ldg(a.w + T.qrow0 * H + u);
+    for (int u = tid; u < nm * H; u += C::THREADS) T.wperm[wperm_index(u / H, u % H)] = __ldg(a.w + T.qrow0 * H + u);
     fence_proxy_async_smem();
     __syncthreads();
     if (nm == 0 || ntiles == 0) {
@@ -170,7 +181,7 @@ __global__ void __launch_bounds__(320, 1) refine_kernel(const __grid_constant__ 
     b_ph ^= 1u;
     (void)b_ph_item;
 
-    if (warp == 9) {
+    if (warp == C::W_TMA) {
       // ------------------------------------------------------------ TMA gather producer
       // lane l gathers candidate rows 4l..4l+3 of each 128-row tile: one 16-byte load of
       // their ids, then one 4-row gather per 64-column k-block (ids past n_c read row 0;
@@ -203,21 +214,71 @@ __global__ void __launch_bounds__(320, 1) refine_kernel(const __grid_constant__ 
           }
           break;
         }
-        if (lane == 0) mbar_arrive_expect_tx(&T.full[p_st], C::A_BYTES);
+        if (lane == 0) mbar_arrive_expect_tx(&T.full[p_st], (uint32_t)(C::TMA_ROWS * D * 2));
         __syncwarp();
         int row[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) row[u] = (int)(T.key_base + (id[u] >= 0 ? id[u] : 0));
         uint8_t* dst = sA + p_st * C::A_BYTES + (4 * lane) * 128;
+        if (4 * lane < C::TMA_ROWS) {
 #pragma unroll
-        for (int kb = 0; kb < C::KB; ++kb)
-          tma_gather4(dst + kb * (C::BM * 128), &kmap, &T.full[p_st], kb * 64, row[0], row[1], row[2], row[3]);
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_gather4(dst + kb * (C::BM * 128), &kmap, &T.full[p_st], kb * 64, row[0], row[1], row[2], row[3]);
+        }
         if (++p_st == C::STAGES) {
           p_st = 0;
           p_ph ^= 1u;
         }
       }
-    } else if (warp == 8) {
+    } else if (warp >= C::W_CPA) {
+      // ------------------------------------------------------------ cp.async gather producer
+      // thread u copies candidate row TMA_ROWS + u of each tile (16-byte chunks into the
+      // 128-byte-swizzled layout the TMA would produce); tile j's copies are committed as
+      // one group, and once the group of tile j-1 has landed the thread makes it visible
+      // to the tensor core (proxy fence) and arrives on that stage's full barrier
+      const int row = C::TMA_ROWS + (tid - 32 * C::W_CPA);
+      auto id_of = [&](int j) {
+        const int slot = j * C::BM + row;
+        const int id = (slot < n_c) ? __ldg(cand + slot) : -1;
+        return id >= 0 ? id : 0;  // slots without a candidate copy row 0 (masked later)
+      };
+      int idn = id_of(0);
+      uint32_t prev_st = 0;
+      bool pending = false;
+      for (int j = 0; j < ntiles; ++j) {
+        const int id = idn;
+        if (j + 1 < ntiles) idn = id_of(j + 1);
+        if (!mbar_wait(&T.empty[p_st], p_ph ^ 1u, a.timeout_ns, &T.abort_flag)) {
+          T.abort_flag = 1;
+          atomicOr(a.status, DEV_ERR_TIMEOUT);
+          break;
+        }
+        const uint16_t* src = a.k + (T.key_base + id) * (int64_t)D;
+        uint8_t* dst = sA + p_st * C::A_BYTES + row * 128;
+#pragma unroll
+        for (int kb = 0; kb < C::KB; ++kb)
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch)
+            cp_async_16(dst + kb * (C::BM * 128) + ((ch ^ (row & 7)) << 4), src + kb * 64 + ch * 8);
+        cp_async_commit();
+        if (pending) {
+          cp_async_wait<1>();
+          fence_proxy_async_smem();
+          mbar_arrive(&T.full[prev_st]);
+        }
+        pending = true;
+        prev_st = p_st;
+        if (++p_st == C::STAGES) {
+          p_st = 0;
+          p_ph ^= 1u;
+        }
+      }
+      if (pending) {
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        mbar_arrive(&T.full[prev_st]);
+      }
+    } else if (warp == C::W_MMA) {
       // ------------------------------------------------------------ MMA issuer
       if (lane == 0) {
         const uint32_t baddr = smem_u32(sB);
@@ -271,51 +332,38 @@ __global__ void __launch_bounds__(320, 1) refine_kernel(const __grid_constant__ 
       // ------------------------------------------------------------ epilogue (warps 0-7)
       // warp w reads TMEM lanes 32*(w%4).. (its candidates); the two warps of a
       // lane quarter split the members of each accumulator half.
+      // warp w reads TMEM lanes 32*(w%4).. (its candidates) and handles member w/4 of
+      // each accumulator half; 16x256b loads, 16 heads per thread, then the quad
+      // reduce-scatter leaves each thread with one candidate's score (lane my_lane)
       const int q4 = warp & 3;
-      const int part = warp >> 2;
-      const uint32_t lane_base = (uint32_t)(q4 * 32) << 16;
+      const int ml = warp >> 2;
+      const int my_lane = quad_key_lane(lane);
       bool stop = false;
       for (int j = 0; j < ntiles && !stop; ++j) {
-        const int slot = j * C::BM + q4 * 32 + lane;
+        const int slot = j * C::BM + q4 * 32 + my_lane;
         const int s = (slot < n_c) ? __ldg(cand + slot) : -1;
         for (int h = 0; h < nhalf; ++h) {
           const bool ok = mbar_wait(&T.accf[e_ab], e_aph, a.timeout_ns, &T.abort_flag);
-          float sc[C::MPW];
+          const int r = h * C::MPH + ml;  // member within the item
+          const bool mv = r < nm;          // uniform across the warp
+          float sc = 0.f;
           if (ok) {
             tc_fence_after();
-            uint32_t v[C::MPW][H];
+            float2 w2[8];
+            if (mv) load_w2(T.wperm, r, lane, w2);
+            float v[4];
 #pragma unroll
-            for (int mi = 0; mi < C::MPW; ++mi) {
-              const int ml = part * C::MPW + mi;
-              if (h * C::MPH + ml < nm) {
-#pragma unroll
-                for (int h0 = 0; h0 < H; h0 += 32)
-                  tmem_ld32(tmem + lane_base + e_ab * 256u + (uint32_t)(ml * H + h0),
-                            *reinterpret_cast<uint32_t(*)[32]>(&v[mi][h0]));
+            for (int slab = 0; slab < 2; ++slab) {
+              uint32_t rr[32];
+              tmem_ld16x256b_x8(tmem + ((uint32_t)(q4 * 32 + slab * 16) << 16) + e_ab * 256u + (uint32_t)(ml * H), rr);
+              tmem_wait_ld();
+              if (slab == 1) {
+                tc_fence_before();
+                mbar_arrive(&T.acce[e_ab]);  // accumulator copied: the MMA may refill it
               }
+              if (mv) slab_head_sums(rr, w2, v[2 * slab], v[2 * slab + 1]);
             }
-            tmem_wait_ld();
-            tc_fence_before();
-            mbar_arrive(&T.acce[e_ab]);  // accumulator copied: the MMA may refill it
-#pragma unroll
-            for (int mi = 0; mi < C::MPW; ++mi) {
-              const int r = h * C::MPH + part * C::MPW + mi;
-              float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
-              if (r < nm) {
-                const float4* wv = reinterpret_cast<const float4*>(&T.w[r * H]);
-#pragma unroll
-                for (int i = 0; i < H / 4; ++i) {
-                  const float4 w4 = wv[i];
-                  const float2 x0 = make_float2(fmaxf(__uint_as_float(v[mi][4 * i + 0]), 0.f),
-                                                fmaxf(__uint_as_float(v[mi][4 * i + 1]), 0.f));
-                  const float2 x1 = make_float2(fmaxf(__uint_as_float(v[mi][4 * i + 2]), 0.f),
-                                                fmaxf(__uint_as_float(v[mi][4 * i + 3]), 0.f));
-                  acc0 = __ffma2_rn(make_float2(w4.x, w4.y), x0, acc0);
-                  acc1 = __ffma2_rn(make_float2(w4.z, w4.w), x1, acc1);
-                }
-              }
-              sc[mi] = (acc0.x + acc0.y) + (acc1.x + acc1.y);
-            }
+            if (mv) sc = quad_reduce_scatter(v, lane);
           } else {
             T.abort_flag = 1;
             atomicOr(a.status, DEV_ERR_TIMEOUT);
@@ -329,16 +377,10 @@ __global__ void __launch_bounds__(320, 1) refine_kernel(const __grid_constant__ 
             break;
           }
           // Eq. (8) with the member's causal mask s <= t; key 0 marks "not eligible"
-          if (slot < a.c) {
-#pragma unroll
-            for (int mi = 0; mi < C::MPW; ++mi) {
-              const int r = h * C::MPH + part * C::MPW + mi;
-              if (r < nm) {
-                const int64_t t = T.t0 + r;
-                const bool valid = (s >= 0) && ((int64_t)s <= t);
-                out_keys[(T.orow0 + r) * (int64_t)a.c + slot] = valid ? score_key(sc[mi]) : 0u;
-              }
-            }
+          if (mv && slot < a.c) {
+            const int64_t t = T.t0 + r;
+            const bool valid = (s >= 0) && ((int64_t)s <= t);
+            out_keys[(T.orow0 + r) * (int64_t)a.c + slot] = valid ? score_key(sc) : 0u;
           }
         }
       }
@@ -352,7 +394,7 @@ __global__ void __launch_bounds__(320, 1) refine_kernel(const __grid_constant__ 
     while (globaltimer_ns() - t0 < 200000ull) {
     }
   }
-  if (warp == 8) tmem_dealloc(tmem, 512);
+  if (warp == C::W_MMA) tmem_dealloc(tmem, 512);
 }
 
 size_t refine_smem_bytes(int H, int D, int /*mc*/) {

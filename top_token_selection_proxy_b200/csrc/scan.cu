@@ -29,6 +29,7 @@
 
 #include <cstddef>
 
+#include "headsum.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
 #include "select.cuh"
@@ -63,26 +64,6 @@ __device__ __forceinline__ int tile_of(int j, int ns) {
   if (ns == 0 || j < ns) return ns == 0 ? j : j * kSampleStride;
   const int r = j - ns;  // the r-th tile that is not a sample tile
   return (r / (kSampleStride - 1)) * kSampleStride + 1 + r % (kSampleStride - 1);
-}
-
-// Eq. (5) partial sums of one 16x256b.x8 slab: sum over this thread's 16 heads of
-// w-bar_h * ReLU(x_h) for its two keys (lanes t/4 and t/4 + 8 of the slab).
-__device__ __forceinline__ void slab_head_sums(const uint32_t (&r)[32], const float2 (&w2)[8], float& ka,
-                                               float& kb) {
-  float2 a0 = make_float2(0.f, 0.f), a1 = a0, b0 = a0, b1 = a0;
-#pragma unroll
-  for (int jj = 0; jj < 8; jj += 2) {
-    a0 = __ffma2_rn(w2[jj], make_float2(fmaxf(__uint_as_float(r[4 * jj + 0]), 0.f),
-                                        fmaxf(__uint_as_float(r[4 * jj + 1]), 0.f)), a0);
-    b0 = __ffma2_rn(w2[jj], make_float2(fmaxf(__uint_as_float(r[4 * jj + 2]), 0.f),
-                                        fmaxf(__uint_as_float(r[4 * jj + 3]), 0.f)), b0);
-    a1 = __ffma2_rn(w2[jj + 1], make_float2(fmaxf(__uint_as_float(r[4 * jj + 4]), 0.f),
-                                            fmaxf(__uint_as_float(r[4 * jj + 5]), 0.f)), a1);
-    b1 = __ffma2_rn(w2[jj + 1], make_float2(fmaxf(__uint_as_float(r[4 * jj + 6]), 0.f),
-                                            fmaxf(__uint_as_float(r[4 * jj + 7]), 0.f)), b1);
-  }
-  ka = (a0.x + a0.y) + (a1.x + a1.y);
-  kb = (b0.x + b0.y) + (b1.x + b1.y);
 }
 
 struct ScanTail {
@@ -273,8 +254,7 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
 #pragma unroll
         for (int u = 0; u < 16; ++u)
           if (u < nm) s += wl[u];
-        const int jj = hj >> 3, m = (hj >> 1) & 3;
-        T.wperm[(b * 4 + m) * 20 + 2 * jj + (hj & 1)] = nm > 1 ? __fdiv_rn(s, (float)nm) : s;
+        T.wperm[wperm_index(b, hj)] = nm > 1 ? __fdiv_rn(s, (float)nm) : s;
       }
     }
     fence_proxy_async_smem();
@@ -349,7 +329,7 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
       const int q4 = warp & 3;
       const int grp_w = (warp - 2) >> 2;  // this warp's group within the item
       // the key (TMEM lane within the quarter) whose score this thread ends up with
-      const int my_lane = (lane >> 2) + 8 * (lane & 1) + 16 * ((lane >> 1) & 1);
+      const int my_lane = quad_key_lane(lane);
 
       const uint32_t need = (uint32_t)a.n_sel;
       const uint32_t gstride = (uint32_t)a.cap;    // 4 sub-buffers per group
@@ -397,12 +377,7 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
           // then a reduce-scatter over the 4 threads of the quad: thread m ends with the
           // full 64-head score of key m (slab m >> 1, lane kq + 8 (m & 1))
           float2 w2[8];
-#pragma unroll
-          for (int jj = 0; jj < 8; jj += 2) {
-            const float4 w4 = *reinterpret_cast<const float4*>(&T.wperm[(grp_w * 4 + (lane & 3)) * 20 + 2 * jj]);
-            w2[jj] = make_float2(w4.x, w4.y);
-            w2[jj + 1] = make_float2(w4.z, w4.w);
-          }
+          load_w2(T.wperm, grp_w, lane, w2);
           float v[4];
 #pragma unroll
           for (int slab = 0; slab < 2; ++slab) {
@@ -415,11 +390,7 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
             }
             slab_head_sums(r, w2, v[2 * slab], v[2 * slab + 1]);
           }
-          const bool x1 = (lane & 1) != 0, x2 = (lane & 2) != 0;
-          float k0 = x1 ? v[1] : v[0], k1 = x1 ? v[3] : v[2];  // keys with bit 0 == lane bit 0
-          k0 += __shfl_xor_sync(0xFFFFFFFFu, x1 ? v[0] : v[1], 1);
-          k1 += __shfl_xor_sync(0xFFFFFFFFu, x1 ? v[2] : v[3], 1);
-          sc = (x2 ? k1 : k0) + __shfl_xor_sync(0xFFFFFFFFu, x2 ? k0 : k1, 2);
+          sc = quad_reduce_scatter(v, lane);
         }
         if (++e_ab == 2) {
           e_ab = 0;
@@ -435,7 +406,7 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
           const uint32_t m = __ballot_sync(0xFFFFFFFFu, pass);
           if (pass) seg_of(grp_w, q4)[qcnt + __popc(m & lanemask_lt())] = p;
           qcnt += __popc(m);
-          if (qcnt > scap - 4u * 32u) {  // the next 4 tiles could overflow this sub-buffer
+          if (qcnt > scap - 8u * 32u) {  // the next 8 tiles could overflow this sub-buffer
             near_full = true;
             if (lane == 0) atomicOr(&T.cflags, 1u << grp_w);
           }
@@ -444,7 +415,7 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
         // execute the same barriers; a thread whose wait ran out fails its next waits fast
         // and reports the abort here): a warp adds at most 32 entries per tile to a sub-buffer
         const bool est_now = (j + 1 == ns);  // the sample is complete
-        if (((j & 3) == 3 || j + 1 == ntiles || est_now) &&
+        if (((j & 7) == 7 || j + 1 == ntiles || est_now) &&
             named_bar_or(1, C::NEPI, near_full || est_now || T.abort_flag != 0)) {  // rare
           if (named_bar_or(1, C::NEPI, T.abort_flag != 0)) break;                   // uniform decision
           const uint32_t flags = T.cflags;
@@ -460,7 +431,7 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
             } else if (flags & (1u << b)) {
               // keep at most sub_cap - 128 in total (>= need + 128 since sub_cap >= need + 256):
               // then every sub-buffer has room for the 4 tiles until the next consensus
-              cut_back(b, need, scap - 128u);
+              cut_back(b, need, scap - 256u);
             }
           }
           if (EG.tid == 0) T.cflags = 0;
