@@ -38,9 +38,9 @@ L2_FLUSH_BYTES = 256 << 20
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum); valid only while
 # the sources the scan kernel is built from hash to `sources_sha256`.
 SCAN_TRAFFIC = {
-    "bytes": 2.78e9 + 1.65e9,
-    "sources": ("scan.cu", "select.cuh", "ptx.cuh", "kernels.cuh"),
-    "sources_sha256": "8455db8b267b93dbe025a7066c02542eedd04712edc95da759c2e550d7abcbe1",
+    "bytes": 2.77e9 + 1.65e9,
+    "sources": ("scan.cu", "select.cuh", "ptx.cuh", "kernels.cuh", "headsum.cuh"),
+    "sources_sha256": "040d4fcbb2fa9ce889147effa01b0dac885389f25455717e3b19594988e29023",
     "profile": "profiles/dram_traffic_prefill_L131072_g8_refine.md",
 }
 
