@@ -18,6 +18,7 @@ JSON line with the max-over-ranks time.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -175,10 +176,9 @@ class Clocks:
 
 
 def dist_env():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return world, rank, local
+    from top_token_selection_proxy_b200 import multigpu
+
+    return multigpu.env()
 
 
 def to_dev(a, dev):
@@ -266,28 +266,23 @@ def main():
         return
     import numpy as np
     import torch
-    import torch.distributed as dist
 
     import top_token_selection_proxy_b200 as P
     from top_token_selection_proxy_b200 import build, inputs
+    from top_token_selection_proxy_b200 import multigpu as M
 
-    world, rank, local = dist_env()
-    if world > 1:
-        import datetime
-
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    world, rank, local = M.env()
+    M.init("nccl", world)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if rank == 0:
         build.build()
-    if world > 1:
-        dist.barrier()
+    M.barrier(world)
     P.lib()
 
     spec = inputs.LONG_128K
     # each rank indexes its own sequence (independent problems)
-    spec_r = spec if rank == 0 else inputs.PrefillSpec(spec.name, spec.L, spec.H, spec.d, spec.k, spec.c, spec.g,
-                                                        seed=spec.seed + 7919 * rank)
+    spec_r = dataclasses.replace(spec, seed=M.rank_seed(spec.seed, rank))
     x = inputs.make_prefill(spec_r)
     q, w, k = to_dev(x["q"], dev), to_dev(x["w"], dev), to_dev(x["k"], dev)
     ws = P.Workspace(dev)
@@ -301,15 +296,16 @@ def main():
     for _ in range(max(args.warmup, 0)):
         step()
     torch.cuda.synchronize()
-    if P.last_device_status(ws) != 0:
+    # every rank takes the same decision (a rank that left alone would strand the others at a barrier)
+    if M.max_over_ranks(1.0 if P.last_device_status(ws) != 0 else 0.0, world, dev) > 0:
+        M.finish(world)
         raise SystemExit("device status not OK after warm-up")
 
     clocks = Clocks(local)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     k_scan, k_ref, k_sel = [], [], []
-    if world > 1:
-        dist.barrier()
+    M.barrier(world)
     torch.cuda.synchronize()
     for i in range(args.steps):
         flush.fill_(i & 0xFF)  # write 256 MiB > L2 so each step starts cold
@@ -323,18 +319,11 @@ def main():
         k_ref.append(b)
         k_sel.append(c)
     torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    M.barrier(world)
     clk = clocks.stop()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    ms, value = M.weak_scaling(sum(step_ms), args.steps, spec.L, world, dev)
     status = P.last_device_status(ws)
-    ms = total_ms / args.steps
-    value = world * spec.L / (ms / 1000.0)
 
     extras = {}
     if not args.no_extras and rank == 0:
@@ -368,7 +357,8 @@ def main():
         del dq, dw, dk
 
     e2e = None
-    if not args.no_e2e and rank == 0:
+    M.barrier(world)  # every rank measures end to end (rank 0 arrives after its side measurements)
+    if not args.no_e2e:
         qh = torch.from_numpy(x["q"].view(np.int16)).pin_memory()
         wh = torch.from_numpy(x["w"]).pin_memory()
         kh = torch.from_numpy(x["k"].view(np.int16)).pin_memory()
@@ -394,15 +384,13 @@ def main():
             e2e_step()
         e1.record()
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1) / n
-        e2e = {"value": spec.L / (e_ms / 1000.0), "unit": UNIT, "ms_per_step": e_ms,
+        e_ms = M.max_over_ranks(e0.elapsed_time(e1) / n, world, dev)
+        e2e = {"value": world * spec.L / (e_ms / 1000.0), "unit": UNIT, "ms_per_step": e_ms,
                "h2d_bytes_per_step": int(qh.numel() * 2 + wh.numel() * 4 + kh.numel() * 2),
                "d2h_bytes_per_step": int(oh.numel() * 4), "host_buffers": "pinned"}
 
     if rank != 0:
-        if world > 1:
-            dist.barrier()
-            dist.destroy_process_group()
+        M.finish(world)
         return
 
     hbm, tf_burst, tf_sust, src = peaks()
@@ -440,9 +428,7 @@ def main():
     }
     line.update(extras)
     print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    M.finish(world)
 
 
 if __name__ == "__main__":
