@@ -474,9 +474,20 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
           EG.sync();
           uint64_t* buf = sbuf;
           // keep-all is th = 1, so the zero pads never survive; otherwise the need-th
-          // largest is a real entry (n_real > need)
-          const uint64_t th =
-              (n_real <= need) ? 1ull : radix11_threshold<C::NEPI>(buf, n, need, need, T.hist11, T.sel, EG);
+          // largest is a real entry (n_real > need), found within the entries' range
+          uint64_t th = 1ull;
+          if (n_real > need) {
+            uint64_t lo = ~0ull, hi = 0ull;
+            for (uint32_t i = EG.tid; i < n; i += C::NEPI) {
+              const uint64_t e = buf[i];
+              if (e != 0ull) {
+                lo = e < lo ? e : lo;
+                hi = e > hi ? e : hi;
+              }
+            }
+            group_minmax64<C::NEPI>(lo, hi, T.sel, EG);
+            th = radix11_threshold<C::NEPI>(buf, n, need, need, T.hist11, T.sel, EG, lo, hi);
+          }
           const uint32_t m = compact_ge<C::NEPI>(buf, buf, n, th, T.sel, EG);
           const int64_t grp = T.grp0 + b;
           if (a.mode == EMIT_DENSE) {

@@ -166,6 +166,33 @@ __device__ uint64_t radix_threshold(const uint64_t* buf, uint32_t n, uint32_t ne
   return prefix;
 }
 
+// Block-wide min and max of 64-bit values (every thread of G calls; all get the result).
+template <int NT>
+__device__ __forceinline__ void group_minmax64(uint64_t& lo, uint64_t& hi, SelSmem& S, const Group<NT>& G) {
+  static_assert(NT / 32 <= 64, "at most 64 warps");
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint64_t l2 = __shfl_xor_sync(0xFFFFFFFFu, lo, o), h2 = __shfl_xor_sync(0xFFFFFFFFu, hi, o);
+    lo = l2 < lo ? l2 : lo;
+    hi = h2 > hi ? h2 : hi;
+  }
+  uint64_t* sc = reinterpret_cast<uint64_t*>(S.hist);  // 128 x uint64 of scratch
+  const int w = G.tid >> 5;
+  if ((G.tid & 31) == 0) {
+    sc[w] = lo;
+    sc[64 + w] = hi;
+  }
+  G.sync();
+  lo = sc[0];
+  hi = sc[64];
+#pragma unroll
+  for (int i = 1; i < NT / 32; ++i) {
+    lo = sc[i] < lo ? sc[i] : lo;
+    hi = sc[64 + i] > hi ? sc[64 + i] : hi;
+  }
+  G.sync();
+}
+
 // Up to 4 disjoint segments of packed entries, read as one set.
 struct Segs {
   const uint64_t* p[4];
@@ -321,33 +348,36 @@ __device__ __forceinline__ uint32_t group_offsets(uint32_t cnt, uint32_t* total,
 }
 
 // ---------------------------------------------------------------- 11-bit digits
-// Digit widths of the 64-bit packed entry, most significant first.
-__host__ __device__ constexpr int r11_width(int d) { return d < 5 ? 11 : 9; }
 
 // The 2048-bin histogram is stored with one pad word after every 32 bins, so
 // the digit search (thread t reads bins BPT*t .. BPT*t + BPT-1, BPT = 4 or 8)
 // hits 32 distinct banks per warp instead of 32 / BPT.
 constexpr int kHist11Words = 2048 + 64;
 __device__ __forceinline__ uint32_t h11(uint32_t bin) { return bin + (bin >> 5); }
-__host__ __device__ constexpr int r11_shift(int d) { return 64 - 11 * (d + 1) < 0 ? 0 : 64 - 11 * (d + 1); }
 
 // Like radix_threshold, with 11-bit digits (at most 6 passes, usually 2) and a
 // 2048-bin shared-memory histogram `hist` (kHist11Words words, padded layout)
 // updated with plain atomics.  The
 // entries are the union of the segments of sg.
+// When [lo, hi] is given (lo <= every entry that can be selected, hi >= every
+// entry, at least `need` entries inside), the digits start below the bits lo
+// and hi share: for scores packed from a narrow range that skips the sign and
+// exponent bits that all of them have in common, so one or two passes suffice.
 template <int NT>
 __device__ uint64_t radix11_threshold(const Segs& sg, uint32_t need, uint32_t max_keep, uint32_t* hist,
-                                      SelSmem& S, const Group<NT>& G) {
+                                      SelSmem& S, const Group<NT>& G, uint64_t lo = 0ull,
+                                      uint64_t hi = ~0ull) {
   static_assert(2048 % NT == 0, "NT must divide 2048");
   constexpr int BPT = 2048 / NT;  // bins per thread in the digit search
   uint32_t n = 0;
   for (int i = 0; i < sg.cnt; ++i) n += sg.n[i];
   if (n <= max_keep) return 0ull;
-  uint64_t prefix = 0;
+  int consumed = (lo == hi) ? 64 : __clzll(lo ^ hi);  // bits every entry of interest shares
+  if (consumed == 64) return lo;
+  uint64_t prefix = consumed ? (hi >> (64 - consumed)) : 0ull;
   uint32_t above = 0;
-  int consumed = 0;
-  for (int d = 0; d < 6; ++d) {
-    const int w = r11_width(d), shift = r11_shift(d);
+  while (consumed < 64) {
+    const int w = (64 - consumed) < 11 ? (64 - consumed) : 11, shift = 64 - consumed - w;
     const uint32_t nb = 1u << w;
     for (uint32_t i = G.tid; i < (uint32_t)kHist11Words; i += NT) hist[i] = 0u;
     G.sync();
@@ -395,12 +425,13 @@ __device__ uint64_t radix11_threshold(const Segs& sg, uint32_t need, uint32_t ma
 template <int NT>
 __device__ __forceinline__ uint64_t radix11_threshold(const uint64_t* buf, uint32_t n, uint32_t need,
                                                       uint32_t max_keep, uint32_t* hist, SelSmem& S,
-                                                      const Group<NT>& G) {
+                                                      const Group<NT>& G, uint64_t lo = 0ull,
+                                                      uint64_t hi = ~0ull) {
   Segs sg;
   sg.cnt = 1;
   sg.p[0] = buf;
   sg.n[0] = n;
-  return radix11_threshold<NT>(sg, need, max_keep, hist, S, G);
+  return radix11_threshold<NT>(sg, need, max_keep, hist, S, G, lo, hi);
 }
 
 // Stream-compact the entries >= T of src[0..n) into dst[0..m) (dst may be
