@@ -411,7 +411,7 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
             if (lane == 0) atomicOr(&T.cflags, 1u << grp_w);
           }
         }
-        // consensus every 4 tiles (the same tiles for every epilogue thread, so all of them
+        // consensus every 8 tiles (the same tiles for every epilogue thread, so all of them
         // execute the same barriers; a thread whose wait ran out fails its next waits fast
         // and reports the abort here): a warp adds at most 32 entries per tile to a sub-buffer
         const bool est_now = (j + 1 == ns);  // the sample is complete
