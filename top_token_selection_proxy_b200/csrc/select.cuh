@@ -200,64 +200,6 @@ struct Segs {
   int cnt;
 };
 
-// radix_threshold over the union of the segments (no first-digit histogram).
-template <int NT>
-__device__ uint64_t radix_threshold_segs(const Segs& sg, uint32_t need, uint32_t max_keep, SelSmem& S,
-                                         const Group<NT>& G) {
-  uint32_t n = 0;
-  for (int i = 0; i < sg.cnt; ++i) n += sg.n[i];
-  if (n <= max_keep) return 0ull;
-  uint64_t prefix = 0;
-  uint32_t above = 0;
-  for (int shift = 56; shift >= 0; shift -= 8) {
-    for (int i = G.tid; i < 256; i += NT) S.hist[i] = 0u;
-    G.sync();
-    for (int sgi = 0; sgi < sg.cnt; ++sgi)
-      visit_entries<NT, 8>(sg.p[sgi], sg.n[sgi], G, [&](uint64_t x, bool valid) {
-        const bool match = valid && (shift == 56 || (x >> (shift + 8)) == prefix);
-        hist_add(S.hist, match ? ((uint32_t)(x >> shift) & 255u) : 256u);
-      });
-    G.sync();
-    if (G.tid < 32) {
-      const int l = G.tid;
-      uint32_t loc[8], sum = 0;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        loc[u] = S.hist[255 - 8 * l - u];
-        sum += loc[u];
-      }
-      uint32_t incl = sum;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (l >= o) incl += v;
-      }
-      const uint32_t excl = incl - sum;
-      if (above + excl < need && need <= above + incl) {
-        uint32_t c = above + excl;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          if (c + loc[u] >= need) {
-            S.scal[0] = 255u - 8u * l - u;
-            S.scal[1] = c;
-            S.scal[2] = loc[u];
-            break;
-          }
-          c += loc[u];
-        }
-      }
-    }
-    G.sync();
-    const uint32_t digit = S.scal[0];
-    above = S.scal[1];
-    const uint32_t h = S.scal[2];
-    prefix = (prefix << 8) | digit;
-    G.sync();
-    if (above + h <= max_keep || shift == 0) return prefix << shift;
-  }
-  return prefix;
-}
-
 // One warp keeps the entries >= T of seg[0..n) in place; returns the new count.
 // seg must be 16-byte aligned; 2*V entries per lane are in flight per chunk.
 __device__ __forceinline__ uint32_t warp_compact_ge(uint64_t* seg, uint32_t n, uint64_t T) {
@@ -471,17 +413,6 @@ __device__ uint32_t compact_ge(const uint64_t* src, uint64_t* dst, uint32_t n, u
     G.sync();
   }
   return base;
-}
-
-// Count entries of buf[0..n) with index <= t (all threads get the total).
-template <int NT>
-__device__ uint32_t count_idx_le(const uint64_t* buf, uint32_t n, uint32_t t, SelSmem& S, const Group<NT>& G) {
-  uint32_t c = 0;
-  for (uint32_t i = G.tid; i < n; i += NT) c += (entry_idx(buf[i]) <= t) ? 1u : 0u;
-  uint32_t total;
-  group_offsets<NT>(c, &total, S, G);
-  G.sync();
-  return total;
 }
 
 // Write the indices (and optionally scores) of the entries of buf[0..n) that
