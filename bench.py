@@ -355,6 +355,18 @@ def main():
         extras["decode"] = {"workload": ds.name, "refine_ms": dref, "reuse_ms": dreu,
                             "key_bytes": key_bytes, "refine_hbm_frac": key_bytes / (dref * 1e-3) / (hbm * 1e9)}
         del dq, dw, dk
+        # guardrail: the guarded Refine call against both of its paths on short prefills
+        guard = []
+        for gs in (inputs.PREFILL_8K, dataclasses.replace(inputs.PREFILL_8K, name="prefill_L3072_g8", L=3072)):
+            xg = inputs.make_prefill(gs)
+            gq, gw, gk = to_dev(xg["q"], dev), to_dev(xg["w"], dev), to_dev(xg["k"], dev)
+            g_ref = timed(lambda: P.refine(gq, gw, gk, gs.k, gs.c, gs.g, ws=ws))
+            g_den = timed(lambda: P.indexer_dense(gq, gw, gk, gs.k, ws=ws))
+            g_grd = timed(lambda: P.refine_guarded(gq, gw, gk, gs.k, gs.c, gs.g, ws=ws))
+            guard.append({"workload": gs.name, "path": "dense" if P.guardrail_dense(P.OP_REFINE, gs.L, gs.c, gs.g)
+                          else "refine", "guarded_ms": g_grd, "refine_ms": g_ref, "dense_ms": g_den})
+            del gq, gw, gk
+        extras["guardrail"] = guard
 
     e2e = None
     M.barrier(world)  # every rank measures end to end (rank 0 arrives after its side measurements)

@@ -109,6 +109,33 @@ PIVOT_API pivot_status pivot_refine(const void *q_I, const float *w_I, const voi
                           int32_t *cand_opt, float *cand_scores_opt, void *ws, size_t ws_bytes,
                           pivot_stream_t stream);
 
+/* Guardrail (PIVOT paper, "Efficiency Results (Figure 4)": PIVOT falls back to
+ * dense DSA at short context to avoid overhead).  The pages give no criterion;
+ * this library uses the work model of the prefill call, in key-row products
+ * q.k (each 2*H*d FLOPs):
+ *   dense  sum_t (t + 1) = L (L + 1) / 2
+ *   Reuse  sum_i P_i                            (the proxy scan, Eq. 5)
+ *   Refine sum_i (P_i + |G_i| * min(c, P_i))    (scan + re-scoring, Eq. 5, 8)
+ * with groups G_i of g consecutive positions and P_i = the group's end + 1.
+ * Returns 1 when dense needs no more work than op (PIVOT_OP_REUSE or
+ * PIVOT_OP_REFINE), 0 when the PIVOT variant is cheaper, -1 for invalid
+ * arguments (L < 1, g < 1, c < 1 for Refine, other ops). */
+PIVOT_API int pivot_guardrail_dense(int op, int64_t L, int c, int g);
+
+/* pivot_reuse / pivot_refine behind the guardrail: when pivot_guardrail_dense
+ * returns 1 the call runs pivot_indexer_dense instead (indices and scores_opt
+ * then hold the dense rows; cand_opt and cand_scores_opt are not written).
+ * *path_out (host pointer, may be NULL) receives 1 for dense, 0 for PIVOT.
+ * ws_bytes must cover the path taken: pivot_workspace_size of PIVOT_OP_DENSE
+ * or of op, as pivot_guardrail_dense says. */
+PIVOT_API pivot_status pivot_reuse_guarded(const void *q_I, const float *w_I, const void *k_I, int64_t L, int H,
+                                           int d, pivot_dtype dt, int k, int g, int32_t *indices, float *scores_opt,
+                                           void *ws, size_t ws_bytes, pivot_stream_t stream, int *path_out);
+PIVOT_API pivot_status pivot_refine_guarded(const void *q_I, const float *w_I, const void *k_I, int64_t L, int H,
+                                            int d, pivot_dtype dt, int k, int c, int g, int32_t *indices,
+                                            float *scores_opt, int32_t *cand_opt, float *cand_scores_opt, void *ws,
+                                            size_t ws_bytes, pivot_stream_t stream, int *path_out);
+
 /* Workspace bytes for the decode calls below.  key_offsets_host [B+1] is the
  * host copy of the key offsets (key_offsets_host[0] = 0, non-decreasing,
  * every P_b = key_offsets_host[b+1] - key_offsets_host[b] >= g). */

@@ -75,3 +75,34 @@ def test_workspace_too_small_rejected(lib):
     ptr = ctypes.c_void_p((ctypes.addressof(buf) + 15) // 16 * 16)
     st = lib.pivot_reuse(ptr, ptr, ptr, 1024, 64, 128, 0, 16, 4, ptr, None, ptr, 256, None)
     assert st == 3
+
+
+# ---------------------------------------------------------------- guardrail decision (host logic)
+
+
+def test_guardrail_decision():
+    g_dense = P.lib().pivot_guardrail_dense
+    # Reuse scans sum_i P_i keys: less than dense's L(L+1)/2 for any g >= 2; equal at g = 1
+    for L in (1, 2, 100, 8192, 131072):
+        assert g_dense(P.OP_REUSE, L, 16, 1) == 1
+    for L in (2, 100, 8192, 131072):
+        for g in (2, 4, 8, 16):
+            assert g_dense(P.OP_REUSE, L, 16, g) == 0
+    # Refine at L = 8192, g = 8, c = 4096, worked by hand: dense 8192*8193/2 = 33,558,528 key-row
+    # products; scan 8*(1+...+1024) = 4,198,400; re-scoring 8*[8*(1+...+512) + 512*4096] =
+    # 25,182,208; Refine total 29,380,608 < dense, so Refine is kept
+    assert g_dense(P.OP_REFINE, 8192, 4096, 8) == 0
+    # c >= L: every candidate set is the whole prefix, Refine only adds the scan to dense's work
+    assert g_dense(P.OP_REFINE, 4096, 4096, 8) == 1
+    assert g_dense(P.OP_REFINE, 3000, 4096, 8) == 1
+    # long context: Refine's work grows like L*c, dense like L^2
+    assert g_dense(P.OP_REFINE, 131072, 4096, 8) == 0
+    # the choice flips once, from dense to Refine, as L grows (g = 8, c = 4096)
+    picks = [g_dense(P.OP_REFINE, L, 4096, 8) for L in range(1000, 20000, 250)]
+    flips = sum(1 for a, b in zip(picks, picks[1:]) if a != b)
+    assert picks[0] == 1 and picks[-1] == 0 and flips == 1
+    # invalid arguments
+    assert g_dense(P.OP_DENSE, 100, 16, 8) == -1
+    assert g_dense(P.OP_REFINE, 0, 16, 8) == -1
+    assert g_dense(P.OP_REFINE, 100, 0, 8) == -1
+    assert g_dense(P.OP_REUSE, 100, 16, 0) == -1

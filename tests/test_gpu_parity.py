@@ -369,6 +369,34 @@ def test_sampled_order_natural_order_and_fallback_agree(orc):
     assert not fails, summarize(fails)
 
 
+# ---------------------------------------------------------------- guardrail
+
+
+def test_guardrail_runs_the_chosen_path_exactly():
+    """Behind the guardrail the call returns exactly the rows of the path it picks:
+    dense at short context (c >= L), Refine / Reuse otherwise."""
+    g, c, topk = 8, 512, 256
+    for L, want_dense in ((400, True), (4096, False)):
+        x = inputs.random_prefill(L, 64, 128, inputs.BF16, seed=40 + L)
+        q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
+        assert P.guardrail_dense(P.OP_REFINE, L, c, g) == want_dense
+        gi, gs, ran_dense = P.refine_guarded(q, w, k, topk, c, g, scores=True)
+        assert ran_dense == want_dense
+        ri, rs = P.indexer_dense(q, w, k, topk, scores=True) if want_dense else \
+            P.refine(q, w, k, topk, c, g, scores=True)[:2]
+        torch.cuda.synchronize()
+        assert np.array_equal(np.sort(host(gi), axis=1), np.sort(host(ri), axis=1))
+        ui, _, ran_dense_u = P.reuse_guarded(q, w, k, topk, g)
+        assert not ran_dense_u
+        assert np.array_equal(np.sort(host(ui), axis=1), np.sort(host(P.reuse(q, w, k, topk, g)[0]), axis=1))
+    # g = 1: Reuse and dense do the same work, the guardrail runs dense
+    x = inputs.random_prefill(300, 64, 128, inputs.BF16, seed=41)
+    q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
+    ui, _, ran_dense_u = P.reuse_guarded(q, w, k, 64, 1)
+    assert ran_dense_u
+    assert np.array_equal(np.sort(host(ui), axis=1), np.sort(host(P.indexer_dense(q, w, k, 64)[0]), axis=1))
+
+
 # ---------------------------------------------------------------- failure paths (no GPU fault)
 
 

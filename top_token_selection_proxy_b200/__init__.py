@@ -41,7 +41,7 @@ EXPORTS = (
     "pivot_varlen_workspace_size", "pivot_reuse_varlen", "pivot_refine_varlen",
     "pivot_last_device_status", "pivot_status_string", "pivot_last_cuda_error", "pivot_path",
     "pivot_set_device_timeout_ns", "pivot_set_debug_flags", "pivot_set_profile_events", "pivot_version",
-    "pivot_reuse_noalloc",
+    "pivot_reuse_noalloc", "pivot_guardrail_dense", "pivot_reuse_guarded", "pivot_refine_guarded",
 )
 
 
@@ -72,8 +72,13 @@ def lib() -> ctypes.CDLL:
         L.pivot_refine.argtypes = [P, P, P, I64, I, I, I, I, I, I, P, P, P, P, P, SZ, P]
         L.pivot_reuse_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P]
         L.pivot_refine_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P, SZ, P]
+        L.pivot_guardrail_dense.argtypes = [I, I64, I, I]
+        L.pivot_guardrail_dense.restype = I
+        L.pivot_reuse_guarded.argtypes = [P, P, P, I64, I, I, I, I, I, P, P, P, SZ, P, P]
+        L.pivot_refine_guarded.argtypes = [P, P, P, I64, I, I, I, I, I, I, P, P, P, P, P, SZ, P, P]
         for f in ("pivot_indexer_dense", "pivot_reuse", "pivot_refine", "pivot_reuse_varlen",
-                  "pivot_refine_varlen", "pivot_last_device_status"):
+                  "pivot_refine_varlen", "pivot_last_device_status", "pivot_reuse_guarded",
+                  "pivot_refine_guarded"):
             getattr(L, f).restype = I
         L.pivot_last_device_status.argtypes = [P, P]
         L.pivot_status_string.argtypes = [I]
@@ -218,6 +223,46 @@ def refine(q, w, k, topk: int, c: int, g: int, *, scores: bool = False, cand=Fal
     return idx, sc, cd, cs
 
 
+def guardrail_dense(op: int, L: int, c: int, g: int) -> bool:
+    """The guardrail's choice (PIVOT paper, Efficiency Results, Figure 4): True when the
+    dense indexer needs no more work than op (OP_REUSE or OP_REFINE) on a prefill of L."""
+    r = lib().pivot_guardrail_dense(op, L, c, g)
+    if r < 0:
+        raise ValueError("invalid guardrail arguments")
+    return bool(r)
+
+
+def reuse_guarded(q, w, k, topk: int, g: int, *, scores: bool = False, ws: Optional[Workspace] = None,
+                  stream=None):
+    """PIVOT-Reuse behind the guardrail.  Returns (indices, scores|None, ran_dense)."""
+    L, H, d, dt = _prefill_common(q, w, k)
+    idx = torch.empty((L, topk), dtype=torch.int32, device=q.device)
+    sc = torch.empty((L, topk), dtype=torch.float32, device=q.device) if scores else None
+    dense = guardrail_dense(OP_REUSE, L, topk, g)
+    nbytes = workspace_size(OP_DENSE if dense else OP_REUSE, L, H, d, topk, topk, g, dt)
+    W = _ws_for(ws, q.device).get(nbytes)
+    path = ctypes.c_int(-1)
+    _check(lib().pivot_reuse_guarded(_ptr(q), _ptr(w), _ptr(k), L, H, d, dt, topk, g, _ptr(idx), _ptr(sc), _ptr(W),
+                                     W.numel(), _stream(stream), ctypes.byref(path)), "pivot_reuse_guarded")
+    return idx, sc, path.value == 1
+
+
+def refine_guarded(q, w, k, topk: int, c: int, g: int, *, scores: bool = False, ws: Optional[Workspace] = None,
+                   stream=None):
+    """PIVOT-Refine behind the guardrail.  Returns (indices, scores|None, ran_dense)."""
+    L, H, d, dt = _prefill_common(q, w, k)
+    idx = torch.empty((L, topk), dtype=torch.int32, device=q.device)
+    sc = torch.empty((L, topk), dtype=torch.float32, device=q.device) if scores else None
+    dense = guardrail_dense(OP_REFINE, L, c, g)
+    nbytes = workspace_size(OP_DENSE if dense else OP_REFINE, L, H, d, topk, c, g, dt)
+    W = _ws_for(ws, q.device).get(nbytes)
+    path = ctypes.c_int(-1)
+    _check(lib().pivot_refine_guarded(_ptr(q), _ptr(w), _ptr(k), L, H, d, dt, topk, c, g, _ptr(idx), _ptr(sc), None,
+                                      None, _ptr(W), W.numel(), _stream(stream), ctypes.byref(path)),
+           "pivot_refine_guarded")
+    return idx, sc, path.value == 1
+
+
 def _varlen_common(q, w, kc, offsets, g):
     _need_cuda(q, w, kc)
     off_h = torch.as_tensor(offsets, dtype=torch.int64).cpu().contiguous()
@@ -299,5 +344,6 @@ class KernelTimer:
 __all__ = [
     "lib", "LIB_PATH", "EXPORTS", "PivotError", "Workspace", "workspace_size", "varlen_workspace_size", "path",
     "indexer_dense", "reuse", "refine", "reuse_varlen", "refine_varlen", "last_device_status",
+    "guardrail_dense", "reuse_guarded", "refine_guarded",
     "set_device_timeout_ns", "set_debug_flags", "KernelTimer", "OP_DENSE", "OP_REUSE", "OP_REFINE", "BF16", "F32", "STATUS",
 ]

@@ -601,6 +601,45 @@ void pivot_set_profile_events(void** events, int n) {
   for (int i = 0; i < 4; ++i)
     g_prof[i] = (events && n >= 4) ? reinterpret_cast<cudaEvent_t>(events[i]) : nullptr;
 }
+// Guardrail work model (see pivot.h): key-row products of each path.
+int pivot_guardrail_dense(int op, int64_t L, int c, int g) {
+  if (L < 1 || g < 1 || (op != PIVOT_OP_REUSE && op != PIVOT_OP_REFINE) || (op == PIVOT_OP_REFINE && c < 1))
+    return -1;
+  const double dense = 0.5 * (double)L * (double)(L + 1);
+  double pivot = 0.0;
+  for (int64_t t0 = 0; t0 < L; t0 += g) {
+    const int64_t t1 = std::min<int64_t>(t0 + g, L);
+    const double P = (double)t1;  // the group's prefix: keys 0 .. group end
+    pivot += P;
+    if (op == PIVOT_OP_REFINE) pivot += (double)(t1 - t0) * std::min<double>((double)c, P);
+  }
+  return dense <= pivot ? 1 : 0;
+}
+
+pivot_status pivot_reuse_guarded(const void* q_I, const float* w_I, const void* k_I, int64_t L, int H, int d,
+                                 pivot_dtype dt, int k, int g, int32_t* indices, float* scores_opt, void* ws,
+                                 size_t ws_bytes, pivot_stream_t stream, int* path_out) {
+  const int use_dense = pivot_guardrail_dense(PIVOT_OP_REUSE, L, k, g);
+  if (use_dense < 0) return PIVOT_ERR_INVALID_ARG;
+  if (path_out) *path_out = use_dense;
+  if (use_dense)
+    return pivot_indexer_dense(q_I, w_I, k_I, L, H, d, dt, k, indices, scores_opt, ws, ws_bytes, stream);
+  return pivot_reuse(q_I, w_I, k_I, L, H, d, dt, k, g, indices, scores_opt, ws, ws_bytes, stream);
+}
+
+pivot_status pivot_refine_guarded(const void* q_I, const float* w_I, const void* k_I, int64_t L, int H, int d,
+                                  pivot_dtype dt, int k, int c, int g, int32_t* indices, float* scores_opt,
+                                  int32_t* cand_opt, float* cand_scores_opt, void* ws, size_t ws_bytes,
+                                  pivot_stream_t stream, int* path_out) {
+  const int use_dense = pivot_guardrail_dense(PIVOT_OP_REFINE, L, c, g);
+  if (use_dense < 0) return PIVOT_ERR_INVALID_ARG;
+  if (path_out) *path_out = use_dense;
+  if (use_dense)
+    return pivot_indexer_dense(q_I, w_I, k_I, L, H, d, dt, k, indices, scores_opt, ws, ws_bytes, stream);
+  return pivot_refine(q_I, w_I, k_I, L, H, d, dt, k, c, g, indices, scores_opt, cand_opt, cand_scores_opt, ws,
+                      ws_bytes, stream);
+}
+
 int pivot_version(void) { return 100; }
 
 }  // extern "C"
