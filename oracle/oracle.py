@@ -55,6 +55,7 @@ def lib():
         L.orc_topn.restype = I64
         L.orc_threads.restype = I32
         L.orc_set_threads.argtypes = [I32]
+        L.orc_set_aggregation.argtypes = [I32]
         _ = D
         _lib = L
     return _lib
@@ -82,6 +83,14 @@ def threads() -> int:
 
 def set_threads(n: int) -> None:
     lib().orc_set_threads(int(n))
+
+
+AGGREGATION = {"mean": 0, "first": 1, "last": 2}
+
+
+def set_aggregation(mode: str) -> None:
+    """Proxy aggregation of the PIVOT calls that follow: "mean" (Eq. 4), "first" or "last"."""
+    lib().orc_set_aggregation(AGGREGATION[mode])
 
 
 def dense(q, w, k, topk, t0=0, t1=None):

@@ -30,6 +30,11 @@
  *   - rows hold min(k, |eligible|) indices; the rest of the row is -1.
  *   - decode: sequence b holds P_b keys, its g members are positions
  *     P_b-g .. P_b-1 (current token, then drafts).  -> parity unpinned (a convention)
+ *   - proxy aggregation (PIVOT paper, Ablation Studies, "Proxy aggregation
+ *     (Table 2)": mean pooling against a first- or last-query proxy): the
+ *     first- / last-query proxy is the pooling of that one member row (q as
+ *     is, since rounding a value of the input dtype is exact; its w).
+ *     Selected with orc_set_aggregation (0 mean, the default; 1 first; 2 last).
  *
  * Arithmetic: every score is accumulated in double from the exact values of
  * the bf16 / fp32 inputs.  Sorting is a full qsort per row (brute force).
@@ -98,6 +103,19 @@ void orc_query_row(const void *q, const float *w, int dtype, int H, int d,
             qv[j * d + x] = orc_elem(q, dtype, (row * H + j) * (int64_t)d + x);
         wv[j] = (double)w[row * H + j];
     }
+}
+
+/* Proxy aggregation: 0 = mean of the members (Eq. 4), 1 = the first member's
+ * query, 2 = the last member's.  Read by the calls below; set between calls. */
+static int g_orc_agg = 0;
+void orc_set_aggregation(int mode) { g_orc_agg = (mode >= 0 && mode <= 2) ? mode : 0; }
+
+/* The member rows the proxy pools: all of them, or the first / last one. */
+static const int64_t *orc_agg_rows(const int64_t *rows, int *nrows)
+{
+    if (g_orc_agg == 1) { *nrows = 1; return rows; }
+    if (g_orc_agg == 2) { const int64_t *r = rows + (*nrows - 1); *nrows = 1; return r; }
+    return rows;
 }
 
 /* Eq. (4): proxy = per-head mean over the member rows (listed in `rows`).
@@ -271,7 +289,9 @@ int64_t orc_proxy_scores(const void *q, const float *w, const void *k, int dtype
     int n = orc_group_rows(L, g, i, rows);
     double *qb = (double *)malloc(sizeof(double) * (size_t)H * d);
     double *wb = (double *)malloc(sizeof(double) * (size_t)H);
-    orc_proxy(q, w, dtype, H, d, rows, n, qb, wb);
+    int na = n;
+    const int64_t *ar = orc_agg_rows(rows, &na);
+    orc_proxy(q, w, dtype, H, d, ar, na, qb, wb);
     int64_t P = rows[n - 1] + 1;
     orc_scores(qb, wb, H, d, k, dtype, NULL, 0, P, out);
     free(rows); free(qb); free(wb);
@@ -387,7 +407,9 @@ void orc_decode(const void *q, const float *w, const void *kc, const int64_t *of
         double *selv = (double *)malloc(sizeof(double) * (size_t)(topk > c ? topk : c));
         int need_proxy = (variant == 0) || (cand_in == NULL);
         if (need_proxy) {
-            orc_proxy(q, w, dtype, H, d, rows, g, qb, wb);
+            int na = g;
+            const int64_t *ar = orc_agg_rows(rows, &na);
+            orc_proxy(q, w, dtype, H, d, ar, na, qb, wb);
             orc_scores(qb, wb, H, d, kb, dtype, NULL, 0, P, pf); /* s <= P_b - 1 */
         }
         if (variant == 0) {

@@ -391,3 +391,46 @@ def test_sample_groups_edges():
     s = inputs.sample_groups(16384, 8, 2048, 4096, 256, 7)
     assert s.size == 256 and s[0] == 0 and s[-1] == 16383
     assert 511 in s and 256 in s  # P_i straddles c=4096 and k+g-1=2055
+
+
+# ---------------------------------------------------------------- proxy aggregation (Table 2 variants)
+
+
+@pytest.mark.parametrize("dt", [inputs.F32, inputs.BF16])
+@pytest.mark.parametrize("mode,member", [("first", 0), ("last", -1)])
+def test_single_query_proxy_member_row_is_dense(orc, dt, mode, member):
+    """With a first- (last-) query proxy, that member's Reuse row ranks its own
+    query's scores over s <= t: exactly its dense row, bit for bit."""
+    L, g, topk = 61, 4, 9
+    x = inputs.random_prefill(L, 3, 16, dt, seed=83)
+    di, dv = orc.dense(x["q"], x["w"], x["k"], topk)
+    try:
+        orc.set_aggregation(mode)
+        ui, uv = orc.reuse(x["q"], x["w"], x["k"], topk, g)
+    finally:
+        orc.set_aggregation("mean")
+    G = (L + g - 1) // g
+    rows = [min(i * g + g, L) - 1 if member == -1 else i * g for i in range(G)]
+    assert np.array_equal(ui[rows], di[rows])
+    assert np.array_equal(np.nan_to_num(uv[rows], nan=7.0), np.nan_to_num(dv[rows], nan=7.0))
+    # the other members rank the proxy's scores, not their own
+    other = [i * g + 1 for i in range(G) if i * g + 1 < L and i * g + 1 not in rows]
+    assert any(not np.array_equal(ui[t], di[t]) for t in other)
+
+
+@pytest.mark.parametrize("mode", ["first", "last"])
+def test_aggregation_reductions(orc, mode):
+    """g = 1: every aggregation is the query itself (Reuse = dense).  c >= L: the
+    candidate set is the whole prefix whatever the proxy (Refine = dense)."""
+    L, topk = 40, 7
+    x = inputs.random_prefill(L, 4, 16, inputs.F32, seed=84)
+    di, dv = orc.dense(x["q"], x["w"], x["k"], topk)
+    try:
+        orc.set_aggregation(mode)
+        ui, uv = orc.reuse(x["q"], x["w"], x["k"], topk, 1)
+        ri, rv, _, _ = orc.refine(x["q"], x["w"], x["k"], topk, L, 4)
+    finally:
+        orc.set_aggregation("mean")
+    nz = lambda v: np.nan_to_num(v, nan=7.0)  # short rows are NaN padded
+    assert np.array_equal(ui, di) and np.array_equal(nz(uv), nz(dv))
+    assert np.array_equal(ri, di) and np.array_equal(nz(rv), nz(dv))
