@@ -341,6 +341,9 @@ def main():
                 ts.append(e0.elapsed_time(e1))
             return statistics.median(ts)
 
+        agg_ms = {a_: timed(lambda a_=a_: P.refine(q, w, k, spec.k, spec.c, spec.g, out=out_idx, ws=ws,
+                                                    aggregation=a_)) for a_ in ("first", "last")}
+        extras["aggregation_refine_ms"] = agg_ms
         dense_ms = timed(lambda: P.indexer_dense(q, w, k, spec.k, out=out_idx, ws=ws), n=2)
         reuse_ms = timed(lambda: P.reuse(q, w, k, spec.k, spec.g, out=out_idx, ws=ws))
         extras.update(dense_ms=dense_ms, reuse_ms=reuse_ms, x_vs_dense=dense_ms / ms, reuse_x_vs_dense=dense_ms / reuse_ms)

@@ -109,6 +109,22 @@ PIVOT_API pivot_status pivot_refine(const void *q_I, const float *w_I, const voi
                           int32_t *cand_opt, float *cand_scores_opt, void *ws, size_t ws_bytes,
                           pivot_stream_t stream);
 
+/* Proxy aggregation variants (PIVOT paper, Ablation Studies, "Proxy aggregation
+ * (Table 2)": mean pooling against a first- or last-query proxy).  As
+ * pivot_reuse / pivot_refine, with the group proxy of Eq. (4) replaced by:
+ *   aggregation 0  the mean of the members (Eq. 4; the calls above),
+ *               1  the first member's query and w (the earliest position),
+ *               2  the last member's query and w.
+ * Other values return PIVOT_ERR_INVALID_ARG. */
+PIVOT_API pivot_status pivot_reuse_agg(const void *q_I, const float *w_I, const void *k_I, int64_t L, int H, int d,
+                                       pivot_dtype dt, int k, int g, int aggregation, int32_t *indices,
+                                       float *scores_opt, void *ws, size_t ws_bytes, pivot_stream_t stream);
+PIVOT_API pivot_status pivot_refine_agg(const void *q_I, const float *w_I, const void *k_I, int64_t L, int H,
+                                        int d, pivot_dtype dt, int k, int c, int g, int aggregation,
+                                        int32_t *indices, float *scores_opt, int32_t *cand_opt,
+                                        float *cand_scores_opt, void *ws, size_t ws_bytes,
+                                        pivot_stream_t stream);
+
 /* Guardrail (PIVOT paper, "Efficiency Results (Figure 4)": PIVOT falls back to
  * dense DSA at short context to avoid overhead).  The pages give no criterion;
  * this library uses the work model of the prefill call, in key-row products

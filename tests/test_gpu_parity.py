@@ -43,6 +43,11 @@ def members(L, g, i):
     return list(range(i * g, min(i * g + g, L)))
 
 
+def pooled(m, agg):
+    """The member rows the proxy pools: all (mean), the first or the last one."""
+    return {"mean": m, "first": m[:1], "last": m[-1:]}[agg]
+
+
 # ---------------------------------------------------------------- checkers
 
 
@@ -59,11 +64,11 @@ def check_dense(orc, x, idx, sc, rows, topk, key_base=None, pos=None):
     return fails
 
 
-def check_reuse(orc, x, idx, sc, groups, topk, g):
+def check_reuse(orc, x, idx, sc, groups, topk, g, agg="mean"):
     q, w, k = x["q"], x["w"], x["k"]
     L = q.shape[0]
     mem = [members(L, g, i) for i in groups]
-    qv, wv = orc.proxies(q, w, mem)
+    qv, wv = orc.proxies(q, w, [pooled(m, agg) for m in mem])
     F = orc.scores_batch(qv, wv, k, plen=np.array([m[-1] + 1 for m in mem]))
     fails = []
     for gi, m in enumerate(mem):
@@ -73,11 +78,11 @@ def check_reuse(orc, x, idx, sc, groups, topk, g):
     return fails
 
 
-def check_refine(orc, x, idx, sc, cand, csc, groups, topk, c, g):
+def check_refine(orc, x, idx, sc, cand, csc, groups, topk, c, g, agg="mean"):
     q, w, k = x["q"], x["w"], x["k"]
     L = q.shape[0]
     mem = [members(L, g, i) for i in groups]
-    qv, wv = orc.proxies(q, w, mem)
+    qv, wv = orc.proxies(q, w, [pooled(m, agg) for m in mem])
     F = orc.scores_batch(qv, wv, k, plen=np.array([m[-1] + 1 for m in mem]))
     fails = []
     for gi, (i, m) in enumerate(zip(groups, mem)):
@@ -367,6 +372,26 @@ def test_sampled_order_natural_order_and_fallback_agree(orc):
     groups = [0, 1, G // 3, G - 2, G - 1]
     fails = check_refine(orc, x, runs[0][2], None, runs[0][3], None, groups, topk, c, g)
     assert not fails, summarize(fails)
+
+
+# ---------------------------------------------------------------- proxy aggregation variants
+
+
+@pytest.mark.parametrize("agg", ["first", "last"])
+def test_aggregation_variants_every_group(orc, agg):
+    """First- / last-query proxies (the ablation's aggregation variants) on both
+    kernel paths, every group against the oracle."""
+    for x, topk, c, g in ((inputs.random_prefill(1337, 64, 128, inputs.BF16, seed=71), 64, 128, 8),
+                          (inputs.make_prefill(inputs.TINY), inputs.TINY.k, inputs.TINY.c, inputs.TINY.g)):
+        q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
+        L = x["q"].shape[0]
+        G = (L + g - 1) // g
+        u_idx, u_sc = P.reuse(q, w, k, topk, g, scores=True, aggregation=agg)
+        r_idx, r_sc, r_c, r_cs = P.refine(q, w, k, topk, c, g, scores=True, cand=True, aggregation=agg)
+        torch.cuda.synchronize()
+        fails = check_reuse(orc, x, host(u_idx), host(u_sc), range(G), topk, g, agg)
+        fails += check_refine(orc, x, host(r_idx), host(r_sc), host(r_c), host(r_cs), range(G), topk, c, g, agg)
+        assert not fails, summarize(fails)
 
 
 # ---------------------------------------------------------------- guardrail

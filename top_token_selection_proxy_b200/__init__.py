@@ -42,7 +42,11 @@ EXPORTS = (
     "pivot_last_device_status", "pivot_status_string", "pivot_last_cuda_error", "pivot_path",
     "pivot_set_device_timeout_ns", "pivot_set_debug_flags", "pivot_set_profile_events", "pivot_version",
     "pivot_reuse_noalloc", "pivot_guardrail_dense", "pivot_reuse_guarded", "pivot_refine_guarded",
+    "pivot_reuse_agg", "pivot_refine_agg",
 )
+
+# proxy aggregation (PIVOT paper, Ablation Studies, Proxy aggregation, Table 2)
+AGGREGATION = {"mean": 0, "first": 1, "last": 2}
 
 
 class PivotError(RuntimeError):
@@ -72,13 +76,15 @@ def lib() -> ctypes.CDLL:
         L.pivot_refine.argtypes = [P, P, P, I64, I, I, I, I, I, I, P, P, P, P, P, SZ, P]
         L.pivot_reuse_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P]
         L.pivot_refine_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P, SZ, P]
+        L.pivot_reuse_agg.argtypes = [P, P, P, I64, I, I, I, I, I, I, P, P, P, SZ, P]
+        L.pivot_refine_agg.argtypes = [P, P, P, I64, I, I, I, I, I, I, I, P, P, P, P, P, SZ, P]
         L.pivot_guardrail_dense.argtypes = [I, I64, I, I]
         L.pivot_guardrail_dense.restype = I
         L.pivot_reuse_guarded.argtypes = [P, P, P, I64, I, I, I, I, I, P, P, P, SZ, P, P]
         L.pivot_refine_guarded.argtypes = [P, P, P, I64, I, I, I, I, I, I, P, P, P, P, P, SZ, P, P]
         for f in ("pivot_indexer_dense", "pivot_reuse", "pivot_refine", "pivot_reuse_varlen",
                   "pivot_refine_varlen", "pivot_last_device_status", "pivot_reuse_guarded",
-                  "pivot_refine_guarded"):
+                  "pivot_refine_guarded", "pivot_reuse_agg", "pivot_refine_agg"):
             getattr(L, f).restype = I
         L.pivot_last_device_status.argtypes = [P, P]
         L.pivot_status_string.argtypes = [I]
@@ -186,20 +192,25 @@ def indexer_dense(q, w, k, topk: int, *, scores: bool = False, out=None, ws: Opt
 
 
 def reuse(q, w, k, topk: int, g: int, *, scores: bool = False, out=None, ws: Optional[Workspace] = None,
-          stream=None):
-    """Eq. (4)-(6): PIVOT-Reuse.  Returns (indices, proxy scores or None)."""
+          stream=None, aggregation: str = "mean"):
+    """Eq. (4)-(6): PIVOT-Reuse.  Returns (indices, proxy scores or None).
+    ``aggregation``: "mean" (Eq. 4), "first" or "last" query proxy."""
     L, H, d, dt = _prefill_common(q, w, k)
     idx = out if out is not None else torch.empty((L, topk), dtype=torch.int32, device=q.device)
     sc = torch.empty((L, topk), dtype=torch.float32, device=q.device) if scores else None
     nbytes = workspace_size(OP_REUSE, L, H, d, topk, topk, g, dt)
     W = _ws_for(ws, q.device).get(nbytes)
-    _check(lib().pivot_reuse(_ptr(q), _ptr(w), _ptr(k), L, H, d, dt, topk, g, _ptr(idx), _ptr(sc), _ptr(W),
-                             W.numel(), _stream(stream)), "pivot_reuse")
+    if aggregation == "mean":
+        _check(lib().pivot_reuse(_ptr(q), _ptr(w), _ptr(k), L, H, d, dt, topk, g, _ptr(idx), _ptr(sc), _ptr(W),
+                                 W.numel(), _stream(stream)), "pivot_reuse")
+    else:
+        _check(lib().pivot_reuse_agg(_ptr(q), _ptr(w), _ptr(k), L, H, d, dt, topk, g, AGGREGATION[aggregation],
+                                     _ptr(idx), _ptr(sc), _ptr(W), W.numel(), _stream(stream)), "pivot_reuse_agg")
     return idx, sc
 
 
 def refine(q, w, k, topk: int, c: int, g: int, *, scores: bool = False, cand=False, out=None,
-           ws: Optional[Workspace] = None, stream=None):
+           ws: Optional[Workspace] = None, stream=None, aggregation: str = "mean"):
     """Eq. (4),(5),(7)-(9): PIVOT-Refine.  Returns (indices, member scores|None, C|None, C scores|None).
 
     `cand` is False, True (allocate C) or a contiguous int32 [G, c] device tensor
@@ -218,8 +229,13 @@ def refine(q, w, k, topk: int, c: int, g: int, *, scores: bool = False, cand=Fal
     cs = torch.empty((G, c), dtype=torch.float32, device=q.device) if (cd is not None and scores) else None
     nbytes = workspace_size(OP_REFINE, L, H, d, topk, c, g, dt)
     W = _ws_for(ws, q.device).get(nbytes)
-    _check(lib().pivot_refine(_ptr(q), _ptr(w), _ptr(k), L, H, d, dt, topk, c, g, _ptr(idx), _ptr(sc), _ptr(cd),
-                              _ptr(cs), _ptr(W), W.numel(), _stream(stream)), "pivot_refine")
+    if aggregation == "mean":
+        _check(lib().pivot_refine(_ptr(q), _ptr(w), _ptr(k), L, H, d, dt, topk, c, g, _ptr(idx), _ptr(sc),
+                                  _ptr(cd), _ptr(cs), _ptr(W), W.numel(), _stream(stream)), "pivot_refine")
+    else:
+        _check(lib().pivot_refine_agg(_ptr(q), _ptr(w), _ptr(k), L, H, d, dt, topk, c, g, AGGREGATION[aggregation],
+                                      _ptr(idx), _ptr(sc), _ptr(cd), _ptr(cs), _ptr(W), W.numel(),
+                                      _stream(stream)), "pivot_refine_agg")
     return idx, sc, cd, cs
 
 
@@ -344,6 +360,6 @@ class KernelTimer:
 __all__ = [
     "lib", "LIB_PATH", "EXPORTS", "PivotError", "Workspace", "workspace_size", "varlen_workspace_size", "path",
     "indexer_dense", "reuse", "refine", "reuse_varlen", "refine_varlen", "last_device_status",
-    "guardrail_dense", "reuse_guarded", "refine_guarded",
+    "guardrail_dense", "reuse_guarded", "refine_guarded", "AGGREGATION",
     "set_device_timeout_ns", "set_debug_flags", "KernelTimer", "OP_DENSE", "OP_REUSE", "OP_REFINE", "BF16", "F32", "STATUS",
 ]

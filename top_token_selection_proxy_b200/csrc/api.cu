@@ -271,9 +271,10 @@ ScanArgs scan_base(const void* q, const float* w, int H, int d, int g, int n_sel
 // ---------------------------------------------------------------- prefill driver
 pivot_status run_prefill(int op, const void* q, const float* w, const void* k_I, int64_t L, int H, int d,
                          pivot_dtype dt, int k, int c, int g, int32_t* indices, float* scores, int32_t* cand_opt,
-                         float* cand_scores, void* ws, size_t ws_bytes, cudaStream_t s) {
+                         float* cand_scores, void* ws, size_t ws_bytes, cudaStream_t s, int agg = 0) {
   g_cuda_err[0] = 0;
   if (op == PIVOT_OP_DENSE) g = 1;
+  if (agg < 0 || agg > 2) return PIVOT_ERR_INVALID_ARG;
   pivot_status st = check_common(L, H, d, dt, k, c, g, op);
   if (st != PIVOT_OK) return st;
   if (!q || !w || !k_I || !indices || !ws) return PIVOT_ERR_INVALID_ARG;
@@ -298,6 +299,7 @@ pivot_status run_prefill(int op, const void* q, const float* w, const void* k_I,
     a.c = c;
     a.topk = k;
     a.variant = op;
+    a.agg = agg;
     a.n_groups = n_groups;
     a.out_idx = indices;
     a.out_scores = scores;
@@ -320,6 +322,7 @@ pivot_status run_prefill(int op, const void* q, const float* w, const void* k_I,
   ScanArgs a = scan_base(q, w, H, d, g, n_sel, k, mode, n_groups, n_items, W.selbuf, sel_cap(n_sel),
                          W.counters + 0, W.status);
   a.L = L;
+  a.agg = agg;
   a.out_idx = indices;
   a.out_scores = scores;
   int32_t* cand = cand_opt ? cand_opt : W.cand;
@@ -601,6 +604,21 @@ void pivot_set_profile_events(void** events, int n) {
   for (int i = 0; i < 4; ++i)
     g_prof[i] = (events && n >= 4) ? reinterpret_cast<cudaEvent_t>(events[i]) : nullptr;
 }
+pivot_status pivot_reuse_agg(const void* q_I, const float* w_I, const void* k_I, int64_t L, int H, int d,
+                             pivot_dtype dt, int k, int g, int aggregation, int32_t* indices, float* scores_opt,
+                             void* ws, size_t ws_bytes, pivot_stream_t stream) {
+  return run_prefill(PIVOT_OP_REUSE, q_I, w_I, k_I, L, H, d, dt, k, k, g, indices, scores_opt, nullptr, nullptr,
+                     ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream), aggregation);
+}
+
+pivot_status pivot_refine_agg(const void* q_I, const float* w_I, const void* k_I, int64_t L, int H, int d,
+                              pivot_dtype dt, int k, int c, int g, int aggregation, int32_t* indices,
+                              float* scores_opt, int32_t* cand_opt, float* cand_scores_opt, void* ws,
+                              size_t ws_bytes, pivot_stream_t stream) {
+  return run_prefill(PIVOT_OP_REFINE, q_I, w_I, k_I, L, H, d, dt, k, c, g, indices, scores_opt, cand_opt,
+                     cand_scores_opt, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream), aggregation);
+}
+
 // Guardrail work model (see pivot.h): key-row products of each path.
 int pivot_guardrail_dense(int op, int64_t L, int c, int g) {
   if (L < 1 || g < 1 || (op != PIVOT_OP_REUSE && op != PIVOT_OP_REFINE) || (op == PIVOT_OP_REFINE && c < 1))

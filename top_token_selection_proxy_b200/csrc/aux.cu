@@ -162,18 +162,21 @@ __global__ void __launch_bounds__(256) simt_kernel(const SimtArgs a) {
       t_first = mrow0;
       orow0 = mrow0;
     }
-    // Eq. (4): proxy = per-head mean, rounded to the input dtype (one member: the query itself)
+    // Eq. (4): proxy = per-head mean, rounded to the input dtype (one member: the query
+    // itself); the first- / last-query aggregation pools that one member
+    const int pn = a.agg != 0 ? 1 : nm;
+    const int64_t prow0 = a.agg == 2 ? mrow0 + nm - 1 : mrow0;
     for (int i = G.tid; i < H * D; i += 256) {
       float s = 0.f;
-      for (int m = 0; m < nm; ++m) s += ld_elem(a.q, a.is_bf16, (mrow0 + m) * (int64_t)H * D + i);
-      float v = nm > 1 ? __fdiv_rn(s, (float)nm) : s;
+      for (int m = 0; m < pn; ++m) s += ld_elem(a.q, a.is_bf16, (prow0 + m) * (int64_t)H * D + i);
+      float v = pn > 1 ? __fdiv_rn(s, (float)pn) : s;
       if (a.is_bf16) v = __bfloat162float(__float2bfloat16_rn(v));
       qv[i] = v;
     }
     for (int j = G.tid; j < H; j += 256) {
       float s = 0.f;
-      for (int m = 0; m < nm; ++m) s += a.w[(mrow0 + m) * H + j];
-      wv[j] = nm > 1 ? __fdiv_rn(s, (float)nm) : s;
+      for (int m = 0; m < pn; ++m) s += a.w[(prow0 + m) * H + j];
+      wv[j] = pn > 1 ? __fdiv_rn(s, (float)pn) : s;
     }
     G.sync();
     // Eq. (5) (Eq. (1) when g == 1) over the causal prefix s <= group end

@@ -32,6 +32,7 @@ struct ScanArgs {
   int topk;            // k
   int nb;              // groups per work item (N = nb * H)
   int mode;            // EmitMode
+  int agg;             // proxy aggregation: 0 mean of the members (Eq. 4), 1 first, 2 last query
   int64_t n_groups;
   int n_items;
   // decode (mode EMIT_PARTIAL): item -> (sequence, key chunk)
@@ -94,6 +95,7 @@ struct SimtArgs {
   int64_t L;
   int H, D, g, c, topk;
   int variant;         // 0 dense, 1 reuse, 2 refine
+  int agg;             // proxy aggregation as in ScanArgs
   int64_t n_groups;
   const int64_t* key_off;  // decode: [B+1] (groups are sequences), else null
   int32_t* out_idx;

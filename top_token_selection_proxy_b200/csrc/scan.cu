@@ -2,6 +2,8 @@
 //
 // PIVOT (picx.dev summary of the paper, Methodology):
 //   Eq. (4)  q-bar_j = mean of q_{t,j} over the group, w-bar_j = mean of w_{t,j}
+//            (or the first / last member's q and w: the aggregation variants of
+//            the paper's ablation, Proxy aggregation, Table 2)
 //   Eq. (5)  I-bar_s = sum_j w-bar_j ReLU(q-bar_j . k_s),  s <= group end
 //   Eq. (6)/(7) the group's top-(k+g-1) (Reuse) or top-c (Refine) by I-bar
 //   Eq. (1)  the dense indexer is the same scan with g = 1 and n_sel = k.
@@ -208,8 +210,12 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
         float acc[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-        const int nm = T.nmem[b];
-        const int64_t r0 = T.mrow0[b];
+        int nm = T.nmem[b];
+        int64_t r0 = T.mrow0[b];
+        if (a.agg != 0 && nm > 0) {  // first- / last-query proxy: pool that one member
+          if (a.agg == 2) r0 += nm - 1;
+          nm = 1;
+        }
         for (int m0 = 0; m0 < nm; m0 += 8) {  // 8 members' loads in flight, summed in member order
           uint4 vv[8];
 #pragma unroll
@@ -245,8 +251,12 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
       }
       for (int u = tid; u < C::NB * H; u += C::THREADS) {
         const int b = u / H, hj = u % H;
-        const int nm = T.nmem[b];
-        const int64_t r0 = T.mrow0[b];
+        int nm = T.nmem[b];
+        int64_t r0 = T.mrow0[b];
+        if (a.agg != 0 && nm > 0) {
+          if (a.agg == 2) r0 += nm - 1;
+          nm = 1;
+        }
         float wl[16];
 #pragma unroll
         for (int u = 0; u < 16; ++u) wl[u] = (u < nm) ? __ldg(a.w + (r0 + u) * H + hj) : 0.f;
