@@ -370,6 +370,17 @@ def main():
                           else "refine", "guarded_ms": g_grd, "refine_ms": g_ref, "dense_ms": g_den})
             del gq, gw, gk
         extras["guardrail"] = guard
+        # the pages' observations O1-O3 on the seeded 8K workload, from the dense indexer's rows
+        from top_token_selection_proxy_b200 import diagnostics
+
+        xg = inputs.make_prefill(inputs.PREFILL_8K)
+        gq, gw, gk = to_dev(xg["q"], dev), to_dev(xg["w"], dev), to_dev(xg["k"], dev)
+        Lg, kg = inputs.PREFILL_8K.L, inputs.PREFILL_8K.k
+        di, _ = P.indexer_dense(gq, gw, gk, kg, ws=ws)
+        _, dfull = P.indexer_dense(gq, gw, gk, Lg, scores=True, ws=ws)  # every prefix score
+        extras["workload_diagnostics"] = {"workload": inputs.PREFILL_8K.name,
+                                          **diagnostics.summary(di.cpu().numpy(), kg, dfull.cpu().numpy())}
+        del gq, gw, gk, di, dfull
 
     e2e = None
     M.barrier(world)  # every rank measures end to end (rank 0 arrives after its side measurements)
