@@ -39,9 +39,9 @@ L2_FLUSH_BYTES = 256 << 20
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum); valid only while
 # the sources the scan kernel is built from hash to `sources_sha256`.
 SCAN_TRAFFIC = {
-    "bytes": 2.77e9 + 1.65e9,
+    "bytes": 2780491520 + 1657540608,
     "sources": ("scan.cu", "select.cuh", "ptx.cuh", "kernels.cuh", "headsum.cuh"),
-    "sources_sha256": "63e24c5574ecf31d8ce181a639f8db031ea7cfc555dca026dbda4baf9015f426",
+    "sources_sha256": "2276ff7c391b0ca3ff38cba462eaeff37e13893b1c30546f4669be63f743a422",
     "profile": "profiles/dram_traffic_prefill_L131072_g8_refine.md",
 }
 

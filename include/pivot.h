@@ -109,6 +109,31 @@ PIVOT_API pivot_status pivot_refine(const void *q_I, const float *w_I, const voi
                           int32_t *cand_opt, float *cand_scores_opt, void *ws, size_t ws_bytes,
                           pivot_stream_t stream);
 
+/* Group ranges of one prefill sequence, for splitting a sequence's groups over
+ * several GPUs (the groups of Eq. (4)-(9) are independent given k_I).  Same
+ * computation as pivot_indexer_dense / pivot_reuse / pivot_refine on a length-L
+ * sequence, restricted to groups [g0, g1) (dense: query rows [t0, t1)); rows
+ * r0 = g0*g .. r1 = min(g1*g, L) - 1 of the output are produced:
+ *   q_rows [r1 + 1 - r0, H, d], w_rows [r1 + 1 - r0, H]: the range's query rows
+ *     only (row r0 first);
+ *   k_prefix [r1 + 1, d]: the key rows 0 .. r1 (all the range reads);
+ *   indices / scores_opt [r1 + 1 - r0, k]; cand_opt / cand_scores_opt [g1 - g0, c].
+ * Indices are positions in the whole sequence.  ws_bytes must cover
+ * pivot_workspace_size of the whole sequence (length L).  0 <= g0 < g1 <=
+ * ceil(L / g), else PIVOT_ERR_INVALID_ARG. */
+PIVOT_API pivot_status pivot_indexer_dense_range(const void *q_rows, const float *w_rows, const void *k_prefix,
+                                                 int64_t L, int H, int d, pivot_dtype dt, int k, int64_t t0,
+                                                 int64_t t1, int32_t *indices, float *scores_opt, void *ws,
+                                                 size_t ws_bytes, pivot_stream_t stream);
+PIVOT_API pivot_status pivot_reuse_range(const void *q_rows, const float *w_rows, const void *k_prefix, int64_t L,
+                                         int H, int d, pivot_dtype dt, int k, int g, int64_t g0, int64_t g1,
+                                         int32_t *indices, float *scores_opt, void *ws, size_t ws_bytes,
+                                         pivot_stream_t stream);
+PIVOT_API pivot_status pivot_refine_range(const void *q_rows, const float *w_rows, const void *k_prefix, int64_t L,
+                                          int H, int d, pivot_dtype dt, int k, int c, int g, int64_t g0, int64_t g1,
+                                          int32_t *indices, float *scores_opt, int32_t *cand_opt,
+                                          float *cand_scores_opt, void *ws, size_t ws_bytes, pivot_stream_t stream);
+
 /* Proxy aggregation variants (PIVOT paper, Ablation Studies, "Proxy aggregation
  * (Table 2)": mean pooling against a first- or last-query proxy).  As
  * pivot_reuse / pivot_refine, with the group proxy of Eq. (4) replaced by:

@@ -374,6 +374,34 @@ def test_sampled_order_natural_order_and_fallback_agree(orc):
     assert not fails, summarize(fails)
 
 
+# ---------------------------------------------------------------- one sequence split into group ranges
+
+
+def test_group_ranges_reproduce_the_whole_sequence():
+    """The zig-zag chunks of a 4-rank split, each run as a group-range call with only
+    its rows and its key prefix, give exactly the rows of the whole-sequence call
+    (dense, Reuse, Refine; tensor-core and CUDA-core paths)."""
+    from top_token_selection_proxy_b200 import multigpu as M
+
+    for x, topk, c, g in ((inputs.random_prefill(4096, 64, 128, inputs.BF16, seed=73), 128, 256, 8),
+                          (inputs.make_prefill(inputs.TINY), inputs.TINY.k, inputs.TINY.c, inputs.TINY.g)):
+        q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
+        L = x["q"].shape[0]
+        full = {"dense": host(P.indexer_dense(q, w, k, topk)[0]), "reuse": host(P.reuse(q, w, k, topk, g)[0]),
+                "refine": host(P.refine(q, w, k, topk, c, g)[0])}
+        world = 4
+        for r in range(world):
+            for t0, t1 in M.zigzag_chunks(L, g, world, r):
+                qr, wr, kp = q[t0:t1].contiguous(), w[t0:t1].contiguous(), k[:t1].contiguous()
+                got = {"dense": host(P.indexer_dense_range(qr, wr, kp, L, topk, t0, t1)[0]),
+                       "reuse": host(P.reuse_range(qr, wr, kp, L, topk, g, t0 // g, t1 // g)[0]),
+                       "refine": host(P.refine_range(qr, wr, kp, L, topk, c, g, t0 // g, t1 // g)[0])}
+                torch.cuda.synchronize()
+                for name in full:
+                    assert np.array_equal(np.sort(got[name], axis=1), np.sort(full[name][t0:t1], axis=1)), \
+                        f"{name} rows [{t0}, {t1}) of L = {L}"
+
+
 # ---------------------------------------------------------------- proxy aggregation variants
 
 

@@ -66,3 +66,71 @@ def test_single_rank_needs_no_process_group():
     assert M.weak_scaling(30.0, 3, 10, 1) == (10.0, pytest.approx(1000.0))
     M.barrier(1)
     M.finish(1)
+
+
+# ---------------------------------------------------------------- one sequence over several ranks
+
+
+def _zigzag_rank(rank: int, world: int, port: int, outdir: str) -> None:
+    import numpy as np
+
+    from oracle import oracle as orc
+
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port), "WORLD_SIZE": str(world),
+                       "RANK": str(rank), "LOCAL_RANK": str(rank)})
+    M.init("gloo", world, timeout_s=60.0)
+    L, g, k, c = 128, 4, 8, 16
+    x = inputs.random_prefill(L, 4, 16, inputs.F32, seed=97)   # every rank draws the same sequence
+    chunks = M.zigzag_chunks(L, g, world, rank)
+    k_local = torch.from_numpy(np.concatenate([x["k"][t0:t1] for t0, t1 in chunks]))
+    k_full = M.gather_keys(k_local, L, g, world).numpy()
+    rows = {}
+    for t0, t1 in chunks:  # the rank's groups, from the gathered keys
+        idx, val, _, _ = orc.refine(x["q"], x["w"], k_full, k, c, g, g0=t0 // g, g1=t1 // g)
+        rows[t0] = (idx.tolist(), np.nan_to_num(val, nan=7.0).tolist())
+    work = [M.chunk_work(L, g, c, t0, t1) for t0, t1 in chunks]
+    with open(os.path.join(outdir, f"zz{rank}.json"), "w") as f:
+        json.dump({"keys_equal": bool(np.array_equal(k_full, x["k"])), "rows": rows, "work": sum(work)}, f)
+    M.finish(world)
+
+
+@pytest.mark.timeout(300)
+def test_one_sequence_zigzag_over_two_ranks(tmp_path, orc):
+    import numpy as np
+
+    world = 2
+    mp.spawn(_zigzag_rank, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    res = [json.load(open(tmp_path / f"zz{r}.json")) for r in range(world)]
+    assert all(r["keys_equal"] for r in res), "gathered keys differ from the sequence's keys"
+    L, g, k, c = 128, 4, 8, 16
+    x = inputs.random_prefill(L, 4, 16, inputs.F32, seed=97)
+    ref_idx, ref_val, _, _ = orc.refine(x["q"], x["w"], x["k"], k, c, g)
+    covered = np.zeros(L, bool)
+    for r in res:
+        for t0, (idx, val) in r["rows"].items():
+            t0 = int(t0)
+            n = len(idx)
+            assert np.array_equal(np.array(idx), ref_idx[t0:t0 + n])
+            assert np.array_equal(np.array(val), np.nan_to_num(ref_val[t0:t0 + n], nan=7.0))
+            assert not covered[t0:t0 + n].any()
+            covered[t0:t0 + n] = True
+    assert covered.all(), "every row is computed by exactly one rank"
+    w0, w1 = res[0]["work"], res[1]["work"]
+    assert abs(w0 - w1) <= 0.1 * max(w0, w1), "zig-zag chunks balance the causal triangle"
+
+
+def test_zigzag_layout():
+    g = 8
+    for world in (1, 2, 4, 8):
+        L = 2 * world * g * 16
+        seen = []
+        for r in range(world):
+            for t0, t1 in M.zigzag_chunks(L, g, world, r):
+                assert t0 % g == 0 and t1 % g == 0 and t1 - t0 == L // (2 * world)
+                seen.append((t0, t1))
+        assert sorted(seen) == [(i * L // (2 * world), (i + 1) * L // (2 * world)) for i in range(2 * world)]
+        works = [sum(M.chunk_work(L, g, 4096, t0, t1) for t0, t1 in M.zigzag_chunks(L, g, world, r))
+                 for r in range(world)]
+        assert max(works) <= 1.12 * min(works)
+    with pytest.raises(ValueError):
+        M.zigzag_chunks(100, 8, 2, 0)

@@ -42,7 +42,8 @@ EXPORTS = (
     "pivot_last_device_status", "pivot_status_string", "pivot_last_cuda_error", "pivot_path",
     "pivot_set_device_timeout_ns", "pivot_set_debug_flags", "pivot_set_profile_events", "pivot_version",
     "pivot_reuse_noalloc", "pivot_guardrail_dense", "pivot_reuse_guarded", "pivot_refine_guarded",
-    "pivot_reuse_agg", "pivot_refine_agg",
+    "pivot_reuse_agg", "pivot_refine_agg", "pivot_indexer_dense_range", "pivot_reuse_range",
+    "pivot_refine_range",
 )
 
 # proxy aggregation (PIVOT paper, Ablation Studies, Proxy aggregation, Table 2)
@@ -76,6 +77,9 @@ def lib() -> ctypes.CDLL:
         L.pivot_refine.argtypes = [P, P, P, I64, I, I, I, I, I, I, P, P, P, P, P, SZ, P]
         L.pivot_reuse_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, SZ, P]
         L.pivot_refine_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, P, P, SZ, P]
+        L.pivot_indexer_dense_range.argtypes = [P, P, P, I64, I, I, I, I, I64, I64, P, P, P, SZ, P]
+        L.pivot_reuse_range.argtypes = [P, P, P, I64, I, I, I, I, I, I64, I64, P, P, P, SZ, P]
+        L.pivot_refine_range.argtypes = [P, P, P, I64, I, I, I, I, I, I, I64, I64, P, P, P, P, P, SZ, P]
         L.pivot_reuse_agg.argtypes = [P, P, P, I64, I, I, I, I, I, I, P, P, P, SZ, P]
         L.pivot_refine_agg.argtypes = [P, P, P, I64, I, I, I, I, I, I, I, P, P, P, P, P, SZ, P]
         L.pivot_guardrail_dense.argtypes = [I, I64, I, I]
@@ -84,7 +88,8 @@ def lib() -> ctypes.CDLL:
         L.pivot_refine_guarded.argtypes = [P, P, P, I64, I, I, I, I, I, I, P, P, P, P, P, SZ, P, P]
         for f in ("pivot_indexer_dense", "pivot_reuse", "pivot_refine", "pivot_reuse_varlen",
                   "pivot_refine_varlen", "pivot_last_device_status", "pivot_reuse_guarded",
-                  "pivot_refine_guarded", "pivot_reuse_agg", "pivot_refine_agg"):
+                  "pivot_refine_guarded", "pivot_reuse_agg", "pivot_refine_agg", "pivot_indexer_dense_range",
+                  "pivot_reuse_range", "pivot_refine_range"):
             getattr(L, f).restype = I
         L.pivot_last_device_status.argtypes = [P, P]
         L.pivot_status_string.argtypes = [I]
@@ -239,6 +244,56 @@ def refine(q, w, k, topk: int, c: int, g: int, *, scores: bool = False, cand=Fal
     return idx, sc, cd, cs
 
 
+def _range_common(q_rows, w_rows, k_prefix, L, g, g0, g1):
+    _need_cuda(q_rows, w_rows, k_prefix)
+    if q_rows.dim() != 3 or w_rows.shape != q_rows.shape[:2] or k_prefix.shape[1] != q_rows.shape[2]:
+        raise ValueError("expected q_rows [rows, H, d], w_rows [rows, H], k_prefix [keys, d]")
+    r0, r1 = g0 * g, min(g1 * g, L)
+    if q_rows.shape[0] != r1 - r0 or k_prefix.shape[0] < r1:
+        raise ValueError(f"groups [{g0}, {g1}) need {r1 - r0} query rows and {r1} key rows")
+    return q_rows.shape[1], q_rows.shape[2], _dt(q_rows), r1 - r0
+
+
+def indexer_dense_range(q_rows, w_rows, k_prefix, L: int, topk: int, t0: int, t1: int, *, scores: bool = False,
+                        ws: Optional[Workspace] = None, stream=None):
+    """Eq. (1) + TopK for query rows [t0, t1) of a length-L sequence (rows given, keys 0..t1-1)."""
+    H, d, dt, n = _range_common(q_rows, w_rows, k_prefix, L, 1, t0, t1)
+    idx = torch.empty((n, topk), dtype=torch.int32, device=q_rows.device)
+    sc = torch.empty((n, topk), dtype=torch.float32, device=q_rows.device) if scores else None
+    W = _ws_for(ws, q_rows.device).get(workspace_size(OP_DENSE, L, H, d, topk, topk, 1, dt))
+    _check(lib().pivot_indexer_dense_range(_ptr(q_rows), _ptr(w_rows), _ptr(k_prefix), L, H, d, dt, topk, t0, t1,
+                                           _ptr(idx), _ptr(sc), _ptr(W), W.numel(), _stream(stream)),
+           "pivot_indexer_dense_range")
+    return idx, sc
+
+
+def reuse_range(q_rows, w_rows, k_prefix, L: int, topk: int, g: int, g0: int, g1: int, *, scores: bool = False,
+                ws: Optional[Workspace] = None, stream=None):
+    """PIVOT-Reuse for groups [g0, g1) of a length-L sequence (their rows given, keys 0..min(g1*g, L)-1)."""
+    H, d, dt, n = _range_common(q_rows, w_rows, k_prefix, L, g, g0, g1)
+    idx = torch.empty((n, topk), dtype=torch.int32, device=q_rows.device)
+    sc = torch.empty((n, topk), dtype=torch.float32, device=q_rows.device) if scores else None
+    W = _ws_for(ws, q_rows.device).get(workspace_size(OP_REUSE, L, H, d, topk, topk, g, dt))
+    _check(lib().pivot_reuse_range(_ptr(q_rows), _ptr(w_rows), _ptr(k_prefix), L, H, d, dt, topk, g, g0, g1,
+                                   _ptr(idx), _ptr(sc), _ptr(W), W.numel(), _stream(stream)), "pivot_reuse_range")
+    return idx, sc
+
+
+def refine_range(q_rows, w_rows, k_prefix, L: int, topk: int, c: int, g: int, g0: int, g1: int, *,
+                 scores: bool = False, cand: bool = False, ws: Optional[Workspace] = None, stream=None):
+    """PIVOT-Refine for groups [g0, g1) of a length-L sequence.  Returns (indices, scores, C, C scores)."""
+    H, d, dt, n = _range_common(q_rows, w_rows, k_prefix, L, g, g0, g1)
+    idx = torch.empty((n, topk), dtype=torch.int32, device=q_rows.device)
+    sc = torch.empty((n, topk), dtype=torch.float32, device=q_rows.device) if scores else None
+    cd = torch.empty((g1 - g0, c), dtype=torch.int32, device=q_rows.device) if cand else None
+    cs = torch.empty((g1 - g0, c), dtype=torch.float32, device=q_rows.device) if (cand and scores) else None
+    W = _ws_for(ws, q_rows.device).get(workspace_size(OP_REFINE, L, H, d, topk, c, g, dt))
+    _check(lib().pivot_refine_range(_ptr(q_rows), _ptr(w_rows), _ptr(k_prefix), L, H, d, dt, topk, c, g, g0, g1,
+                                    _ptr(idx), _ptr(sc), _ptr(cd), _ptr(cs), _ptr(W), W.numel(), _stream(stream)),
+           "pivot_refine_range")
+    return idx, sc, cd, cs
+
+
 def guardrail_dense(op: int, L: int, c: int, g: int) -> bool:
     """The guardrail's choice (PIVOT paper, Efficiency Results, Figure 4): True when the
     dense indexer needs no more work than op (OP_REUSE or OP_REFINE) on a prefill of L."""
@@ -360,6 +415,7 @@ class KernelTimer:
 __all__ = [
     "lib", "LIB_PATH", "EXPORTS", "PivotError", "Workspace", "workspace_size", "varlen_workspace_size", "path",
     "indexer_dense", "reuse", "refine", "reuse_varlen", "refine_varlen", "last_device_status",
-    "guardrail_dense", "reuse_guarded", "refine_guarded", "AGGREGATION",
+    "guardrail_dense", "reuse_guarded", "refine_guarded", "AGGREGATION", "indexer_dense_range", "reuse_range",
+    "refine_range",
     "set_device_timeout_ns", "set_debug_flags", "KernelTimer", "OP_DENSE", "OP_REUSE", "OP_REFINE", "BF16", "F32", "STATUS",
 ]

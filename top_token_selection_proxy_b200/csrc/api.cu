@@ -269,9 +269,24 @@ ScanArgs scan_base(const void* q, const float* w, int H, int d, int g, int n_sel
 }
 
 // ---------------------------------------------------------------- prefill driver
+// Shift a caller's pointer to rows [r0, ...) down by r0 rows of `row` elements, so that
+// kernels indexing rows of the whole sequence land in the caller's buffer.
+template <typename T>
+T* rows_from(T* p, int64_t r0, int64_t row) {
+  if (!p) return p;
+  return reinterpret_cast<T*>(reinterpret_cast<uintptr_t>(p) - (uintptr_t)(r0 * row) * sizeof(*p));
+}
+const void* rows_from_bytes(const void* p, int64_t r0, int64_t row_bytes) {
+  return reinterpret_cast<const void*>(reinterpret_cast<uintptr_t>(p) - (uintptr_t)(r0 * row_bytes));
+}
+
+// Prefill over groups [g_lo, g_hi) of a length-L sequence (g_hi < 0: all groups).  For a
+// proper range, q / w / indices / scores hold only the range's rows, cand_opt only its
+// groups, and k_I the key rows [0, min(g_hi * g, L)) the range reads.
 pivot_status run_prefill(int op, const void* q, const float* w, const void* k_I, int64_t L, int H, int d,
                          pivot_dtype dt, int k, int c, int g, int32_t* indices, float* scores, int32_t* cand_opt,
-                         float* cand_scores, void* ws, size_t ws_bytes, cudaStream_t s, int agg = 0) {
+                         float* cand_scores, void* ws, size_t ws_bytes, cudaStream_t s, int agg = 0,
+                         int64_t g_lo = 0, int64_t g_hi = -1) {
   g_cuda_err[0] = 0;
   if (op == PIVOT_OP_DENSE) g = 1;
   if (agg < 0 || agg > 2) return PIVOT_ERR_INVALID_ARG;
@@ -279,12 +294,24 @@ pivot_status run_prefill(int op, const void* q, const float* w, const void* k_I,
   if (st != PIVOT_OK) return st;
   if (!q || !w || !k_I || !indices || !ws) return PIVOT_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_I) || !aligned16(ws)) return PIVOT_ERR_INVALID_ARG;
+  const int64_t n_groups_all = (L + g - 1) / g;
+  if (g_hi < 0) g_hi = n_groups_all;
+  if (g_lo < 0 || g_lo >= g_hi || g_hi > n_groups_all) return PIVOT_ERR_INVALID_ARG;
+  const int64_t r_lo = g_lo * g, r_hi = std::min<int64_t>(g_hi * g, L);  // the range's query rows
+  const int64_t L_keys = r_hi;                                            // key rows it reads
+  const size_t esz = dt == PIVOT_BF16 ? 2 : 4;
+  q = rows_from_bytes(q, r_lo, (int64_t)H * d * (int64_t)esz);
+  w = rows_from(w, r_lo, H);
+  indices = rows_from(indices, r_lo, k);
+  scores = rows_from(scores, r_lo, k);
+  cand_opt = rows_from(cand_opt, g_lo, c);
+  cand_scores = rows_from(cand_scores, g_lo, c);
   const PrefillWs need = carve_prefill(nullptr, op, L, H, d, k, c, g, dt, cand_opt != nullptr);
   if (ws_bytes < need.bytes) return PIVOT_ERR_WORKSPACE_TOO_SMALL;
   const PrefillWs W = carve_prefill(ws, op, L, H, d, k, c, g, dt, cand_opt != nullptr);
   cudaError_t e = cudaMemsetAsync(ws, 0, kHdr, s);
   if (e != cudaSuccess) return cuda_fail(e, "memset");
-  const int64_t n_groups = (L + g - 1) / g;
+  const int64_t n_groups = g_hi;  // kernels cover groups [g_lo, g_hi)
 
   if (!tc_shape(H, d, dt)) {
     SimtArgs a{};
@@ -300,6 +327,7 @@ pivot_status run_prefill(int op, const void* q, const float* w, const void* k_I,
     a.topk = k;
     a.variant = op;
     a.agg = agg;
+    a.grp_base = g_lo;
     a.n_groups = n_groups;
     a.out_idx = indices;
     a.out_scores = scores;
@@ -314,15 +342,16 @@ pivot_status run_prefill(int op, const void* q, const float* w, const void* k_I,
   }
 
   CUtensorMap kmap;
-  if (!make_kmap(&kmap, k_I, L, d, 128)) return cuda_fail(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+  if (!make_kmap(&kmap, k_I, L_keys, d, 128)) return cuda_fail(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
   const int nb = 256 / H;
   const int n_sel = sel_size(op, k, c, g);
-  const int n_items = (int)((n_groups + nb - 1) / nb);
+  const int n_items = (int)((g_hi - g_lo + nb - 1) / nb);
   const int mode = op == PIVOT_OP_DENSE ? EMIT_DENSE : (op == PIVOT_OP_REUSE ? EMIT_REUSE : EMIT_CAND);
   ScanArgs a = scan_base(q, w, H, d, g, n_sel, k, mode, n_groups, n_items, W.selbuf, sel_cap(n_sel),
                          W.counters + 0, W.status);
   a.L = L;
   a.agg = agg;
+  a.grp_base = g_lo;
   a.out_idx = indices;
   a.out_scores = scores;
   int32_t* cand = cand_opt ? cand_opt : W.cand;
@@ -348,8 +377,8 @@ pivot_status run_prefill(int op, const void* q, const float* w, const void* k_I,
   r.c = c;
   r.topk = k;
   r.mc = 512 / H;
-  r.n_groups = n_groups;
-  r.n_items = (int)(n_groups * ((g + r.mc - 1) / r.mc));
+  r.n_groups = n_groups;  // items count down from group g_hi - 1 to g_lo
+  r.n_items = (int)((g_hi - g_lo) * ((g + r.mc - 1) / r.mc));
   r.cand = cand;
   r.key_off = nullptr;
   r.keys = W.keys;
@@ -357,7 +386,7 @@ pivot_status run_prefill(int op, const void* q, const float* w, const void* k_I,
   r.status = W.status;
   r.timeout_ns = g_timeout_ns;
   CUtensorMap gmap, qmap;  // one-row boxes for the candidate gather; 256-row boxes of q rows
-  if (!make_kmap(&gmap, k_I, L, d, 1) || !make_kmap(&qmap, q, L * H, d, 256))
+  if (!make_kmap(&gmap, k_I, L_keys, d, 1) || !make_kmap(&qmap, q, r_hi * H, d, 256))
     return cuda_fail(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
   e = launch_refine(r, &gmap, &qmap, (int)std::min<int64_t>(num_sms(), r.n_items), s);
   if (e != cudaSuccess) return cuda_fail(e, "refine kernel");
@@ -366,7 +395,8 @@ pivot_status run_prefill(int op, const void* q, const float* w, const void* k_I,
   RowSelArgs rs{};
   rs.keys = W.keys;
   rs.cand = cand;
-  rs.n_rows = L;
+  rs.row_base = r_lo;
+  rs.n_rows = r_hi;
   rs.L = L;
   rs.key_off = nullptr;
   rs.g = g;
@@ -374,7 +404,7 @@ pivot_status run_prefill(int op, const void* q, const float* w, const void* k_I,
   rs.topk = k;
   rs.out_idx = indices;
   rs.out_scores = scores;
-  e = launch_rowselect(rs, (int)std::min<int64_t>(8 * num_sms(), L), s);
+  e = launch_rowselect(rs, (int)std::min<int64_t>(8 * num_sms(), r_hi - r_lo), s);
   if (e != cudaSuccess) return cuda_fail(e, "rowselect kernel");
   prof(3, s);
   return PIVOT_OK;
@@ -604,6 +634,29 @@ void pivot_set_profile_events(void** events, int n) {
   for (int i = 0; i < 4; ++i)
     g_prof[i] = (events && n >= 4) ? reinterpret_cast<cudaEvent_t>(events[i]) : nullptr;
 }
+pivot_status pivot_indexer_dense_range(const void* q_rows, const float* w_rows, const void* k_prefix, int64_t L,
+                                       int H, int d, pivot_dtype dt, int k, int64_t t0, int64_t t1,
+                                       int32_t* indices, float* scores_opt, void* ws, size_t ws_bytes,
+                                       pivot_stream_t stream) {
+  return run_prefill(PIVOT_OP_DENSE, q_rows, w_rows, k_prefix, L, H, d, dt, k, k, 1, indices, scores_opt, nullptr,
+                     nullptr, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream), 0, t0, t1);
+}
+
+pivot_status pivot_reuse_range(const void* q_rows, const float* w_rows, const void* k_prefix, int64_t L, int H,
+                               int d, pivot_dtype dt, int k, int g, int64_t g0, int64_t g1, int32_t* indices,
+                               float* scores_opt, void* ws, size_t ws_bytes, pivot_stream_t stream) {
+  return run_prefill(PIVOT_OP_REUSE, q_rows, w_rows, k_prefix, L, H, d, dt, k, k, g, indices, scores_opt, nullptr,
+                     nullptr, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream), 0, g0, g1);
+}
+
+pivot_status pivot_refine_range(const void* q_rows, const float* w_rows, const void* k_prefix, int64_t L, int H,
+                                int d, pivot_dtype dt, int k, int c, int g, int64_t g0, int64_t g1,
+                                int32_t* indices, float* scores_opt, int32_t* cand_opt, float* cand_scores_opt,
+                                void* ws, size_t ws_bytes, pivot_stream_t stream) {
+  return run_prefill(PIVOT_OP_REFINE, q_rows, w_rows, k_prefix, L, H, d, dt, k, c, g, indices, scores_opt,
+                     cand_opt, cand_scores_opt, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream), 0, g0, g1);
+}
+
 pivot_status pivot_reuse_agg(const void* q_I, const float* w_I, const void* k_I, int64_t L, int H, int d,
                              pivot_dtype dt, int k, int g, int aggregation, int32_t* indices, float* scores_opt,
                              void* ws, size_t ws_bytes, pivot_stream_t stream) {

@@ -23,7 +23,7 @@ __global__ void __launch_bounds__(256) rowselect_kernel(const RowSelArgs a) {
   __shared__ SelSmem S;
   __shared__ uint32_t hist11[kHist11Words];
   const Group<256> G{(int)threadIdx.x, 0};
-  for (int64_t row = blockIdx.x; row < a.n_rows; row += gridDim.x) {
+  for (int64_t row = a.row_base + blockIdx.x; row < a.n_rows; row += gridDim.x) {
     const int64_t grp = row / a.g;
     int64_t P;
     if (a.key_off)
@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(256) simt_kernel(const SimtArgs a) {
   float* wv = qv + H * D;
   uint64_t* buf = a.scratch + (int64_t)blockIdx.x * a.scratch_per_block;
   uint64_t* mb = buf + a.member_off;  // member entries (Refine)
-  for (int64_t grp = blockIdx.x; grp < a.n_groups; grp += gridDim.x) {
+  for (int64_t grp = a.grp_base + blockIdx.x; grp < a.n_groups; grp += gridDim.x) {
     int64_t kbase, P, mrow0, t_first, orow0;
     int nm;
     if (a.key_off) {

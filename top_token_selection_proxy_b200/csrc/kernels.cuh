@@ -33,6 +33,7 @@ struct ScanArgs {
   int nb;              // groups per work item (N = nb * H)
   int mode;            // EmitMode
   int agg;             // proxy aggregation: 0 mean of the members (Eq. 4), 1 first, 2 last query
+  int64_t grp_base;    // prefill: first group of the call (items cover groups [grp_base, n_groups))
   int64_t n_groups;
   int n_items;
   // decode (mode EMIT_PARTIAL): item -> (sequence, key chunk)
@@ -79,6 +80,7 @@ struct RefineArgs {
 struct RowSelArgs {
   const uint32_t* keys;  // [rows, c]
   const int32_t* cand;   // [n_groups, c]
+  int64_t row_base;      // first row of the call (rows [row_base, n_rows))
   int64_t n_rows;
   int64_t L;             // prefill sequence length (decode: 0)
   const int64_t* key_off;  // decode: [B+1]
@@ -96,6 +98,7 @@ struct SimtArgs {
   int H, D, g, c, topk;
   int variant;         // 0 dense, 1 reuse, 2 refine
   int agg;             // proxy aggregation as in ScanArgs
+  int64_t grp_base;    // first group of the call (groups [grp_base, n_groups))
   int64_t n_groups;
   const int64_t* key_off;  // decode: [B+1] (groups are sequences), else null
   int32_t* out_idx;

@@ -149,7 +149,7 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
       if (item < a.n_items) {
         if (!decode) {
           const int64_t blk = (int64_t)a.n_items - 1 - item;  // longest prefix first
-          const int64_t g0 = blk * C::NB;
+          const int64_t g0 = a.grp_base + blk * C::NB;
           const int nb_act = (int)min64(C::NB, a.n_groups - g0);
           T.grp0 = g0;
           T.nb_act = nb_act;

@@ -1,10 +1,13 @@
-"""One process per GPU, independent sequences per rank (weak scaling).
+"""One process per GPU.
 
-PIVOT indexes each sequence's groups independently of every other sequence,
-so N GPUs index N sequences with no collective on the data path; the only
-collectives are the barriers around a timed region and one max-reduction of
-the per-rank time.  The whole-job throughput is the queries of all ranks over
-the slowest rank's time.
+Independent sequences per rank (weak scaling): PIVOT indexes each sequence's
+groups independently of every other sequence, so N GPUs index N sequences with
+no collective on the data path; the only collectives are the barriers around a
+timed region and one max-reduction of the per-rank time.  The whole-job
+throughput is the queries of all ranks over the slowest rank's time.
+
+One sequence over N GPUs: zig-zag chunks of its groups per rank and one
+all-gather of the key chunks (below).
 """
 from __future__ import annotations
 
@@ -57,6 +60,50 @@ def weak_scaling(total_ms_local: float, steps: int, units_per_rank: int, world: 
     return ms, world * units_per_rank / (ms / 1000.0)
 
 
+# ---------------------------------------------------------------- one sequence over several GPUs
+# The groups of one prefill sequence are independent given its keys.  A zig-zag
+# layout (the sequence cut into 2W equal chunks of whole groups; rank r holds
+# chunks r and 2W-1-r) gives every rank an early and a late part of the causal
+# triangle, so the per-rank work sum_i (P_i + |G_i| min(c, P_i)) is nearly equal.
+# Each rank holds the queries, weights and keys of its own chunks; one
+# all-gather of the key chunks gives every rank the keys its groups read.
+
+
+def zigzag_chunks(L: int, g: int, world: int, rank: int):
+    """Token ranges [(t0, t1), (t0', t1')] of rank `rank`: chunks rank and 2W-1-rank of
+    2W chunks of equal size (a multiple of g; L must be a multiple of 2W*g)."""
+    n = 2 * world
+    if L % (n * g) != 0:
+        raise ValueError(f"L = {L} must be a multiple of 2 * world * g = {n * g}")
+    cs = L // n
+    return [(rank * cs, (rank + 1) * cs), ((n - 1 - rank) * cs, (n - rank) * cs)]
+
+
+def chunk_work(L: int, g: int, c: int, t0: int, t1: int) -> int:
+    """sum over the groups of rows [t0, t1) of P_i + |G_i| * min(c, P_i) (Refine's key-row products)."""
+    w = 0
+    for i0 in range(t0, t1, g):
+        P = min(i0 + g, L)
+        w += P + (P - i0) * min(c, P)
+    return w
+
+
+def gather_keys(k_local: torch.Tensor, L: int, g: int, world: int) -> torch.Tensor:
+    """All-gather of the zig-zag key chunks: k_local [2 * L / (2W), d] holds this rank's two
+    chunks (in zigzag_chunks order); returns all L key rows in position order."""
+    n = 2 * world
+    cs = L // n
+    if world <= 1:
+        return k_local
+    parts = [torch.empty_like(k_local) for _ in range(world)]
+    dist.all_gather(parts, k_local.contiguous())
+    full = torch.empty((L,) + tuple(k_local.shape[1:]), dtype=k_local.dtype, device=k_local.device)
+    for r in range(world):
+        for j, (t0, t1) in enumerate(zigzag_chunks(L, g, world, r)):
+            full[t0:t1] = parts[r][j * cs:(j + 1) * cs]
+    return full
+
+
 def finish(world: int) -> None:
     """Every rank calls this last: a final barrier, then leave the process group."""
     if world > 1 and dist.is_initialized():
@@ -64,4 +111,5 @@ def finish(world: int) -> None:
         dist.destroy_process_group()
 
 
-__all__ = ["SEED_STRIDE", "env", "init", "rank_seed", "barrier", "max_over_ranks", "weak_scaling", "finish"]
+__all__ = ["SEED_STRIDE", "env", "init", "rank_seed", "barrier", "max_over_ranks", "weak_scaling", "finish",
+           "zigzag_chunks", "chunk_work", "gather_keys"]
