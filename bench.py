@@ -39,9 +39,9 @@ L2_FLUSH_BYTES = 256 << 20
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum); valid only while
 # the sources the scan kernel is built from hash to `sources_sha256`.
 SCAN_TRAFFIC = {
-    "bytes": 2780491520 + 1657540608,
+    "bytes": 2764699392 + 1645043200,
     "sources": ("scan.cu", "select.cuh", "ptx.cuh", "kernels.cuh", "headsum.cuh"),
-    "sources_sha256": "2276ff7c391b0ca3ff38cba462eaeff37e13893b1c30546f4669be63f743a422",
+    "sources_sha256": "e958954c05d754c3c30a335dba5fca923bc87f6193ecc7998d18a5747895ab10",
     "profile": "profiles/dram_traffic_prefill_L131072_g8_refine.md",
 }
 
@@ -76,6 +76,9 @@ def parse():
     p.add_argument("--profile-case", type=int, default=0, metavar="L",
                    help="profiling run: two PIVOT-Refine calls at sequence length L (H_I=64, d=128, k=2048, "
                         "c=4096, g=8) and exit; no timing, no JSON")
+    p.add_argument("--profile-decode", action="store_true",
+                   help="profiling run: the MTP decode batch (B=32, P_b in [16384, 200000], g=4), two PIVOT-Refine "
+                        "then two PIVOT-Reuse calls, and exit; no timing, no JSON")
     return p.parse_args()
 
 
@@ -256,10 +259,37 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_profile_decode():
+    """The decode batch for ncu launch lists: per variant a warm-up call, then the captured call."""
+    import torch
+
+    import top_token_selection_proxy_b200 as P
+    from top_token_selection_proxy_b200 import build, inputs
+
+    build.build()
+    ds = inputs.DECODE
+    x = inputs.make_decode(ds)
+    dev = torch.device("cuda", 0)
+    q, w, kc = to_dev(x["q"], dev), to_dev(x["w"], dev), to_dev(x["k"], dev)
+    ws = P.Workspace(dev)
+    for _ in range(2):
+        P.refine_varlen(q, w, kc, x["offsets"], ds.k, ds.c, ds.g, ws=ws)
+    for _ in range(2):
+        P.reuse_varlen(q, w, kc, x["offsets"], ds.k, ds.g, ws=ws)
+    torch.cuda.synchronize()
+    st = P.last_device_status(ws)
+    print(f"profile decode {ds.name}: status {P.STATUS.get(st, st)}")
+    if st != 0:
+        raise SystemExit(1)
+
+
 def main():
     args = parse()
     if args.profile_case:
         run_profile_case(args.profile_case)
+        return
+    if args.profile_decode:
+        run_profile_decode()
         return
     if args.impl == "reference":
         run_reference(args)

@@ -292,9 +292,8 @@ def test_long_128k_refine_reuse_dense_sampled(orc, long_inputs):
     assert not fails, summarize(fails)
 
 
-def test_decode_batch_every_sequence(orc):
-    s = inputs.DECODE
-    x = inputs.make_decode(s)
+def _decode_batch_fails(orc, s, x):
+    """Every sequence's C row and Reuse rows, and every Refine row, against the oracle."""
     off = x["offsets"]
     q, w, kc = dev(x["q"]), dev(x["w"]), dev(x["k"])
     u_idx, u_sc = P.reuse_varlen(q, w, kc, off, s.k, s.g, scores=True)
@@ -323,7 +322,48 @@ def test_decode_batch_every_sequence(orc):
         ok = (C[row] >= 0) & (C[row] <= t)
         fails += check_row(r_idx[row], r_sc[row], C[row][ok], M[row][ok], min(s.k, int(ok.sum())), orc,
                            f"decode refine b={b} r={r}")
+    return fails, (u_idx, u_sc, r_idx, r_sc, r_c, r_cs)
+
+
+def test_decode_batch_every_sequence(orc):
+    s = inputs.DECODE
+    fails, _ = _decode_batch_fails(orc, s, inputs.make_decode(s))
     assert not fails, summarize(fails)
+
+
+def test_decode_many_short_sequences(orc):
+    # about 5 scan sets per CTA over several sequences: the proxy ring turns over and the
+    # per-CTA digit counts are flushed at every sequence change; many P_b <= c (keep all)
+    s = inputs.DecodeSpec("short", B=600, p_lo=4, p_hi=700, H=64, d=128, k=64, c=128, g=4, seed=23)
+    fails, _ = _decode_batch_fails(orc, s, inputs.make_decode(s))
+    assert not fails, summarize(fails)
+
+
+def test_decode_duplicate_keys_lowest_index_wins(orc):
+    # every cached key is one of 40 vectors, so whole blocks of keys tie exactly and the
+    # selection's final bin holds hundreds of equal scores: the lower index must win
+    s = inputs.DecodeSpec("dup", B=3, p_lo=3000, p_hi=20000, H=64, d=128, k=256, c=512, g=4, seed=29)
+    x = inputs.make_decode(s)
+    vid = np.random.default_rng(31).integers(0, 40, size=x["k"].shape[0])
+    x["k"] = np.ascontiguousarray(x["k"][vid])
+    fails, (u_idx, u_sc, r_idx, r_sc, r_c, r_cs) = _decode_batch_fails(orc, s, x)
+    assert not fails, summarize(fails)
+    off = x["offsets"]
+
+    def lowest_copies(row, sc, b, t, what):
+        got = row[row >= 0].astype(np.int64)
+        v = vid[off[b] + got]
+        for u in np.unique(v):
+            mine = got[v == u]
+            assert np.unique(sc[row >= 0][v == u]).size == 1, f"{what}: copies of one key scored differently"
+            pos = np.flatnonzero(vid[off[b]:off[b] + t + 1] == u)
+            assert np.array_equal(np.sort(mine), pos[:mine.size]), f"{what}: vector {u} not its lowest copies"
+
+    for b in range(s.B):
+        Pb = int(off[b + 1] - off[b])
+        lowest_copies(r_c[b], r_cs[b], b, Pb - 1, f"C_{b}")
+        for r in range(s.g):
+            lowest_copies(u_idx[b * s.g + r], u_sc[b * s.g + r], b, Pb - s.g + r, f"reuse b={b} r={r}")
 
 
 def test_decode_small_ragged(orc):

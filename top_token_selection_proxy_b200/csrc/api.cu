@@ -169,19 +169,13 @@ PrefillWs carve_prefill(void* base, int op, int64_t L, int H, int d, int k, int 
 struct DecodeWs {
   int* status;
   unsigned* counters;
-  int32_t* item_seq;
-  int64_t *item_s0, *item_s1;
-  int32_t* seq_item0;
-  uint64_t* selbuf;
-  uint64_t* partial;
-  uint32_t* partial_cnt;
-  uint64_t* mscratch;
+  DecodeArgs d;  // workspace pointers of the tensor-core path
   int32_t* cand;
   uint32_t* keys;
   uint64_t* sscratch;
   float* fscratch;
-  int grid, mgrid, simt_grid, n_items, partial_stride;
-  int64_t chunk, simt_per_block, simt_member_off;
+  int scan_grid, slices, simt_grid;
+  int64_t simt_per_block, simt_member_off;
   size_t bytes;
 };
 
@@ -193,34 +187,29 @@ DecodeWs carve_decode(void* base, int op, int B, const int64_t* off, int H, int 
   w.status = reinterpret_cast<int*>(hdr ? hdr + kStatusOff : nullptr);
   w.counters = reinterpret_cast<unsigned*>(hdr ? hdr + kCounterOff : nullptr);
   const int sms = num_sms();
-  int64_t total = 0, pmax = 0;
+  int64_t total = 0, pmax = 0, n_sets = 0;
   for (int b = 0; b < B; ++b) {
     const int64_t P = off[b + 1] - off[b];
     total += P;
     pmax = std::max(pmax, P);
+    n_sets += (P + kDecodeSetKeys - 1) / kDecodeSetKeys;
   }
   if (tc_shape(H, d, dt)) {
     const int n_sel = sel_size(op, k, c, g);
-    // chunks of at least 2*n_sel keys, ~4 chunks per SM over the batch
-    const int64_t target = (total + 4 * (int64_t)sms - 1) / (4 * (int64_t)sms);
-    w.chunk = (int64_t)align_up((size_t)std::max<int64_t>(2 * (int64_t)n_sel, target), 128);
-    int64_t items = 0;
-    for (int b = 0; b < B; ++b) {
-      const int64_t P = off[b + 1] - off[b];
-      items += std::max<int64_t>(1, (P + w.chunk - 1) / w.chunk);
-    }
-    w.n_items = (int)items;
-    w.grid = (int)std::min<int64_t>(sms, items);
-    w.mgrid = std::min(B, sms);
-    w.item_seq = cv.take<int32_t>(items);
-    w.item_s0 = cv.take<int64_t>(items);
-    w.item_s1 = cv.take<int64_t>(items);
-    w.seq_item0 = cv.take<int32_t>((size_t)B + 1);
-    w.selbuf = cv.take<uint64_t>((size_t)sms * (256 / H) * sel_cap(n_sel));
-    w.partial_stride = (int)align_up((size_t)n_sel, 32);
-    w.partial = cv.take<uint64_t>((size_t)items * w.partial_stride);
-    w.partial_cnt = cv.take<uint32_t>(items);
-    w.mscratch = cv.take<uint64_t>((size_t)w.mgrid * w.partial_stride);
+    DecodeArgs& a = w.d;
+    a.n_sets = n_sets;
+    w.scan_grid = (int)std::min<int64_t>(sms, n_sets);
+    w.slices = (int)((pmax + kDecodeSlice - 1) / kDecodeSlice);
+    a.proxy = cv.take<uint16_t>((size_t)B * H * d);
+    a.wbar = cv.take<float>((size_t)B * kWbarStride);
+    a.set_off = cv.take<int32_t>((size_t)B + 1);
+    a.scores = cv.take<uint32_t>((size_t)total);
+    a.ties = cv.take<uint64_t>((size_t)total);
+    a.hist1 = cv.take<uint32_t>((size_t)B * 2048);
+    a.hist2 = cv.take<uint32_t>((size_t)B * 2048);
+    a.sel = cv.take<uint64_t>((size_t)B * n_sel);
+    a.cnt = cv.take<uint32_t>((size_t)B);
+    a.tcnt = cv.take<uint32_t>((size_t)B);
     if (op == PIVOT_OP_REFINE) {
       if (!user_cand) w.cand = cv.take<int32_t>((size_t)B * c);
       w.keys = cv.take<uint32_t>((size_t)B * g * c);
@@ -377,6 +366,7 @@ pivot_status run_prefill(int op, const void* q, const float* w, const void* k_I,
   r.c = c;
   r.topk = k;
   r.mc = 512 / H;
+  r.cparts = 1;
   r.n_groups = n_groups;  // items count down from group g_hi - 1 to g_lo
   r.n_items = (int)((g_hi - g_lo) * ((g + r.mc - 1) / r.mc));
   r.cand = cand;
@@ -454,44 +444,31 @@ pivot_status run_decode(int op, const void* q, const float* w, const void* kc, c
     return e == cudaSuccess ? PIVOT_OK : cuda_fail(e, "simt kernel");
   }
 
-  e = launch_plan_items(off_dev, B, W.chunk, W.item_seq, W.item_s0, W.item_s1, W.seq_item0, s);
-  if (e != cudaSuccess) return cuda_fail(e, "plan kernel");
-  CUtensorMap kmap;
-  if (!make_kmap(&kmap, kc, off_host[B], d, 128)) return cuda_fail(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+  if ((int64_t)B * W.slices > 0x7FFFFFFFLL) return PIVOT_ERR_UNSUPPORTED_SHAPE;  // selection grid
   const int n_sel = sel_size(op, k, c, g);
-  ScanArgs a = scan_base(q, w, H, d, g, n_sel, k, EMIT_PARTIAL, B, W.n_items, W.selbuf, sel_cap(n_sel),
-                         W.counters + 0, W.status);
-  a.L = 0;
-  a.key_off = off_dev;
-  a.item_seq = W.item_seq;
-  a.item_s0 = W.item_s0;
-  a.item_s1 = W.item_s1;
-  a.partial = W.partial;
-  a.partial_stride = W.partial_stride;
-  a.partial_cnt = W.partial_cnt;
-  e = launch_scan(a, &kmap, W.grid, s);
-  if (e != cudaSuccess) return cuda_fail(e, "scan kernel");
-
   int32_t* cand = cand_opt ? cand_opt : W.cand;
-  MergeArgs m{};
-  m.partial = W.partial;
-  m.partial_cnt = W.partial_cnt;
-  m.seq_item0 = W.seq_item0;
-  m.n_sel = n_sel;
-  m.partial_stride = W.partial_stride;
-  m.B = B;
-  m.g = g;
-  m.topk = k;
-  m.mode = op == PIVOT_OP_REUSE ? EMIT_REUSE : EMIT_CAND;
-  m.key_off = off_dev;
-  m.scratch = W.mscratch;
-  m.cap = W.partial_stride;
-  m.cand = cand;
-  m.cand_scores = cand_scores;
-  m.out_idx = indices;
-  m.out_scores = scores;
-  e = launch_merge(m, W.mgrid, s);
-  if (e != cudaSuccess) return cuda_fail(e, "merge kernel");
+  DecodeArgs a = W.d;
+  a.q = reinterpret_cast<const uint16_t*>(q);
+  a.w = w;
+  a.key_off = off_dev;
+  a.B = B;
+  a.H = H;
+  a.D = d;
+  a.g = g;
+  a.n_sel = n_sel;
+  a.topk = k;
+  a.mode = op == PIVOT_OP_REUSE ? EMIT_REUSE : EMIT_CAND;
+  a.cand = cand;
+  a.cand_scores = cand_scores;
+  a.out_idx = indices;
+  a.out_scores = scores;
+  a.status = W.status;
+  a.timeout_ns = g_timeout_ns;
+  CUtensorMap kmap, pmap;  // 128-key tiles of the cache; the 64-row proxy of a sequence
+  if (!make_kmap(&kmap, kc, off_host[B], d, 128) || !make_kmap(&pmap, a.proxy, (int64_t)B * H, d, H))
+    return cuda_fail(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+  e = launch_decode(a, &kmap, &pmap, W.scan_grid, W.slices, s);
+  if (e != cudaSuccess) return cuda_fail(e, "decode kernels");
   if (op == PIVOT_OP_REUSE) return PIVOT_OK;
 
   RefineArgs r{};
@@ -506,7 +483,12 @@ pivot_status run_decode(int op, const void* q, const float* w, const void* kc, c
   r.topk = k;
   r.mc = 512 / H;
   r.n_groups = B;
-  r.n_items = B * ((g + r.mc - 1) / r.mc);
+  {
+    // few groups: split each group's candidate tiles so that the items cover the SMs
+    const int chunks = (g + r.mc - 1) / r.mc, tiles = (c + 127) / 128;
+    r.cparts = std::max(1, std::min(tiles, num_sms() / std::max(1, B * chunks)));
+    r.n_items = B * chunks * r.cparts;
+  }
   r.cand = cand;
   r.key_off = off_dev;
   r.keys = W.keys;

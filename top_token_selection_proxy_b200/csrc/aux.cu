@@ -1,10 +1,6 @@
 // aux.cu -- the non-tensor-core kernels of the library:
 //   * rowselect_kernel  Eq. (9): per member row, the top-k of its candidates'
 //                       re-scored keys (written by the refine kernel);
-//   * plan_kernel       decode: split each sequence's prefix into chunks;
-//   * merge_kernel      decode: exact top-n of the union of a sequence's
-//                       chunk-partial top-n lists, then emit C (Refine) or the
-//                       Reuse rows (Eq. 6);
 //   * simt_kernel       portable CUDA-core path (fp32 inputs, or shapes the
 //                       tensor-core kernels do not take): Eq. (1)/(4)-(9) per
 //                       group with the same exact selection.
@@ -59,63 +55,6 @@ cudaError_t launch_rowselect(const RowSelArgs& a, int grid, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-// ------------------------------------------------------------------ decode plan
-// Sequence b (P_b keys) is cut into max(1, ceil(P_b / chunk)) near-equal chunks.
-__global__ void plan_kernel(const int64_t* __restrict__ key_off, int B, int64_t chunk, int32_t* item_seq,
-                            int64_t* item_s0, int64_t* item_s1, int32_t* seq_item0) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  int it = 0;
-  for (int b = 0; b < B; ++b) {
-    seq_item0[b] = it;
-    const int64_t P = key_off[b + 1] - key_off[b];
-    const int64_t n = max64(1, (P + chunk - 1) / chunk);
-    for (int64_t c = 0; c < n; ++c) {
-      item_seq[it] = b;
-      item_s0[it] = P * c / n;
-      item_s1[it] = P * (c + 1) / n;
-      ++it;
-    }
-  }
-  seq_item0[B] = it;
-}
-
-cudaError_t launch_plan_items(const int64_t* key_off, int B, int64_t chunk, int32_t* item_seq, int64_t* item_s0,
-                              int64_t* item_s1, int32_t* seq_item0, cudaStream_t s) {
-  plan_kernel<<<1, 32, 0, s>>>(key_off, B, chunk, item_seq, item_s0, item_s1, seq_item0);
-  return cudaGetLastError();
-}
-
-// ------------------------------------------------------------------ decode merge
-__global__ void __launch_bounds__(256) merge_kernel(const MergeArgs a) {
-  __shared__ SelSmem S;
-  __shared__ uint64_t bot[16];
-  __shared__ uint32_t nbot;
-  const Group<256> G{(int)threadIdx.x, 0};
-  uint64_t* scr = a.scratch + (uint64_t)blockIdx.x * a.cap;
-  for (int b = blockIdx.x; b < a.B; b += gridDim.x) {
-    const int i0 = a.seq_item0[b], i1 = a.seq_item0[b + 1];
-    const uint64_t* region = a.partial + (uint64_t)i0 * a.partial_stride;
-    const uint32_t n = (uint32_t)(i1 - i0) * (uint32_t)a.partial_stride;
-    uint32_t real = 0;
-    for (int i = i0; i < i1; ++i) real += a.partial_cnt[i];
-    const uint64_t th = (real <= (uint32_t)a.n_sel) ? 1ull : radix_threshold<256>(region, n, a.n_sel, a.n_sel, S, G);
-    const uint32_t m = compact_ge<256>(region, scr, n, th, S, G);
-    const int64_t P = a.key_off[b + 1] - a.key_off[b];
-    if (a.mode == EMIT_CAND) {
-      emit_row<256>(scr, m, 0xFFFFFFFFu, 0ull, a.cand + (int64_t)b * a.n_sel,
-                    a.cand_scores ? a.cand_scores + (int64_t)b * a.n_sel : nullptr, (uint32_t)a.n_sel, S, G);
-    } else {
-      emit_reuse<256>(scr, m, a.topk, P - a.g, a.g, (int64_t)b * a.g, a.out_idx, a.out_scores, S, bot, &nbot, G);
-    }
-    G.sync();
-  }
-}
-
-cudaError_t launch_merge(const MergeArgs& a, int grid, cudaStream_t s) {
-  merge_kernel<<<grid, 256, 0, s>>>(a);
-  return cudaGetLastError();
-}
-
 // ------------------------------------------------------------------ portable path
 __device__ __forceinline__ float ld_elem(const void* p, int is_bf16, int64_t i) {
   if (is_bf16) return __uint_as_float((uint32_t)(reinterpret_cast<const uint16_t*>(p)[i]) << 16);
@@ -137,7 +76,7 @@ __device__ __forceinline__ float simt_score(const float* qv, const float* wv, in
 __global__ void __launch_bounds__(256) simt_kernel(const SimtArgs a) {
   __shared__ SelSmem S;
   __shared__ uint64_t bot[16];
-  __shared__ uint32_t nbot, cnt2;
+  __shared__ uint32_t cnt2;
   const Group<256> G{(int)threadIdx.x, 0};
   const int H = a.H, D = a.D;
   float* qv = a.fscratch + (int64_t)blockIdx.x * (H * D + H);
@@ -193,7 +132,7 @@ __global__ void __launch_bounds__(256) simt_kernel(const SimtArgs a) {
       const uint32_t nsel = (uint32_t)(a.topk + a.g - 1);
       const uint64_t th = radix_threshold<256>(buf, n, nsel, nsel, S, G);
       const uint32_t m = compact_ge<256>(buf, buf, n, th, S, G);
-      emit_reuse<256>(buf, m, a.topk, t_first, nm, orow0, a.out_idx, a.out_scores, S, bot, &nbot, G);
+      emit_reuse<256>(buf, m, a.topk, t_first, nm, orow0, a.out_idx, a.out_scores, S, bot, G);
     } else {
       const uint64_t th = radix_threshold<256>(buf, n, a.c, a.c, S, G);  // Eq. (7)
       const uint32_t m = compact_ge<256>(buf, buf, n, th, S, G);

@@ -1,0 +1,627 @@
+// decode.cu -- MTP decode groups (PIVOT, picx.dev summary of the paper,
+// Methodology, Eq. 3): sequence b holds P_b cached keys and one group of g
+// draft positions at the end of its prefix, so each sequence is one group
+// with one proxy (Eq. 4) scanned over its whole prefix (Eq. 5), followed by
+// the group's exact top-(k+g-1) (Reuse, Eq. 6) or top-c (Refine, Eq. 7).
+//
+// With one group per sequence the whole proxy-score vector of the batch is
+// small (4 bytes per cached key, against 2*d bytes of key read to make it),
+// so the selection runs on stored scores instead of inside the scan:
+//   1. prep: pool the proxies (bf16, row-major, read by TMA) and w-bar, and
+//      plan the scan (512-key sets, a block scan over the sequences);
+//   2. scan: persistent CTAs over equal shares of the batch's sets.  One set
+//      is 4 key tiles of one sequence; each tile is an M=128, N=64 MMA
+//      against the sequence's proxy into its own 64-column slot of a TMEM
+//      accumulator, so the 16 epilogue warps read (tile, lane quarter)
+//      blocks exactly as the prefill scan reads (group, lane quarter).  The
+//      epilogue writes each key's order key and counts its top 11 bits in a
+//      per-sequence histogram;
+//   3. select (two passes over the order keys, many CTAs per sequence): the
+//      histogram's threshold bin, then the next 11 bits inside that bin;
+//      keys above the thresholds are appended as winners, keys in the final
+//      bin pair as ties;
+//   4. emit (one CTA per sequence): the best of the ties by the full (score,
+//      index) order complete the exact selection; the candidate row (Refine)
+//      or the g member rows (Reuse) are written from it.
+#include <cuda_bf16.h>
+
+#include <cstddef>
+
+#include "headsum.cuh"
+#include "kernels.cuh"
+#include "ptx.cuh"
+#include "select.cuh"
+
+namespace pivot {
+
+namespace {
+
+constexpr int kDH = 64;          // heads (the tensor-core shape)
+constexpr int kSetTiles = kDecodeSetKeys / 128;  // key tiles per accumulator: one per 64-column slot
+constexpr int kSelThreads = 256;
+
+template <int D>
+struct DScanCfg {
+  static constexpr int KB = D / 64;            // 128-byte k-blocks per row
+  static constexpr int BM = 128;               // keys per tile (MMA M)
+  static constexpr int STAGES = 4;
+  static constexpr int A_BYTES = BM * D * 2;   // one key tile
+  static constexpr int P_BYTES = kDH * D * 2;  // one proxy (MMA B, N = 64)
+  static constexpr int NEPI = 512;             // 16 epilogue warps: (tile slot, lane quarter)
+  static constexpr int THREADS = 64 + NEPI;    // warp 0 TMA, warp 1 MMA
+};
+
+struct DScanTail {
+  uint64_t full[4], empty[4], accf[2], acce[2], pfull[2], pempty[2];
+  uint32_t tmem_slot;
+  volatile int abort_flag;
+  uint32_t hist[kHist11Words];  // this CTA's counts of the current sequence's top-11-bit digits
+};
+
+template <int D>
+constexpr size_t dscan_smem() {
+  using C = DScanCfg<D>;
+  return 1024 + C::STAGES * C::A_BYTES + 2 * C::P_BYTES + sizeof(DScanTail);
+}
+
+// Sequence holding set `s`: the largest b with set_off[b] <= s.
+__device__ __forceinline__ int seq_of_set(const int32_t* set_off, int B, int64_t s) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((int64_t)set_off[mid] <= s) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ 1. prep
+// Blocks per sequence: one 16-byte chunk of the proxy per thread.
+__host__ __device__ constexpr int prep_blocks_per_seq(int D) { return (kDH * (D / 8) + 255) / 256; }
+
+// Blocks b*PB .. b*PB+PB-1: sequence b's proxy (Eq. 4: the fp32 mean of its g
+// query rows, summed in member order, rounded to bf16), w-bar (written in the
+// epilogue's permuted layout) and zeroed selection state.  Last block:
+// set_off[b] = sum over b' < b of ceil(P_b' / kDecodeSetKeys).
+__global__ void __launch_bounds__(256) dprep_kernel(const DecodeArgs a) {
+  const int tid = threadIdx.x;
+  const int PB = prep_blocks_per_seq(a.D);
+  if ((int64_t)blockIdx.x == (int64_t)a.B * PB) {
+    __shared__ int32_t wsum[8];
+    __shared__ int32_t carry;
+    if (tid == 0) carry = 0;
+    __syncthreads();
+    for (int base = 0; base < a.B; base += 256) {
+      const int b = base + tid;
+      const int32_t v =
+          b < a.B ? (int32_t)((a.key_off[b + 1] - a.key_off[b] + kDecodeSetKeys - 1) / kDecodeSetKeys) : 0;
+      const int32_t incl = (int32_t)warp_incl_scan((uint32_t)v);
+      if ((tid & 31) == 31) wsum[tid >> 5] = incl;
+      __syncthreads();
+      int32_t before = carry;
+      for (int u = 0; u < (tid >> 5); ++u) before += wsum[u];
+      if (b < a.B) a.set_off[b + 1] = before + incl;
+      __syncthreads();
+      if (tid == 255) carry = before + incl;
+      __syncthreads();
+    }
+    if (tid == 0) a.set_off[0] = 0;
+    return;
+  }
+  const int b = blockIdx.x / PB, part = blockIdx.x % PB;
+  for (int i = part * 256 + tid; i < 4096; i += PB * 256) {
+    if (i < 2048) a.hist1[(int64_t)b * 2048 + i] = 0u;
+    else a.hist2[(int64_t)b * 2048 + i - 2048] = 0u;
+  }
+  if (part == 0 && tid == 0) {
+    a.cnt[b] = 0u;
+    a.tcnt[b] = 0u;
+  }
+  const int XC = a.D / 8;  // 16-byte chunks per row
+  const int g = a.g;       // <= 16
+  const int64_t r0 = (int64_t)b * g;
+  const int u = part * 256 + tid;
+  if (u < kDH * XC) {
+    const int hj = u / XC, xc = u % XC;
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int m0 = 0; m0 < g; m0 += 8) {  // 8 members' loads in flight, summed in member order
+      uint4 vv[8];
+#pragma unroll
+      for (int x = 0; x < 8; ++x)
+        vv[x] = (m0 + x < g) ? __ldg(reinterpret_cast<const uint4*>(a.q + ((r0 + m0 + x) * kDH + hj) * (int64_t)a.D) + xc)
+                             : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        if (m0 + x < g) {
+          const uint32_t wv[4] = {vv[x].x, vv[x].y, vv[x].z, vv[x].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc[2 * i] += __uint_as_float(wv[i] << 16);
+            acc[2 * i + 1] += __uint_as_float(wv[i] & 0xFFFF0000u);
+          }
+        }
+      }
+    }
+    uint32_t pk[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float lo = acc[2 * i], hi = acc[2 * i + 1];
+      if (g > 1) {
+        lo = __fdiv_rn(lo, (float)g);
+        hi = __fdiv_rn(hi, (float)g);
+      }
+      const __nv_bfloat162 h2 = __floats2bfloat162_rn(lo, hi);
+      pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
+    }
+    *reinterpret_cast<uint4*>(a.proxy + ((int64_t)b * kDH + hj) * a.D + xc * 8) =
+        make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  }
+  if (part == 0 && tid < kDH) {
+    const int hj = tid;
+    float wl[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x) wl[x] = (x < g) ? __ldg(a.w + (r0 + x) * kDH + hj) : 0.f;
+    float sw = 0.f;
+#pragma unroll
+    for (int x = 0; x < 16; ++x)
+      if (x < g) sw += wl[x];
+    a.wbar[(int64_t)b * kWbarStride + wperm_index(0, hj)] = g > 1 ? __fdiv_rn(sw, (float)g) : sw;
+  }
+}
+
+// ------------------------------------------------------------------ 2. scan
+template <int D>
+__global__ void __launch_bounds__(576, 1) dscan_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                       const __grid_constant__ CUtensorMap pmap, const DecodeArgs a) {
+  using C = DScanCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sP = smem + C::STAGES * C::A_BYTES;
+  DScanTail& T = *reinterpret_cast<DScanTail*>(sP + 2 * C::P_BYTES);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  if (tid == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&T.full[s], 1);
+      mbar_init(&T.empty[s], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&T.accf[x], 1);
+      mbar_init(&T.acce[x], C::NEPI);
+      mbar_init(&T.pfull[x], 1);
+      mbar_init(&T.pempty[x], 1);
+    }
+    T.abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&kmap);
+    prefetch_tmap(&pmap);
+  }
+  for (int i = tid; i < kHist11Words; i += C::THREADS) T.hist[i] = 0u;
+  if (warp == 1) {
+    tmem_alloc(&T.tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = T.tmem_slot;
+
+  // this CTA's share of the batch's sets
+  const int64_t set0 = a.n_sets * (int64_t)blockIdx.x / gridDim.x;
+  const int64_t set1 = a.n_sets * (int64_t)(blockIdx.x + 1) / gridDim.x;
+  int b = set0 < set1 ? seq_of_set(a.set_off, a.B, set0) : 0;
+  auto fail = [&]() {
+    T.abort_flag = 1;
+    atomicOr(a.status, DEV_ERR_TIMEOUT);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t st = 0, ph = 0, ps = 0, pph = 0;
+      int cur = -1;
+      for (int64_t sg = set0; sg < set1; ++sg) {
+        while (sg >= (int64_t)a.set_off[b + 1]) ++b;
+        if (b != cur) {  // the sequence's proxy into the next proxy slot
+          if (cur >= 0 && ++ps == 2) {
+            ps = 0;
+            pph ^= 1u;
+          }
+          if (!mbar_wait(&T.pempty[ps], pph ^ 1u, a.timeout_ns, &T.abort_flag)) {
+            fail();
+            break;
+          }
+          mbar_arrive_expect_tx(&T.pfull[ps], C::P_BYTES);
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_2d(sP + ps * C::P_BYTES + kb * (kDH * 128), &pmap, &T.pfull[ps], kb * 64, b * kDH);
+          cur = b;
+        }
+        const int64_t P = a.key_off[b + 1] - a.key_off[b];
+        const int64_t t0 = (sg - a.set_off[b]) * kSetTiles;
+        const int nt = (int)min64(kSetTiles, (P + C::BM - 1) / C::BM - t0);
+        bool ok = true;
+        for (int t = 0; t < nt; ++t) {
+          if (!mbar_wait(&T.empty[st], ph ^ 1u, a.timeout_ns, &T.abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&T.full[st], C::A_BYTES);
+          const int row = (int)(a.key_off[b] + (t0 + t) * C::BM);
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb)
+            tma_load_2d(sA + st * C::A_BYTES + kb * (C::BM * 128), &kmap, &T.full[st], kb * 64, row);
+          if (++st == C::STAGES) {
+            st = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) {
+          fail();
+          break;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(C::BM, kDH);
+      uint32_t st = 0, ph = 0, ab = 0, aph = 0, ps = 0, pph = 0;
+      int cur = -1;
+      for (int64_t sg = set0; sg < set1; ++sg) {
+        while (sg >= (int64_t)a.set_off[b + 1]) ++b;
+        const int64_t P = a.key_off[b + 1] - a.key_off[b];
+        const int64_t t0 = (sg - a.set_off[b]) * kSetTiles;
+        const int nt = (int)min64(kSetTiles, (P + C::BM - 1) / C::BM - t0);
+        if (!mbar_wait(&T.acce[ab], aph ^ 1u, a.timeout_ns, &T.abort_flag)) {
+          fail();
+          break;
+        }
+        if (b != cur) {
+          if (cur >= 0 && ++ps == 2) {
+            ps = 0;
+            pph ^= 1u;
+          }
+          if (!mbar_wait(&T.pfull[ps], pph, a.timeout_ns, &T.abort_flag)) {
+            fail();
+            break;
+          }
+          cur = b;
+        }
+        const uint32_t baddr = smem_u32(sP + ps * C::P_BYTES);
+        bool ok = true;
+        for (int t = 0; t < nt; ++t) {
+          if (!mbar_wait(&T.full[st], ph, a.timeout_ns, &T.abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t aaddr = smem_u32(sA + st * C::A_BYTES);
+          const uint32_t dtm = tmem + ab * 256u + (uint32_t)(t * kDH);
+#pragma unroll
+          for (int kb = 0; kb < C::KB; ++kb)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = sw128_kmajor_desc(aaddr + kb * (C::BM * 128) + kk * 32);
+              const uint64_t bd = sw128_kmajor_desc(baddr + kb * (kDH * 128) + kk * 32);
+              umma_bf16(dtm, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+            }
+          umma_commit(&T.empty[st]);
+          if (++st == C::STAGES) {
+            st = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) {
+          fail();
+          break;
+        }
+        umma_commit(&T.accf[ab]);
+        if (sg + 1 == set1 || sg + 1 >= (int64_t)a.set_off[b + 1]) umma_commit(&T.pempty[ps]);  // proxy slot free
+        if (++ab == 2) {
+          ab = 0;
+          aph ^= 1u;
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // warp w reads TMEM lanes 32*(w%4).. of tile slot (w-2)/4: Eq. (5) for 32 keys
+    const int q4 = warp & 3;
+    const int slot = (warp - 2) >> 2;
+    const int etid = tid - 64;
+    const int my_lane = quad_key_lane(lane);
+    uint32_t eab = 0, eaph = 0;
+    int cur = -1;
+    int64_t P = 0, kbase = 0;
+    auto flush = [&](int seq) {  // this CTA's digit counts of sequence seq -> its global histogram
+      named_bar_sync(1, C::NEPI);
+      for (int i = etid; i < 2048; i += C::NEPI) {
+        const uint32_t v = T.hist[h11(i)];
+        if (v) {
+          atomicAdd(&a.hist1[(int64_t)seq * 2048 + i], v);
+          T.hist[h11(i)] = 0u;
+        }
+      }
+      named_bar_sync(1, C::NEPI);
+    };
+    for (int64_t sg = set0; sg < set1; ++sg) {
+      while (sg >= (int64_t)a.set_off[b + 1]) ++b;
+      if (b != cur) {
+        if (cur >= 0) flush(cur);
+        cur = b;
+        P = a.key_off[b + 1] - a.key_off[b];
+        kbase = a.key_off[b];
+      }
+      const int64_t t0 = (sg - a.set_off[b]) * kSetTiles;
+      const int nt = (int)min64(kSetTiles, (P + C::BM - 1) / C::BM - t0);
+      const bool ok = mbar_wait(&T.accf[eab], eaph, a.timeout_ns, &T.abort_flag);
+      if (!ok) fail();
+      if (ok) {
+        tc_fence_after();
+        if (slot < nt) {
+          float2 w2[8];
+          load_w2(a.wbar + (int64_t)b * kWbarStride, 0, lane, w2);
+          float v[4];
+#pragma unroll
+          for (int slab = 0; slab < 2; ++slab) {
+            uint32_t r[32];
+            tmem_ld16x256b_x8(tmem + ((uint32_t)(q4 * 32 + slab * 16) << 16) + eab * 256u + (uint32_t)(slot * kDH),
+                              r);
+            tmem_wait_ld();
+            if (slab == 1) {
+              tc_fence_before();
+              mbar_arrive(&T.acce[eab]);
+            }
+            slab_head_sums(r, w2, v[2 * slab], v[2 * slab + 1]);
+          }
+          const float sc = quad_reduce_scatter(v, lane);
+          const int64_t s = (t0 + slot) * C::BM + q4 * 32 + my_lane;
+          const bool valid = s < P;
+          const uint32_t u = score_key(sc);
+          if (valid) a.scores[kbase + s] = u;
+          const uint32_t bin = valid ? (u >> 21) : 0xFFFFFFFFu;
+          const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
+          if (valid && lane == __ffs(peers) - 1) atomicAdd(&T.hist[h11(bin)], (uint32_t)__popc(peers));
+        } else {  // no tile in this slot (the sequence's last set)
+          tc_fence_before();
+          mbar_arrive(&T.acce[eab]);
+        }
+      }
+      if (++eab == 2) {
+        eab = 0;
+        eaph ^= 1u;
+      }
+    }
+    if (cur >= 0) flush(cur);
+  }
+
+  __syncthreads();
+  if (T.abort_flag) {  // let in-flight async copies / MMAs drain before releasing TMEM
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < 200000ull) {
+    }
+  }
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------ 3. select
+namespace {
+
+struct BinThr {
+  int T;           // threshold bin (-1: every entry is selected)
+  uint32_t above;  // entries in bins above T
+  uint32_t at;     // entries in bin T
+};
+
+// Over a 2048-bin histogram hg (global) with `total` entries: the bin T where the
+// count from the top first reaches `need` (need <= total).  All threads call.
+__device__ BinThr hist_threshold(const uint32_t* hg, uint32_t need, uint32_t total, uint32_t* wtot, int* scal) {
+  BinThr r{-1, total, 0u};
+  if (need >= total) return r;
+  const int t = threadIdx.x;
+  if (t == 0) {  // kept only if the counts do not reach `need` (an aborted scan): select everything
+    scal[0] = -1;
+    scal[1] = (int)total;
+    scal[2] = 0;
+  }
+  uint32_t loc[8], sum = 0;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    loc[u] = hg[2047 - 8 * t - u];
+    sum += loc[u];
+  }
+  const uint32_t incl = warp_incl_scan(sum);
+  if ((t & 31) == 31) wtot[t >> 5] = incl;
+  __syncthreads();
+  uint32_t excl = incl - sum;
+  for (int w = 0; w < (t >> 5); ++w) excl += wtot[w];
+  if (excl < need && need <= excl + sum) {
+    uint32_t c = excl;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (c + loc[u] >= need) {
+        scal[0] = 2047 - 8 * t - u;
+        scal[1] = (int)c;
+        scal[2] = (int)loc[u];
+        break;
+      }
+      c += loc[u];
+    }
+  }
+  __syncthreads();
+  r.T = scal[0];
+  r.above = (uint32_t)scal[1];
+  r.at = (uint32_t)scal[2];
+  __syncthreads();
+  return r;
+}
+
+}  // namespace
+
+// Block b * slices + z handles keys [z * kDecodeSlice, (z + 1) * kDecodeSlice) of sequence b.
+// level 1: winners = digit1 > T1; counts digit2 of the keys in bin T1.
+// level 2: winners = digit1 == T1 && digit2 > T2; ties = (T1, T2).
+// Every thread holds its 32 keys in registers; the block claims room for all
+// of its winners (and ties) with one atomic per counter.
+__global__ void __launch_bounds__(kSelThreads) dselect_kernel(const DecodeArgs a, int slices, int level) {
+  constexpr int U = kDecodeSlice / kSelThreads;
+  static_assert(U == 32, "one bit per key of a thread");
+  __shared__ uint32_t h[kHist11Words];
+  __shared__ uint32_t wtot[8];
+  __shared__ uint32_t wcnt[2][8];
+  __shared__ uint32_t base_s[2];
+  __shared__ int scal[4];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = (int)(blockIdx.x / (unsigned)slices);
+  const int64_t P = a.key_off[b + 1] - a.key_off[b];
+  const int64_t s0 = (int64_t)(blockIdx.x % (unsigned)slices) * kDecodeSlice;
+  if (s0 >= P) return;
+  const int64_t s1 = min64(P, s0 + kDecodeSlice);
+  const uint32_t need = (uint32_t)min64(a.n_sel, P);
+  const uint32_t* keys = a.scores + a.key_off[b];
+  const BinThr t1 = hist_threshold(a.hist1 + (int64_t)b * 2048, need, (uint32_t)P, wtot, scal);
+  if (level == 2 && t1.T < 0) return;  // level 1 took every key
+  BinThr t2{-1, 0u, 0u};
+  if (level == 2) t2 = hist_threshold(a.hist2 + (int64_t)b * 2048, need - t1.above, t1.at, wtot, scal);
+  if (level == 1) {
+    for (int i = tid; i < kHist11Words; i += kSelThreads) h[i] = 0u;
+    __syncthreads();
+  }
+  uint32_t v[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int64_t s = s0 + u * kSelThreads + tid;
+    v[u] = s < s1 ? keys[s] : 0u;
+  }
+  uint32_t win = 0u, tie = 0u;
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const bool valid = s0 + u * kSelThreads + tid < s1;
+    const int d1 = (int)(v[u] >> 21), d2 = (int)((v[u] >> 10) & 2047u);
+    if (level == 1) {
+      if (valid && d1 > t1.T) win |= 1u << u;
+      if (valid && d1 == t1.T) atomicAdd(&h[h11((uint32_t)d2)], 1u);
+    } else if (valid && d1 == t1.T) {
+      if (d2 > t2.T) win |= 1u << u;
+      if (d2 == t2.T) tie |= 1u << u;
+    }
+  }
+  const uint32_t nw = __popc(win), nt = __popc(tie);
+  const uint32_t iw = warp_incl_scan(nw), it = warp_incl_scan(nt);
+  if (lane == 31) {
+    wcnt[0][warp] = iw;
+    wcnt[1][warp] = it;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t tw = 0, tt = 0;
+    for (int x = 0; x < kSelThreads / 32; ++x) {
+      tw += wcnt[0][x];
+      tt += wcnt[1][x];
+    }
+    base_s[0] = tw ? atomicAdd(&a.cnt[b], tw) : 0u;
+    base_s[1] = tt ? atomicAdd(&a.tcnt[b], tt) : 0u;
+  }
+  __syncthreads();
+  uint32_t pw = base_s[0] + iw - nw, pt = base_s[1] + it - nt;
+  for (int x = 0; x < warp; ++x) {
+    pw += wcnt[0][x];
+    pt += wcnt[1][x];
+  }
+  uint64_t* sel = a.sel + (int64_t)b * a.n_sel;
+  uint64_t* ties = a.ties + a.key_off[b];
+  bool over = false;  // counts that do not match the stored keys (an aborted scan)
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const uint32_t s = (uint32_t)(s0 + u * kSelThreads + tid);
+    if (win & (1u << u)) {
+      if (pw < need) sel[pw] = pack_entry(v[u], s);
+      else over = true;
+      ++pw;
+    }
+    if (tie & (1u << u)) {
+      if (pt < (uint32_t)P) ties[pt] = pack_entry(v[u], s);
+      else over = true;
+      ++pt;
+    }
+  }
+  if (over) atomicOr(a.status, DEV_ERR_BOUNDS);
+  if (level == 1 && t1.T >= 0) {
+    __syncthreads();
+    for (int i = tid; i < 2048; i += kSelThreads) {
+      const uint32_t c = h[h11(i)];
+      if (c) atomicAdd(&a.hist2[(int64_t)b * 2048 + i], c);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ 4. emit
+__global__ void __launch_bounds__(kSelThreads) demit_kernel(const DecodeArgs a) {
+  __shared__ SelSmem S;
+  __shared__ uint64_t bot[16];
+  const Group<kSelThreads> G{(int)threadIdx.x, 0};
+  for (int b = blockIdx.x; b < a.B; b += gridDim.x) {
+    const int64_t P = a.key_off[b + 1] - a.key_off[b];
+    const uint32_t need = (uint32_t)min64(a.n_sel, P);
+    uint64_t* sel = a.sel + (int64_t)b * a.n_sel;
+    const uint32_t nw = min(a.cnt[b], need);
+    uint32_t m = nw;
+    if (nw < need) {  // the best (need - nw) ties, by the full (score, index) order
+      const uint64_t* ties = a.ties + a.key_off[b];
+      const uint32_t nt = min(a.tcnt[b], (uint32_t)P), need3 = need - nw;
+      const uint64_t th = radix_threshold<kSelThreads>(ties, nt, need3, need3, S, G);
+      m += compact_ge<kSelThreads>(ties, sel + nw, nt, th, S, G);
+    }
+    G.sync();
+    if (a.mode == EMIT_CAND) {
+      emit_row<kSelThreads>(sel, m, 0xFFFFFFFFu, 0ull, a.cand + (int64_t)b * a.n_sel,
+                            a.cand_scores ? a.cand_scores + (int64_t)b * a.n_sel : nullptr, (uint32_t)a.n_sel, S, G);
+    } else {
+      emit_reuse<kSelThreads>(sel, m, a.topk, P - a.g, a.g, (int64_t)b * a.g, a.out_idx, a.out_scores, S, bot, G);
+    }
+    G.sync();
+  }
+}
+
+// ------------------------------------------------------------------ launchers
+size_t decode_scan_smem_bytes(int D) {
+  if (D == 128) return dscan_smem<128>();
+  if (D == 64) return dscan_smem<64>();
+  return 0;
+}
+
+cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, const CUtensorMap* pmap, int scan_grid,
+                          int slices, cudaStream_t s) {
+  if (a.H != kDH || (a.D != 64 && a.D != 128)) return cudaErrorInvalidValue;
+  const int64_t prep_grid = (int64_t)a.B * prep_blocks_per_seq(a.D) + 1;
+  if (prep_grid > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+  dprep_kernel<<<(unsigned)prep_grid, 256, 0, s>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = decode_scan_smem_bytes(a.D);
+  if (a.D == 128) {
+    auto k = dscan_kernel<128>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<scan_grid, DScanCfg<128>::THREADS, smem, s>>>(*kmap, *pmap, a);
+  } else {
+    auto k = dscan_kernel<64>;
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k<<<scan_grid, DScanCfg<64>::THREADS, smem, s>>>(*kmap, *pmap, a);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const unsigned sg = (unsigned)slices * (unsigned)a.B;
+  dselect_kernel<<<sg, kSelThreads, 0, s>>>(a, slices, 1);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  dselect_kernel<<<sg, kSelThreads, 0, s>>>(a, slices, 2);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  demit_kernel<<<a.B < 1184 ? a.B : 1184, kSelThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace pivot

@@ -13,8 +13,7 @@ namespace pivot {
 enum EmitMode : int {
   EMIT_DENSE = 0,   // g == 1: row t = top-k of the query's own scores (Eq. 1)
   EMIT_REUSE = 1,   // Eq. 6: each member t takes the proxy top-k under s <= t
-  EMIT_CAND = 2,    // Eq. 7: write the proxy top-c candidate set C_i
-  EMIT_PARTIAL = 3  // decode chunk: write the chunk's top-n_sel packed entries
+  EMIT_CAND = 2     // Eq. 7: write the proxy top-c candidate set C_i
 };
 
 // Device status word bits (written with atomicOr, read by pivot_last_device_status).
@@ -36,14 +35,6 @@ struct ScanArgs {
   int64_t grp_base;    // prefill: first group of the call (items cover groups [grp_base, n_groups))
   int64_t n_groups;
   int n_items;
-  // decode (mode EMIT_PARTIAL): item -> (sequence, key chunk)
-  const int64_t* key_off;     // [B+1] row offsets of each sequence in the key tensor
-  const int32_t* item_seq;    // [n_items] sequence of each item
-  const int64_t* item_s0;     // [n_items] first local key of the chunk
-  const int64_t* item_s1;     // [n_items] one past the last local key
-  uint64_t* partial;          // [n_items, partial_stride] packed entries (EMIT_PARTIAL)
-  int partial_stride;         // >= n_sel, multiple of 32 (zero padded)
-  uint32_t* partial_cnt;      // [n_items]
   // outputs
   int32_t* out_idx;    // [rows, topk]
   float* out_scores;   // [rows, topk] or null
@@ -66,8 +57,9 @@ struct RefineArgs {
   int64_t L;             // prefill sequence length (0 for decode)
   int H, D, g, c, topk;
   int mc;                // members per work item (mc * H <= 512)
+  int cparts;            // parts the candidate tiles of a (group, member chunk) are split into
   int64_t n_groups;
-  int n_items;           // n_groups * ceil(g / mc)
+  int n_items;           // n_groups * ceil(g / mc) * cparts
   const int32_t* cand;   // [n_groups, c]  (-1 padded)
   const int64_t* key_off;  // decode: [B+1]; null for prefill
   uint32_t* keys;        // [rows, c] member score keys (0 = not eligible)
@@ -111,22 +103,39 @@ struct SimtArgs {
   float* fscratch;     // [gridDim.x, H*D + H] pooled proxy / member query
 };
 
-struct MergeArgs {
-  const uint64_t* partial;     // [n_items, n_sel]
-  const uint32_t* partial_cnt; // [n_items]
-  const int32_t* seq_item0;    // [B+1] first item of each sequence
-  int n_sel;                   // c (refine) or k+g-1 (reuse)
-  int partial_stride;          // entries per item in `partial` (>= n_sel, zero padded)
-  int B, g, topk, mode;        // mode: EMIT_CAND or EMIT_REUSE
-  const int64_t* key_off;      // [B+1]
-  uint64_t* scratch;           // [gridDim.x, cap]
-  int cap;
-  int32_t* cand;               // [B, n_sel]
-  float* cand_scores;
-  int32_t* out_idx;            // [B*g, topk]
-  float* out_scores;
-};
 
+// MTP decode groups: one group of g draft rows per sequence (decode.cu).
+constexpr int kDecodeSetKeys = 512;  // keys per scan set (4 tiles of 128, one per accumulator slot)
+constexpr int kDecodeSlice = 8192;   // keys per selection block
+constexpr int kWbarStride = 80;      // floats per sequence of the permuted w-bar table (4 rows of 20)
+struct DecodeArgs {
+  const uint16_t* q;        // bf16 bits [B*g, H, D]
+  const float* w;           // [B*g, H]
+  const int64_t* key_off;   // [B+1] row offsets of each sequence in the key cache
+  int B, H, D, g;
+  int n_sel;                // k+g-1 (Reuse) or c (Refine)
+  int topk;
+  int mode;                 // EMIT_CAND or EMIT_REUSE
+  int64_t n_sets;           // sum over b of ceil(P_b / kDecodeSetKeys)
+  // workspace
+  uint16_t* proxy;          // [B*H, D] bf16 bits: the pooled proxies (Eq. 4)
+  float* wbar;              // [B, kWbarStride] w-bar, permuted for the epilogue
+  int32_t* set_off;         // [B+1] first scan set of each sequence
+  uint32_t* scores;         // [sum P] order keys of the proxy scores (Eq. 5)
+  uint32_t* hist1;          // [B, 2048] counts of the order keys' top 11 bits
+  uint32_t* hist2;          // [B, 2048] counts of the next 11 bits inside the level-1 threshold bin
+  uint64_t* sel;            // [B, n_sel] packed selected entries
+  uint32_t* cnt;            // [B] entries in sel
+  uint64_t* ties;           // [sum P] packed entries of the final threshold bin pair
+  uint32_t* tcnt;           // [B]
+  // outputs
+  int32_t* cand;            // [B, n_sel] (Refine)
+  float* cand_scores;       // or null
+  int32_t* out_idx;         // [B*g, topk] (Reuse)
+  float* out_scores;        // or null
+  int* status;
+  uint64_t timeout_ns;
+};
 // launchers (return cudaError_t of the launch)
 cudaError_t launch_scan(const ScanArgs& a, const CUtensorMap* kmap, int grid, cudaStream_t s);
 size_t scan_smem_bytes(int H, int D);
@@ -134,9 +143,11 @@ cudaError_t launch_refine(const RefineArgs& a, const CUtensorMap* gather_kmap, c
                           cudaStream_t s);
 size_t refine_smem_bytes(int H, int D, int mc);
 cudaError_t launch_simt(const SimtArgs& a, int grid, cudaStream_t s);
-cudaError_t launch_merge(const MergeArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_rowselect(const RowSelArgs& a, int grid, cudaStream_t s);
-cudaError_t launch_plan_items(const int64_t* key_off, int B, int64_t chunk, int32_t* item_seq, int64_t* item_s0,
-                              int64_t* item_s1, int32_t* seq_item0, cudaStream_t s);
+// prep, scan, two selection passes and emit of a decode batch; scan_grid <= n_sets,
+// slices = ceil(max P_b / kDecodeSlice)
+cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, const CUtensorMap* pmap, int scan_grid,
+                          int slices, cudaStream_t s);
+size_t decode_scan_smem_bytes(int D);
 
 }  // namespace pivot

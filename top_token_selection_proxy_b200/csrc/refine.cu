@@ -9,7 +9,8 @@
 // row-select kernel.
 //
 // One persistent CTA per SM; a work item is (group, chunk of MC = 512/H
-// members).  Per item the members' query rows (MC*H rows x D, bf16) are the
+// members, part of the candidate tiles: one part for prefill, several when
+// there are few groups, as in a decode batch).  Per item the members' query rows (MC*H rows x D, bf16) are the
 // MMA's B operand in shared memory (K-major, 128-byte swizzle), loaded by TMA.
 // Each 128-candidate A tile (3-stage ring) is gathered in two halves that
 // complete on the same barrier: rows 0-63 by TMA 4-row gathers (warp 17),
@@ -57,7 +58,7 @@ struct RefTail {
   uint64_t full[3], empty[3], accf[2], acce[2];
   uint64_t bfull;  // members' q rows (B operand) landed
   uint32_t tmem_slot;
-  int item, nm, ntiles, nhalf, n_c;
+  int item, nm, ntiles, nhalf, n_c, tile0;
   volatile int abort_flag;
   int64_t grp, key_base, qrow0, t0, orow0;
   alignas(16) float wperm[8 * 4 * 20];  // members' w in the row-permuted layout of wperm_index
@@ -124,9 +125,11 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(const __grid_constant__ 
       const int item = (int)atomicAdd(a.counter, 1u);
       T.item = item;
       if (item < a.n_items) {
-        // longest prefix first: prefill groups in descending order
-        const int64_t grp = decode ? (int64_t)(item / chunks) : (a.n_groups - 1 - item / chunks);
-        const int mc = item % chunks;
+        // longest prefix first: prefill groups in descending order; an item is
+        // (group, member chunk, candidate part)
+        const int cp = item % a.cparts, gi = item / a.cparts;
+        const int64_t grp = decode ? (int64_t)(gi / chunks) : (a.n_groups - 1 - gi / chunks);
+        const int mc = gi % chunks;
         const int r0 = mc * C::MC;
         int64_t P, nmem_g;
         if (decode) {
@@ -149,14 +152,16 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(const __grid_constant__ 
         T.grp = grp;
         T.nm = (int)max64(0, min64(C::MC, nmem_g - r0));
         T.n_c = (int)min64(a.c, P);
-        T.ntiles = (T.n_c + C::BM - 1) / C::BM;
+        const int tiles = (T.n_c + C::BM - 1) / C::BM, tpp = (tiles + a.cparts - 1) / a.cparts;
+        T.tile0 = min(tiles, cp * tpp);
+        T.ntiles = min(tiles, T.tile0 + tpp) - T.tile0;
         T.nhalf = (T.nm * H + 255) / 256;
       }
     }
     __syncthreads();
     const int item = T.item;
     if (item >= a.n_items || T.abort_flag) break;
-    const int nm = T.nm, ntiles = T.ntiles, nhalf = T.nhalf, n_c = T.n_c;
+    const int nm = T.nm, ntiles = T.ntiles, nhalf = T.nhalf, n_c = T.n_c, tile0 = T.tile0;
     const int32_t* cand = a.cand + T.grp * (int64_t)a.c;
 
     // ---------------------------------------------------------------- members' q rows -> B (TMA), w -> smem
@@ -187,7 +192,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(const __grid_constant__ 
       // their ids, then one 4-row gather per 64-column k-block (ids past n_c read row 0;
       // those slots are masked by the epilogue)
       auto load_ids = [&](int j, int (&id)[4]) {
-        const int slot0 = j * C::BM + 4 * lane;
+        const int slot0 = (tile0 + j) * C::BM + 4 * lane;
         if (slot0 + 3 < n_c && (reinterpret_cast<uintptr_t>(cand + slot0) & 15u) == 0) {
           const int4 v = __ldg(reinterpret_cast<const int4*>(cand + slot0));
           id[0] = v.x;
@@ -238,7 +243,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(const __grid_constant__ 
       // to the tensor core (proxy fence) and arrives on that stage's full barrier
       const int row = C::TMA_ROWS + (tid - 32 * C::W_CPA);
       auto id_of = [&](int j) {
-        const int slot = j * C::BM + row;
+        const int slot = (tile0 + j) * C::BM + row;
         const int id = (slot < n_c) ? __ldg(cand + slot) : -1;
         return id >= 0 ? id : 0;  // slots without a candidate copy row 0 (masked later)
       };
@@ -340,7 +345,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(const __grid_constant__ 
       const int my_lane = quad_key_lane(lane);
       bool stop = false;
       for (int j = 0; j < ntiles && !stop; ++j) {
-        const int slot = j * C::BM + q4 * 32 + my_lane;
+        const int slot = (tile0 + j) * C::BM + q4 * 32 + my_lane;
         const int s = (slot < n_c) ? __ldg(cand + slot) : -1;
         for (int h = 0; h < nhalf; ++h) {
           const bool ok = mbar_wait(&T.accf[e_ab], e_aph, a.timeout_ns, &T.abort_flag);

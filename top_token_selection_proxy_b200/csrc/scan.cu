@@ -25,8 +25,7 @@
 //     buffer fills it is cut back (radix threshold + compaction) and the
 //     threshold rises.  No score matrix ever reaches HBM.
 //   * at the end of the item the epilogue warps run the exact top-n_sel and
-//     emit rows (dense / Reuse), the candidate set C_i (Refine), or a
-//     chunk's partial top-n_sel (decode).
+//     emit rows (dense / Reuse) or the candidate set C_i (Refine).
 #include <cuda_bf16.h>
 
 #include <cstddef>
@@ -85,7 +84,6 @@ struct ScanTail {
   int retry;                // the attempt's estimate was too high: scan the item again
   uint32_t hist11[kHist11Words];    // radix-select histogram (11-bit digits)
   uint64_t bot[16];
-  uint32_t nbot;
   SelSmem sel;
   // w-bar of the item's groups, permuted for the epilogue: row (b, m) holds heads
   // 8j + 2m, 8j + 2m + 1 (j = 0..7) of group b in 16 floats, rows 20 floats apart
@@ -139,7 +137,6 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
   uint32_t e_ab = 0, e_aph = 0;                         // epilogue: accumulator
   uint64_t* selbase = a.selbuf + (uint64_t)blockIdx.x * C::NB * (uint64_t)a.cap;
   const Group<C::NEPI> EG{tid - 64, 1};
-  const bool decode = (a.mode == EMIT_PARTIAL);
 
   for (;;) {
     // ---------------------------------------------------------------- item geometry
@@ -147,43 +144,28 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
       const int item = (int)atomicAdd(a.counter, 1u);
       T.item = item;
       if (item < a.n_items) {
-        if (!decode) {
-          const int64_t blk = (int64_t)a.n_items - 1 - item;  // longest prefix first
-          const int64_t g0 = a.grp_base + blk * C::NB;
-          const int nb_act = (int)min64(C::NB, a.n_groups - g0);
-          T.grp0 = g0;
-          T.nb_act = nb_act;
-          for (int b = 0; b < C::NB; ++b) {
-            const int64_t grp = g0 + b;
-            if (b < nb_act) {
-              const int64_t t0 = grp * a.g;
-              const int64_t t1 = min64(t0 + a.g, a.L);
-              T.mrow0[b] = t0;
-              T.nmem[b] = (int)(t1 - t0);
-              T.e[b] = t1 - 1;
-            } else {
-              T.mrow0[b] = 0;
-              T.nmem[b] = 0;
-              T.e[b] = -1;
-            }
+        const int64_t blk = (int64_t)a.n_items - 1 - item;  // longest prefix first
+        const int64_t g0 = a.grp_base + blk * C::NB;
+        const int nb_act = (int)min64(C::NB, a.n_groups - g0);
+        T.grp0 = g0;
+        T.nb_act = nb_act;
+        for (int b = 0; b < C::NB; ++b) {
+          const int64_t grp = g0 + b;
+          if (b < nb_act) {
+            const int64_t t0 = grp * a.g;
+            const int64_t t1 = min64(t0 + a.g, a.L);
+            T.mrow0[b] = t0;
+            T.nmem[b] = (int)(t1 - t0);
+            T.e[b] = t1 - 1;
+          } else {
+            T.mrow0[b] = 0;
+            T.nmem[b] = 0;
+            T.e[b] = -1;
           }
-          T.row_base = 0;
-          T.s_begin = 0;
-          T.s_end = T.e[nb_act - 1] + 1;
-        } else {
-          const int b = a.item_seq[item];
-          const int64_t P = a.key_off[b + 1] - a.key_off[b];
-          T.grp0 = b;
-          T.nb_act = 1;
-          for (int x = 0; x < C::NB; ++x) {
-            T.mrow0[x] = (x == 0) ? (int64_t)b * a.g : 0;
-            T.nmem[x] = (x == 0) ? a.g : 0;
-            T.e[x] = (x == 0) ? P - 1 : -1;
-          }
-          T.row_base = a.key_off[b];
-          T.s_begin = a.item_s0[item];
-          T.s_end = a.item_s1[item];
         }
+        T.row_base = 0;
+        T.s_begin = 0;
+        T.s_end = T.e[nb_act - 1] + 1;
         T.ntiles = (int)((T.s_end - T.s_begin + C::BM - 1) / C::BM);
         for (int b = 0; b < C::NB; ++b) {
           T.tau[b] = 0;
@@ -506,13 +488,9 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
           } else if (a.mode == EMIT_CAND) {
             emit_row<C::NEPI>(buf, m, 0xFFFFFFFFu, 0ull, a.cand + grp * a.n_sel,
                           a.cand_scores ? a.cand_scores + grp * a.n_sel : nullptr, need, T.sel, EG);
-          } else if (a.mode == EMIT_REUSE) {
+          } else {  // EMIT_REUSE
             emit_reuse<C::NEPI>(buf, m, a.topk, T.mrow0[b], T.nmem[b], T.mrow0[b], a.out_idx, a.out_scores, T.sel,
-                            T.bot, &T.nbot, EG);
-          } else {  // EMIT_PARTIAL: the chunk's exact top-n_sel, zero padded
-            uint64_t* dst = a.partial + (uint64_t)item * (uint32_t)a.partial_stride;
-            for (uint32_t i = EG.tid; i < (uint32_t)a.partial_stride; i += C::NEPI) dst[i] = (i < m) ? buf[i] : 0ull;
-            if (EG.tid == 0) a.partial_cnt[item] = m;
+                            T.bot, EG);
           }
           EG.sync();
         }

@@ -463,35 +463,35 @@ __device__ uint32_t emit_row(const uint64_t* buf, uint32_t n, uint32_t t_max, ui
 // is free; rows are padded with -1 to width topk).  nmem <= 16.
 template <int NT>
 __device__ void emit_reuse(uint64_t* buf, uint32_t m, int topk, int64_t t_first, int nmem, int64_t out_row0,
-                           int32_t* out_idx, float* out_sc, SelSmem& S, uint64_t* bot, uint32_t* nbot,
-                           const Group<NT>& G) {
-  // bottom entries (the m - topk lowest, at most 15), sorted ascending
+                           int32_t* out_idx, float* out_sc, SelSmem& S, uint64_t* bot, const Group<NT>& G) {
+  // bottom entries (the m - topk lowest, at most 15), ascending: one group-wide
+  // minimum per entry (packed entries are distinct)
   uint32_t nb = 0;
   if (m > (uint32_t)topk) {
-    const uint64_t Tk = radix_threshold<NT>(buf, m, topk, topk, S, G);
-    if (G.tid == 0) *nbot = 0;
-    G.sync();
-    for (uint32_t i = G.tid; i < m; i += NT) {
-      const uint64_t x = buf[i];
-      if (x < Tk) {
-        const uint32_t p = atomicAdd(nbot, 1u);
-        if (p < 16) bot[p] = x;
+    nb = m - (uint32_t)topk;
+    if (nb > 16u) nb = 16u;
+    static_assert(NT / 32 <= 16, "one minimum per warp in hist[128..159]");
+    uint64_t* wmin = reinterpret_cast<uint64_t*>(&S.hist[128]);
+    uint64_t last = 0ull;
+    for (uint32_t r = 0; r < nb; ++r) {
+      uint64_t mn = ~0ull;
+      for (uint32_t i = G.tid; i < m; i += NT) {
+        const uint64_t x = buf[i];
+        if ((r == 0 || x > last) && x < mn) mn = x;
       }
-    }
-    G.sync();
-    nb = *nbot;
-    if (G.tid == 0) {
-      for (uint32_t i = 1; i < nb && i < 16; ++i) {
-        const uint64_t v = bot[i];
-        int j = (int)i - 1;
-        while (j >= 0 && bot[j] > v) {
-          bot[j + 1] = bot[j];
-          --j;
-        }
-        bot[j + 1] = v;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t y = __shfl_xor_sync(0xFFFFFFFFu, mn, o);
+        mn = y < mn ? y : mn;
       }
+      if ((G.tid & 31) == 0) wmin[G.tid >> 5] = mn;
+      G.sync();
+      mn = wmin[0];
+      for (int x = 1; x < NT / 32; ++x) mn = wmin[x] < mn ? wmin[x] : mn;
+      if (G.tid == 0) bot[r] = mn;
+      last = mn;
+      G.sync();  // every warp has read wmin before the next round rewrites it
     }
-    G.sync();
   }
   // eligible count of every member: entry i is eligible for members r >= first(i)
   for (int i = G.tid; i < 16; i += NT) S.hist[i] = 0u;
