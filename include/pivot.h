@@ -179,7 +179,10 @@ PIVOT_API pivot_status pivot_refine_guarded(const void *q_I, const float *w_I, c
 
 /* Workspace bytes for the decode calls below.  key_offsets_host [B+1] is the
  * host copy of the key offsets (key_offsets_host[0] = 0, non-decreasing,
- * every P_b = key_offsets_host[b+1] - key_offsets_host[b] >= g). */
+ * every P_b = key_offsets_host[b+1] - key_offsets_host[b] >= g).  On the
+ * tensor-core path (bf16, H = 64, d in {64, 128}) it grows with the batch's
+ * keys: 12 bytes per cached key (a 32-bit score key and room for a packed tie
+ * entry) plus per-sequence proxies, histograms and the selection. */
 PIVOT_API size_t pivot_varlen_workspace_size(int op, int B, const int64_t *key_offsets_host, int H, int d, int k, int c,
                                    int g, pivot_dtype dt);
 
@@ -188,7 +191,11 @@ PIVOT_API size_t pivot_varlen_workspace_size(int op, int B, const int64_t *key_o
  * w [B*g,H], k_cache [sum P_b, d] (sequence b's keys are rows
  * key_offsets[b] .. key_offsets[b+1]-1), key_offsets_dev / key_offsets_host
  * [B+1] (same values, device and host copies) -> indices [B*g,k] of
- * positions local to each sequence. */
+ * positions local to each sequence.  Asynchronous on `stream`.  Returns
+ * PIVOT_ERR_UNSUPPORTED_SHAPE when B * ceil(max P_b / 8192) exceeds 2^31 - 1
+ * (the selection grid).  A device-side wait that runs out (PIVOT_ERR_DEVICE_TIMEOUT
+ * from pivot_last_device_status) leaves the outputs undefined; the selection
+ * then never writes past its buffers and may also flag PIVOT_ERR_DEVICE_BOUNDS. */
 PIVOT_API pivot_status pivot_reuse_varlen(const void *q, const float *w, const void *k_cache, const int64_t *key_offsets_dev,
                                 const int64_t *key_offsets_host, int B, int H, int d, pivot_dtype dt, int k, int g,
                                 int32_t *indices, float *scores_opt, void *ws, size_t ws_bytes,
