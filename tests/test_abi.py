@@ -106,3 +106,18 @@ def test_guardrail_decision():
     assert g_dense(P.OP_REFINE, 0, 16, 8) == -1
     assert g_dense(P.OP_REFINE, 100, 0, 8) == -1
     assert g_dense(P.OP_REUSE, 100, 16, 0) == -1
+
+
+def test_group_chunks_cover_the_rows_in_whole_groups():
+    from top_token_selection_proxy_b200 import group_chunks
+
+    for L, g, n in ((6001, 8, 8), (6001, 8, 3), (64, 8, 8), (5, 8, 4), (131072, 8, 8), (100, 1, 7)):
+        ch = group_chunks(L, g, n)
+        assert 1 <= len(ch) <= n
+        assert ch[0][0] == 0 and ch[-1][1] == L
+        for (a0, a1), (b0, _) in zip(ch, ch[1:]):
+            assert a1 == b0
+        for t0, t1 in ch:
+            assert t0 < t1 and t0 % g == 0 and (t1 % g == 0 or t1 == L)
+    with pytest.raises(ValueError):
+        group_chunks(0, 8, 2)

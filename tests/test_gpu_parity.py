@@ -442,6 +442,26 @@ def test_group_ranges_reproduce_the_whole_sequence():
                         f"{name} rows [{t0}, {t1}) of L = {L}"
 
 
+def test_streamed_refine_from_host_memory_matches_one_call():
+    """refine_streamed (pinned host inputs, copies overlapped with group-range calls in
+    chunks) writes exactly the rows of one device-resident refine call, for a ragged
+    length and chunk counts that do and do not divide the groups; twice in a row
+    (buffer reuse, earlier output overwritten)."""
+    x = inputs.random_prefill(6001, 64, 128, inputs.BF16, seed=79)
+    topk, c, g = 128, 256, 8
+    q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
+    want = np.sort(host(P.refine(q, w, k, topk, c, g)[0]), axis=1)
+    qh = torch.from_numpy(x["q"].view(np.int16)).pin_memory().view(torch.bfloat16)
+    wh = torch.from_numpy(x["w"]).pin_memory()
+    kh = torch.from_numpy(x["k"].view(np.int16)).pin_memory().view(torch.bfloat16)
+    oh = torch.empty((q.shape[0], topk), dtype=torch.int32).pin_memory()
+    for chunks in (1, 3, 8, 8):
+        oh.fill_(-7)
+        P.refine_streamed(qh, wh, kh, topk, c, g, out_host=oh, chunks=chunks)
+        torch.cuda.current_stream().synchronize()
+        assert np.array_equal(np.sort(oh.numpy(), axis=1), want), f"chunks = {chunks}"
+
+
 # ---------------------------------------------------------------- proxy aggregation variants
 
 

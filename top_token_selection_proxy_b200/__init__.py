@@ -294,6 +294,78 @@ def refine_range(q_rows, w_rows, k_prefix, L: int, topk: int, c: int, g: int, g0
     return idx, sc, cd, cs
 
 
+def group_chunks(L: int, g: int, chunks: int):
+    """[(t0, t1)]: rows [0, L) cut into at most `chunks` runs of whole groups of g."""
+    if L <= 0 or g <= 0 or chunks <= 0:
+        raise ValueError("L, g and chunks must be positive")
+    G = (L + g - 1) // g
+    per = (G + chunks - 1) // chunks
+    return [(i * g, min(L, (i + per) * g)) for i in range(0, G, per)]
+
+
+class _HostPipeline:
+    """Device copies and the two copy streams that refine_streamed reuses for one shape."""
+
+    def __init__(self, dev, L, H, d, topk):
+        self.q = torch.empty((L, H, d), dtype=torch.bfloat16, device=dev)
+        self.w = torch.empty((L, H), dtype=torch.float32, device=dev)
+        self.k = torch.empty((L, d), dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty((L, topk), dtype=torch.int32, device=dev)
+        self.s_in = torch.cuda.Stream(dev)
+        self.s_out = torch.cuda.Stream(dev)
+
+
+_pipelines = {}
+
+
+def refine_streamed(q_host, w_host, k_host, topk: int, c: int, g: int, *, out_host, chunks: int = 8,
+                    ws: Optional[Workspace] = None, device=None):
+    """PIVOT-Refine of one prefill sequence held in pinned host memory.
+
+    q_host [L, H, d] bf16, w_host [L, H] fp32, k_host [L, d] bf16 and out_host [L, topk]
+    int32 are pinned CPU tensors.  Keys and weights are copied first, then the queries
+    in `chunks` runs of whole groups.  Run i is indexed with the group-range call on the
+    current stream while run i+1 is copied in (a second stream) and run i-1's rows are
+    copied out (a third), so the transfers overlap the kernels.  The rows equal those of
+    one `refine` call.  Asynchronous: the current stream is ordered after the last copy
+    out, so synchronise it before reading out_host."""
+    for t, dt_ in ((q_host, torch.bfloat16), (w_host, torch.float32), (k_host, torch.bfloat16),
+                   (out_host, torch.int32)):
+        if t.is_cuda or not t.is_pinned() or not t.is_contiguous() or t.dtype != dt_:
+            raise ValueError("q/w/k/out must be contiguous pinned CPU tensors (bf16, fp32, bf16, int32)")
+    L, H, d = q_host.shape
+    if w_host.shape != (L, H) or k_host.shape != (L, d) or out_host.shape != (L, topk):
+        raise ValueError("expected q [L,H,d], w [L,H], k [L,d], out [L,topk]")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    key = (dev.index, L, H, d, topk)
+    pl = _pipelines.get(key)
+    if pl is None:
+        pl = _pipelines[key] = _HostPipeline(dev, L, H, d, topk)
+    W = _ws_for(ws, dev).get(workspace_size(OP_REFINE, L, H, d, topk, c, g, BF16))
+    cur = torch.cuda.current_stream(dev)
+    pl.s_in.wait_stream(cur)   # earlier work on the pipeline's buffers is done
+    pl.s_out.wait_stream(cur)
+    with torch.cuda.stream(pl.s_in):
+        pl.k.copy_(k_host, non_blocking=True)
+        pl.w.copy_(w_host, non_blocking=True)
+    for t0, t1 in group_chunks(L, g, chunks):
+        with torch.cuda.stream(pl.s_in):
+            pl.q[t0:t1].copy_(q_host[t0:t1], non_blocking=True)
+            landed = torch.cuda.Event()
+            landed.record(pl.s_in)
+        cur.wait_event(landed)
+        _check(lib().pivot_refine_range(_ptr(pl.q[t0:t1]), _ptr(pl.w[t0:t1]), _ptr(pl.k), L, H, d, BF16, topk, c, g,
+                                        t0 // g, (t1 + g - 1) // g, _ptr(pl.out[t0:t1]), None, None, None, _ptr(W),
+                                        W.numel(), ctypes.c_void_p(cur.cuda_stream)), "pivot_refine_range")
+        done = torch.cuda.Event()
+        done.record(cur)
+        pl.s_out.wait_event(done)
+        with torch.cuda.stream(pl.s_out):
+            out_host[t0:t1].copy_(pl.out[t0:t1], non_blocking=True)
+    cur.wait_stream(pl.s_out)
+    return out_host
+
+
 def guardrail_dense(op: int, L: int, c: int, g: int) -> bool:
     """The guardrail's choice (PIVOT paper, Efficiency Results, Figure 4): True when the
     dense indexer needs no more work than op (OP_REUSE or OP_REFINE) on a prefill of L."""
@@ -413,7 +485,7 @@ class KernelTimer:
 
 
 __all__ = [
-    "lib", "LIB_PATH", "EXPORTS", "PivotError", "Workspace", "workspace_size", "varlen_workspace_size", "path",
+    "lib", "LIB_PATH", "group_chunks", "refine_streamed", "EXPORTS", "PivotError", "Workspace", "workspace_size", "varlen_workspace_size", "path",
     "indexer_dense", "reuse", "refine", "reuse_varlen", "refine_varlen", "last_device_status",
     "guardrail_dense", "reuse_guarded", "refine_guarded", "AGGREGATION", "indexer_dense_range", "reuse_range",
     "refine_range",
