@@ -121,3 +121,15 @@ def test_group_chunks_cover_the_rows_in_whole_groups():
             assert t0 < t1 and t0 % g == 0 and (t1 % g == 0 or t1 == L)
     with pytest.raises(ValueError):
         group_chunks(0, 8, 2)
+
+
+def test_decode_workspace_grows_with_the_cached_keys(lib):
+    # tensor-core decode path: a 32-bit score key and a tie slot per cached key
+    off_a = np.array([0, 20000, 50000], dtype=np.int64)
+    off_b = np.array([0, 20000, 50000 + 100000], dtype=np.int64)
+    for op, c in ((P.OP_REUSE, 2048), (P.OP_REFINE, 4096)):
+        a = P.varlen_workspace_size(op, off_a, 64, 128, 2048, c, 4)
+        b = P.varlen_workspace_size(op, off_b, 64, 128, 2048, c, 4)
+        assert 0 < a and b - a >= 12 * 100000 - 8 * 256  # buffers start on 256-byte boundaries
+    assert P.varlen_workspace_size(P.OP_REUSE, np.array([0, 3], dtype=np.int64), 64, 128, 8, 8, 4) == 0  # P_b < g
+    assert P.varlen_workspace_size(P.OP_REUSE, np.array([5, 20], dtype=np.int64), 64, 128, 8, 8, 4) == 0  # off[0] != 0
