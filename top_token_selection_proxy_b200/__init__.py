@@ -485,9 +485,10 @@ class KernelTimer:
 
 
 __all__ = [
-    "lib", "LIB_PATH", "group_chunks", "refine_streamed", "EXPORTS", "PivotError", "Workspace", "workspace_size", "varlen_workspace_size", "path",
+    "lib", "LIB_PATH", "EXPORTS", "PivotError", "Workspace", "workspace_size", "varlen_workspace_size", "path",
     "indexer_dense", "reuse", "refine", "reuse_varlen", "refine_varlen", "last_device_status",
-    "guardrail_dense", "reuse_guarded", "refine_guarded", "AGGREGATION", "indexer_dense_range", "reuse_range",
-    "refine_range",
-    "set_device_timeout_ns", "set_debug_flags", "KernelTimer", "OP_DENSE", "OP_REUSE", "OP_REFINE", "BF16", "F32", "STATUS",
+    "guardrail_dense", "reuse_guarded", "refine_guarded", "AGGREGATION",
+    "indexer_dense_range", "reuse_range", "refine_range", "group_chunks", "refine_streamed",
+    "set_device_timeout_ns", "set_debug_flags", "KernelTimer", "OP_DENSE", "OP_REUSE", "OP_REFINE", "BF16", "F32",
+    "STATUS",
 ]
