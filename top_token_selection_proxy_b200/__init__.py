@@ -307,6 +307,7 @@ class _HostPipeline:
     """Device copies and the two copy streams that refine_streamed reuses for one shape."""
 
     def __init__(self, dev, L, H, d, topk):
+        self.shape = (L, H, d, topk)
         self.q = torch.empty((L, H, d), dtype=torch.bfloat16, device=dev)
         self.w = torch.empty((L, H), dtype=torch.float32, device=dev)
         self.k = torch.empty((L, d), dtype=torch.bfloat16, device=dev)
@@ -315,7 +316,20 @@ class _HostPipeline:
         self.s_out = torch.cuda.Stream(dev)
 
 
-_pipelines = {}
+_pipelines = {}  # device index -> the _HostPipeline of the last shape used there
+
+
+def _drop_pipeline(index) -> None:
+    pl = _pipelines.pop(index, None)
+    if pl is not None:  # its copies may still be in flight: let them finish before the buffers go
+        pl.s_in.synchronize()
+        pl.s_out.synchronize()
+
+
+def release_streamed_buffers() -> None:
+    """Free the device buffers refine_streamed keeps between calls (waits for its copies)."""
+    for index in list(_pipelines):
+        _drop_pipeline(index)
 
 
 def refine_streamed(q_host, w_host, k_host, topk: int, c: int, g: int, *, out_host, chunks: int = 8,
@@ -327,8 +341,10 @@ def refine_streamed(q_host, w_host, k_host, topk: int, c: int, g: int, *, out_ho
     in `chunks` runs of whole groups.  Run i is indexed with the group-range call on the
     current stream while run i+1 is copied in (a second stream) and run i-1's rows are
     copied out (a third), so the transfers overlap the kernels.  The rows equal those of
-    one `refine` call.  Asynchronous: the current stream is ordered after the last copy
-    out, so synchronise it before reading out_host."""
+    one `refine` call.  Device copies of the inputs are kept for the next call of the same
+    shape (one shape per device; release_streamed_buffers frees them).  Asynchronous: the
+    current stream is ordered after the last copy out, so synchronise it before reading
+    out_host."""
     for t, dt_ in ((q_host, torch.bfloat16), (w_host, torch.float32), (k_host, torch.bfloat16),
                    (out_host, torch.int32)):
         if t.is_cuda or not t.is_pinned() or not t.is_contiguous() or t.dtype != dt_:
@@ -337,10 +353,10 @@ def refine_streamed(q_host, w_host, k_host, topk: int, c: int, g: int, *, out_ho
     if w_host.shape != (L, H) or k_host.shape != (L, d) or out_host.shape != (L, topk):
         raise ValueError("expected q [L,H,d], w [L,H], k [L,d], out [L,topk]")
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
-    key = (dev.index, L, H, d, topk)
-    pl = _pipelines.get(key)
-    if pl is None:
-        pl = _pipelines[key] = _HostPipeline(dev, L, H, d, topk)
+    pl = _pipelines.get(dev.index)
+    if pl is None or pl.shape != (L, H, d, topk):
+        _drop_pipeline(dev.index)
+        pl = _pipelines[dev.index] = _HostPipeline(dev, L, H, d, topk)
     W = _ws_for(ws, dev).get(workspace_size(OP_REFINE, L, H, d, topk, c, g, BF16))
     cur = torch.cuda.current_stream(dev)
     pl.s_in.wait_stream(cur)   # earlier work on the pipeline's buffers is done
@@ -488,7 +504,8 @@ __all__ = [
     "lib", "LIB_PATH", "EXPORTS", "PivotError", "Workspace", "workspace_size", "varlen_workspace_size", "path",
     "indexer_dense", "reuse", "refine", "reuse_varlen", "refine_varlen", "last_device_status",
     "guardrail_dense", "reuse_guarded", "refine_guarded", "AGGREGATION",
-    "indexer_dense_range", "reuse_range", "refine_range", "group_chunks", "refine_streamed",
+    "indexer_dense_range", "reuse_range", "refine_range",
+    "group_chunks", "refine_streamed", "release_streamed_buffers",
     "set_device_timeout_ns", "set_debug_flags", "KernelTimer", "OP_DENSE", "OP_REUSE", "OP_REFINE", "BF16", "F32",
     "STATUS",
 ]
