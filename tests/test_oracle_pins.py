@@ -434,3 +434,103 @@ def test_aggregation_reductions(orc, mode):
     nz = lambda v: np.nan_to_num(v, nan=7.0)  # short rows are NaN padded
     assert np.array_equal(ui, di) and np.array_equal(nz(uv), nz(dv))
     assert np.array_equal(ri, di) and np.array_equal(nz(rv), nz(dv))
+
+
+# ----------------------------------------------------------------- the batch scorer used by the GPU checks
+
+
+def test_scores_batch_prefix_form_hand_example(orc):
+    """Prefix form (plen): row t of the hand-worked example holds I_{t,s} for s <= t, as
+    derived by hand in the golden file, and NaN past its prefix."""
+    q, w, k = _hand()
+    L = q.shape[0]
+    qv, wv = orc.query_rows(q, w, range(L))
+    F = orc.scores_batch(qv, wv, k, plen=np.arange(L) + 1)
+    assert F.shape == (L, L)
+    for t in range(L):
+        assert F[t, :t + 1].tolist() == GOLD["dense_scores"][t][:t + 1]
+        assert np.isnan(F[t, t + 1:]).all()
+
+
+def test_scores_batch_key_rows_form_closed_form(orc):
+    """key_rows form: entry i scores key key_rows[r, i] (NaN where it is -1).  With one-hot
+    keys k_s = e_s the score has the closed form sum_j w_j max(0, q_{j,s})."""
+    L, H = 11, 3
+    q, w, k = _onehot(L, H, 21)
+    rows = [2, 7, 10]
+    qv, wv = orc.query_rows(q, w, rows)
+    rng = np.random.default_rng(22)
+    kr = rng.integers(0, L, size=(len(rows), 6))
+    kr[0, 1] = -1
+    kr[2, 4] = -1
+    kr[1, 5] = -1
+    F = orc.scores_batch(qv, wv, k, key_rows=kr)
+    for r, t in enumerate(rows):
+        for i, s in enumerate(kr[r]):
+            if s < 0:
+                assert np.isnan(F[r, i])
+                continue
+            closed = sum(float(w[t, j]) * max(0.0, float(q[t, j, s])) for j in range(H))
+            assert abs(F[r, i] - closed) <= 1e-12 * (1 + abs(closed)), (r, i)
+
+
+def test_scores_batch_key_base_offsets_each_vector(orc):
+    """key_base: vector r reads its keys from row key_base[r] on, in both forms.  The keys
+    are a block of filler rows followed by one-hot rows, so only the right offset lands on
+    the closed form; a vector with base 0 must see the filler instead."""
+    H, n1 = 2, 7
+    rng = np.random.default_rng(23)
+    filler = (rng.standard_normal((5, n1)) + 3.0).astype(np.float32)
+    k = np.concatenate([filler, np.eye(n1, dtype=np.float32)])
+    qv = rng.standard_normal((3, H * n1))
+    wv = rng.standard_normal((3, H))
+    base = np.array([5, 5, 0])
+    Fp = orc.scores_batch(qv, wv, k, plen=np.array([n1, 4, n1]), key_base=base)
+    kr = np.array([[0, 3, 6], [6, -1, 1], [0, 1, 2]])
+    Fk = orc.scores_batch(qv, wv, k, key_rows=kr, key_base=base, m=3)
+    for r in range(2):  # one-hot block at rows 5..11
+        qq = qv[r].reshape(H, n1)
+        closed = [sum(wv[r, j] * max(0.0, qq[j, s]) for j in range(H)) for s in range(n1)]
+        plen = (n1, 4)[r]
+        assert np.allclose(Fp[r, :plen], closed[:plen], rtol=1e-12, atol=1e-12)
+        assert np.isnan(Fp[r, plen:]).all()
+        for i, s in enumerate(kr[r]):
+            assert np.isnan(Fk[r, i]) if s < 0 else abs(Fk[r, i] - closed[s]) <= 1e-12
+    # base 0: filler rows, whose scores are the plain double dot products
+    qq = qv[2].reshape(H, n1)
+    want = [sum(wv[2, j] * max(0.0, float(np.dot(qq[j].astype(np.float64), filler[s].astype(np.float64))))
+                for j in range(H)) for s in range(3)]
+    assert np.allclose(Fk[2], want, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("dt", [np.float32, np.uint16])
+def test_scores_batch_agrees_with_the_pinned_entry_points(orc, dt):
+    """The batch scorer reproduces what the pinned calls return: the dense indexer's row
+    scores, the proxy scores of a group (prefix form) and a Refine member row's scores
+    over its candidate set (key_rows form), value for value."""
+    L, H, d, topk, c, g = 45, 3, 16, 7, 14, 4
+    q, w, k = _rand(L, H, d, 24, dt)
+    didx, dval = orc.dense(q, w, k, topk)
+    rows = [0, 13, 44]
+    qv, wv = orc.query_rows(q, w, rows)
+    F = orc.scores_batch(qv, wv, k, plen=np.array(rows) + 1)
+    for r, t in enumerate(rows):
+        for s, v in zip(didx[t], dval[t]):
+            if s >= 0:
+                assert F[r, s] == v
+    groups = [0, 5, (L + g - 1) // g - 1]
+    mem = [list(range(i * g, min(i * g + g, L))) for i in groups]
+    pq, pw = orc.proxies(q, w, mem)
+    Fp = orc.scores_batch(pq, pw, k, plen=np.array([m[-1] + 1 for m in mem]))
+    for r, i in enumerate(groups):
+        ps = orc.proxy_scores(q, w, k, g, i)
+        assert np.array_equal(Fp[r, :ps.size], ps)
+    ridx, rval, cand, _ = orc.refine(q, w, k, topk, c, g)
+    t = 22
+    grp = t // g
+    qv, wv = orc.query_rows(q, w, [t])
+    C = cand[grp:grp + 1].astype(np.int64)
+    M = orc.scores_batch(qv, wv, k, key_rows=C)
+    for s, v in zip(ridx[t], rval[t]):
+        if s >= 0:
+            assert M[0, list(C[0]).index(s)] == v
