@@ -51,49 +51,72 @@ def pooled(m, agg):
 # ---------------------------------------------------------------- checkers
 
 
-def check_dense(orc, x, idx, sc, rows, topk, key_base=None, pos=None):
+def check_dense(orc, x, idx, sc, rows, topk, pos=None, block=512):
+    """Dense rows `rows` of idx/sc (positions `pos`, default the row numbers) against
+    the oracle's scores of those queries over their prefixes; oracle scores are
+    computed `block` rows at a time."""
     q, w, k = x["q"], x["w"], x["k"]
     rows = list(rows)
     pos = rows if pos is None else list(pos)
-    qv, wv = orc.query_rows(q, w, rows)
-    F = orc.scores_batch(qv, wv, k, plen=np.array(pos) + 1, key_base=key_base)
     fails = []
-    for i, (r, t) in enumerate(zip(rows, pos)):
-        fails += check_row(idx[r], None if sc is None else sc[r], np.arange(t + 1), F[i, :t + 1],
-                           min(topk, t + 1), orc, f"dense row {r}")
+    for b0 in range(0, len(rows), block):
+        rb, pb = rows[b0:b0 + block], pos[b0:b0 + block]
+        qv, wv = orc.query_rows(q, w, rb)
+        F = orc.scores_batch(qv, wv, k, plen=np.array(pb) + 1)
+        for i, (r, t) in enumerate(zip(rb, pb)):
+            fails += check_row(idx[r], None if sc is None else sc[r], np.arange(t + 1), F[i, :t + 1],
+                               min(topk, t + 1), orc, f"dense row {r}")
     return fails
 
 
-def check_reuse(orc, x, idx, sc, groups, topk, g, agg="mean"):
+def check_reuse(orc, x, idx, sc, groups, topk, g, agg="mean", block=256):
     q, w, k = x["q"], x["w"], x["k"]
     L = q.shape[0]
-    mem = [members(L, g, i) for i in groups]
-    qv, wv = orc.proxies(q, w, [pooled(m, agg) for m in mem])
-    F = orc.scores_batch(qv, wv, k, plen=np.array([m[-1] + 1 for m in mem]))
+    groups = list(groups)
     fails = []
-    for gi, m in enumerate(mem):
-        for t in m:
-            fails += check_row(idx[t], None if sc is None else sc[t], np.arange(t + 1), F[gi, :t + 1],
-                               min(topk, t + 1), orc, f"reuse g={g} t={t}")
+    for b0 in range(0, len(groups), block):
+        mem = [members(L, g, i) for i in groups[b0:b0 + block]]
+        qv, wv = orc.proxies(q, w, [pooled(m, agg) for m in mem])
+        F = orc.scores_batch(qv, wv, k, plen=np.array([m[-1] + 1 for m in mem]))
+        for gi, m in enumerate(mem):
+            for t in m:
+                fails += check_row(idx[t], None if sc is None else sc[t], np.arange(t + 1), F[gi, :t + 1],
+                                   min(topk, t + 1), orc, f"reuse g={g} t={t}")
     return fails
 
 
-def check_refine(orc, x, idx, sc, cand, csc, groups, topk, c, g, agg="mean"):
+def check_refine(orc, x, idx, sc, cand, csc, groups, topk, c, g, agg="mean", block=64):
+    """Two levels: each group's C_i against the oracle's proxy scores, then every member
+    row against the oracle's re-scoring (Eq. 8) and top-k (Eq. 9) over that C_i."""
+    q, w, k = x["q"], x["w"], x["k"]
+    L = q.shape[0]
+    groups = list(groups)
+    fails = []
+    for b0 in range(0, len(groups), block):
+        gb = groups[b0:b0 + block]
+        mem = [members(L, g, i) for i in gb]
+        qv, wv = orc.proxies(q, w, [pooled(m, agg) for m in mem])
+        F = orc.scores_batch(qv, wv, k, plen=np.array([m[-1] + 1 for m in mem]))
+        for gi, (i, m) in enumerate(zip(gb, mem)):
+            e = m[-1]
+            fails += check_row(cand[i], None if csc is None else csc[i], np.arange(e + 1), F[gi, :e + 1],
+                               min(c, e + 1), orc, f"C_{i}")
+        fails += check_refine_rows(orc, x, idx, sc, cand, gb, topk, g)
+    return fails
+
+
+def check_refine_rows(orc, x, idx, sc, cand, groups, topk, g):
+    """Member rows of the given groups against the oracle's Eq. (8)-(9) over the
+    candidate sets `cand` (the GPU's own C_i)."""
     q, w, k = x["q"], x["w"], x["k"]
     L = q.shape[0]
     mem = [members(L, g, i) for i in groups]
-    qv, wv = orc.proxies(q, w, [pooled(m, agg) for m in mem])
-    F = orc.scores_batch(qv, wv, k, plen=np.array([m[-1] + 1 for m in mem]))
-    fails = []
-    for gi, (i, m) in enumerate(zip(groups, mem)):
-        e = m[-1]
-        fails += check_row(cand[i], None if csc is None else csc[i], np.arange(e + 1), F[gi, :e + 1],
-                           min(c, e + 1), orc, f"C_{i}")
     rows = [t for m in mem for t in m]
     grp_of = [i for i, m in zip(groups, mem) for _ in m]
     qv, wv = orc.query_rows(q, w, rows)
     C = np.stack([cand[i] for i in grp_of]).astype(np.int64)
     M = orc.scores_batch(qv, wv, k, key_rows=C)
+    fails = []
     for r, (t, i) in enumerate(zip(rows, grp_of)):
         ok = (C[r] >= 0) & (C[r] <= t)
         E, f = C[r][ok], M[r][ok]
@@ -243,29 +266,29 @@ def test_reuse_g1_equals_dense_on_gpu():
 # ---------------------------------------------------------------- the workloads at full size
 
 
-def test_prefill_8k_sampled(orc):
+def test_prefill_8k_every_group(orc):
+    """The 8K prefill workload: every one of its 1024 groups (Refine at both levels,
+    Reuse on every member row) and every dense row, against the oracle."""
     s = inputs.PREFILL_8K
     x = inputs.make_prefill(s)
     res = run_all(x, s.k, s.c, s.g)
-    G = (s.L + s.g - 1) // s.g
-    groups = inputs.sample_groups(G, s.g, s.k, s.c, 96, s.seed + 1000)
-    rows = sorted({int(t) for i in groups for t in members(s.L, s.g, int(i))})[::4]
-    fails = full_check(orc, x, res, s.k, s.c, s.g, groups=groups, dense_rows=rows)
+    fails = full_check(orc, x, res, s.k, s.c, s.g)
     assert not fails, summarize(fails)
 
 
 @pytest.mark.parametrize("rho", inputs.SWEEP_RHO)
 @pytest.mark.parametrize("g", inputs.SWEEP_G)
 def test_sweep_32k_sampled(orc, g, rho):
+    """Each point of the L = 32768 group-size sweep: Reuse and Refine on 256 seeded groups."""
     s = inputs.sweep_32k(g, rho)
     x = inputs.make_prefill(s)
     q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
-    u_idx, _ = P.reuse(q, w, k, s.k, g)
+    u_idx, u_sc = P.reuse(q, w, k, s.k, g, scores=True)
     r_idx, r_sc, r_c, r_cs = P.refine(q, w, k, s.k, s.c, g, scores=True, cand=True)
     torch.cuda.synchronize()
     G = (s.L + g - 1) // g
-    groups = inputs.sample_groups(G, g, s.k, s.c, 24, s.seed + 1000 + g)
-    fails = check_reuse(orc, x, host(u_idx), None, groups, s.k, g)
+    groups = inputs.sample_groups(G, g, s.k, s.c, 256, s.seed + 1000 + g)
+    fails = check_reuse(orc, x, host(u_idx), host(u_sc), groups, s.k, g)
     fails += check_refine(orc, x, host(r_idx), host(r_sc), host(r_c), host(r_cs), groups, s.k, s.c, g)
     assert not fails, summarize(fails)
 
@@ -276,6 +299,8 @@ def long_inputs():
 
 
 def test_long_128k_refine_reuse_dense_sampled(orc, long_inputs):
+    """The L = 131072 headline workload on 256 seeded groups: Refine at both levels,
+    Reuse and the dense indexer on every member row of those groups."""
     s = inputs.LONG_128K
     x = long_inputs
     q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
@@ -286,8 +311,8 @@ def test_long_128k_refine_reuse_dense_sampled(orc, long_inputs):
     G = (s.L + s.g - 1) // s.g
     groups = inputs.sample_groups(G, s.g, s.k, s.c, 256, s.seed + 1000)
     fails = check_refine(orc, x, host(r_idx), host(r_sc), host(r_c), host(r_cs), groups, s.k, s.c, s.g)
-    fails += check_reuse(orc, x, host(u_idx), host(u_sc), groups[::4], s.k, s.g)
-    rows = [int(i) * s.g + (int(i) % s.g) for i in groups[::2]]
+    fails += check_reuse(orc, x, host(u_idx), host(u_sc), groups, s.k, s.g)
+    rows = [t for i in groups for t in members(s.L, s.g, int(i))]
     fails += check_dense(orc, x, host(d_idx), host(d_sc), rows, s.k)
     assert not fails, summarize(fails)
 
@@ -367,19 +392,11 @@ def test_decode_duplicate_keys_lowest_index_wins(orc):
 
 
 def test_decode_small_ragged(orc):
-    spec = inputs.DecodeSpec("small", B=5, p_lo=4, p_hi=3000, H=64, d=128, k=64, c=128, g=4, seed=21)
-    x = inputs.make_decode(spec)
-    off = x["offsets"]
-    q, w, kc = dev(x["q"]), dev(x["w"]), dev(x["k"])
-    u_idx, _ = P.reuse_varlen(q, w, kc, off, spec.k, spec.g)
-    r_idx, _, r_c, _ = P.refine_varlen(q, w, kc, off, spec.k, spec.c, spec.g, cand=True)
-    o_u, _, _, _ = orc.decode(x["q"], x["w"], x["k"], off, spec.k, spec.c, spec.g, 0)
-    o_r, _, _, _ = orc.decode(x["q"], x["w"], x["k"], off, spec.k, spec.c, spec.g, 1, cand_in=host(r_c))
-    for got, want in ((host(u_idx), o_u), (host(r_idx), o_r)):
-        for row in range(got.shape[0]):
-            a = set(got[row][got[row] >= 0].tolist())
-            b = set(want[row][want[row] >= 0].tolist())
-            assert len(a ^ b) <= 2, (row, len(a ^ b))
+    """Five sequences with prefixes from 4 to 3000 keys (several at or under c and k + g - 1):
+    every C row, Reuse row and Refine row against the oracle."""
+    s = inputs.DecodeSpec("small", B=5, p_lo=4, p_hi=3000, H=64, d=128, k=64, c=128, g=4, seed=21)
+    fails, _ = _decode_batch_fails(orc, s, inputs.make_decode(s))
+    assert not fails, summarize(fails)
 
 
 # ---------------------------------------------------------------- scan visiting orders
@@ -417,49 +434,69 @@ def test_sampled_order_natural_order_and_fallback_agree(orc):
 # ---------------------------------------------------------------- one sequence split into group ranges
 
 
-def test_group_ranges_reproduce_the_whole_sequence():
+def test_group_ranges_reproduce_the_whole_sequence(orc):
     """The zig-zag chunks of a 4-rank split, each run as a group-range call with only
     its rows and its key prefix, give exactly the rows of the whole-sequence call
-    (dense, Reuse, Refine; tensor-core and CUDA-core paths)."""
+    (dense, Reuse, Refine; tensor-core and CUDA-core paths), and the rows assembled
+    from the chunks pass the oracle checks on every group."""
     from top_token_selection_proxy_b200 import multigpu as M
 
     for x, topk, c, g in ((inputs.random_prefill(4096, 64, 128, inputs.BF16, seed=73), 128, 256, 8),
                           (inputs.make_prefill(inputs.TINY), inputs.TINY.k, inputs.TINY.c, inputs.TINY.g)):
         q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
         L = x["q"].shape[0]
+        G = (L + g - 1) // g
         full = {"dense": host(P.indexer_dense(q, w, k, topk)[0]), "reuse": host(P.reuse(q, w, k, topk, g)[0]),
                 "refine": host(P.refine(q, w, k, topk, c, g)[0])}
+        got = {n: np.full((L, topk), -2, np.int32) for n in ("dense", "reuse", "refine")}
+        got_sc = {n: np.full((L, topk), np.nan, np.float32) for n in got}
+        cand = np.full((G, c), -2, np.int32)
         world = 4
         for r in range(world):
             for t0, t1 in M.zigzag_chunks(L, g, world, r):
                 qr, wr, kp = q[t0:t1].contiguous(), w[t0:t1].contiguous(), k[:t1].contiguous()
-                got = {"dense": host(P.indexer_dense_range(qr, wr, kp, L, topk, t0, t1)[0]),
-                       "reuse": host(P.reuse_range(qr, wr, kp, L, topk, g, t0 // g, t1 // g)[0]),
-                       "refine": host(P.refine_range(qr, wr, kp, L, topk, c, g, t0 // g, t1 // g)[0])}
+                d_i, d_s = P.indexer_dense_range(qr, wr, kp, L, topk, t0, t1, scores=True)
+                u_i, u_s = P.reuse_range(qr, wr, kp, L, topk, g, t0 // g, t1 // g if t1 < L else G, scores=True)
+                r_i, r_s, r_c, _ = P.refine_range(qr, wr, kp, L, topk, c, g, t0 // g, t1 // g if t1 < L else G,
+                                                  scores=True, cand=True)
                 torch.cuda.synchronize()
-                for name in full:
-                    assert np.array_equal(np.sort(got[name], axis=1), np.sort(full[name][t0:t1], axis=1)), \
-                        f"{name} rows [{t0}, {t1}) of L = {L}"
+                for n, (i_, s_) in (("dense", (d_i, d_s)), ("reuse", (u_i, u_s)), ("refine", (r_i, r_s))):
+                    got[n][t0:t1], got_sc[n][t0:t1] = host(i_), host(s_)
+                cand[t0 // g:(t1 + g - 1) // g] = host(r_c)
+        for name in full:
+            assert (got[name] != -2).all(), f"{name}: rows not covered by the chunks"
+            assert np.array_equal(np.sort(got[name], axis=1), np.sort(full[name], axis=1)), f"{name}, L = {L}"
+        assert (cand != -2).all()
+        fails = check_dense(orc, x, got["dense"], got_sc["dense"], range(L), topk)
+        fails += check_reuse(orc, x, got["reuse"], got_sc["reuse"], range(G), topk, g)
+        fails += check_refine(orc, x, got["refine"], got_sc["refine"], cand, None, range(G), topk, c, g)
+        assert not fails, summarize(fails)
 
 
-def test_streamed_refine_from_host_memory_matches_one_call():
+def test_streamed_refine_from_host_memory_matches_one_call(orc):
     """refine_streamed (pinned host inputs, copies overlapped with group-range calls in
     chunks) writes exactly the rows of one device-resident refine call, for a ragged
     length and chunk counts that do and do not divide the groups; twice in a row
-    (buffer reuse, earlier output overwritten)."""
+    (buffer reuse, earlier output overwritten).  Its rows also pass the oracle's
+    re-scoring and top-k (Eq. 8-9) over the one call's candidate sets, every group."""
     x = inputs.random_prefill(6001, 64, 128, inputs.BF16, seed=79)
     topk, c, g = 128, 256, 8
     q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
-    want = np.sort(host(P.refine(q, w, k, topk, c, g)[0]), axis=1)
+    one_idx, _, one_c, one_cs = P.refine(q, w, k, topk, c, g, scores=True, cand=True)
+    want = np.sort(host(one_idx), axis=1)
+    cand, cand_sc = host(one_c), host(one_cs)
     qh = torch.from_numpy(x["q"].view(np.int16)).pin_memory().view(torch.bfloat16)
     wh = torch.from_numpy(x["w"]).pin_memory()
     kh = torch.from_numpy(x["k"].view(np.int16)).pin_memory().view(torch.bfloat16)
     oh = torch.empty((q.shape[0], topk), dtype=torch.int32).pin_memory()
+    G = (6001 + g - 1) // g
     for chunks in (1, 3, 8, 8):
         oh.fill_(-7)
         P.refine_streamed(qh, wh, kh, topk, c, g, out_host=oh, chunks=chunks)
         torch.cuda.current_stream().synchronize()
         assert np.array_equal(np.sort(oh.numpy(), axis=1), want), f"chunks = {chunks}"
+    fails = check_refine(orc, x, oh.numpy().copy(), None, cand, cand_sc, range(G), topk, c, g)
+    assert not fails, summarize(fails)
 
 
 # ---------------------------------------------------------------- proxy aggregation variants
@@ -485,29 +522,43 @@ def test_aggregation_variants_every_group(orc, agg):
 # ---------------------------------------------------------------- guardrail
 
 
-def test_guardrail_runs_the_chosen_path_exactly():
+def test_guardrail_runs_the_chosen_path_exactly(orc):
     """Behind the guardrail the call returns exactly the rows of the path it picks:
-    dense at short context (c >= L), Refine / Reuse otherwise."""
+    dense at short context (c >= L), Refine / Reuse otherwise; the guarded rows also
+    pass the oracle checks of that path on every row."""
     g, c, topk = 8, 512, 256
     for L, want_dense in ((400, True), (4096, False)):
         x = inputs.random_prefill(L, 64, 128, inputs.BF16, seed=40 + L)
         q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
+        G = (L + g - 1) // g
         assert P.guardrail_dense(P.OP_REFINE, L, c, g) == want_dense
         gi, gs, ran_dense = P.refine_guarded(q, w, k, topk, c, g, scores=True)
         assert ran_dense == want_dense
-        ri, rs = P.indexer_dense(q, w, k, topk, scores=True) if want_dense else \
-            P.refine(q, w, k, topk, c, g, scores=True)[:2]
+        if want_dense:
+            ri, rs = P.indexer_dense(q, w, k, topk, scores=True)
+            rc = None
+        else:
+            ri, rs, rc, _ = P.refine(q, w, k, topk, c, g, scores=True, cand=True)
         torch.cuda.synchronize()
         assert np.array_equal(np.sort(host(gi), axis=1), np.sort(host(ri), axis=1))
-        ui, _, ran_dense_u = P.reuse_guarded(q, w, k, topk, g)
+        if want_dense:
+            fails = check_dense(orc, x, host(gi), host(gs), range(L), topk)
+        else:  # the guarded call's rows against the oracle over the Refine path's C_i
+            fails = check_refine_rows(orc, x, host(gi), host(gs), host(rc), range(G), topk, g)
+        ui, us, ran_dense_u = P.reuse_guarded(q, w, k, topk, g, scores=True)
         assert not ran_dense_u
+        torch.cuda.synchronize()
         assert np.array_equal(np.sort(host(ui), axis=1), np.sort(host(P.reuse(q, w, k, topk, g)[0]), axis=1))
+        fails += check_reuse(orc, x, host(ui), host(us), range(G), topk, g)
+        assert not fails, summarize(fails)
     # g = 1: Reuse and dense do the same work, the guardrail runs dense
     x = inputs.random_prefill(300, 64, 128, inputs.BF16, seed=41)
     q, w, k = dev(x["q"]), dev(x["w"]), dev(x["k"])
-    ui, _, ran_dense_u = P.reuse_guarded(q, w, k, 64, 1)
+    ui, us, ran_dense_u = P.reuse_guarded(q, w, k, 64, 1, scores=True)
     assert ran_dense_u
     assert np.array_equal(np.sort(host(ui), axis=1), np.sort(host(P.indexer_dense(q, w, k, 64)[0]), axis=1))
+    fails = check_dense(orc, x, host(ui), host(us), range(300), 64)
+    assert not fails, summarize(fails)
 
 
 # ---------------------------------------------------------------- failure paths (no GPU fault)
