@@ -254,17 +254,22 @@ PIVOT_API void pivot_set_profile_events(void **events, int n);
  * nor hand over a workspace.  Computes exactly what pivot_reuse computes,
  * with the same arguments minus the workspace, on the tensor-core scan
  * kernel; its scratch (status word, work counter, candidate buffers) is a
- * fixed static device array of 8 MiB + 256 B that every process loading this
- * library holds on every device it uses until exit.
+ * fixed static device array of 12,124,416 B + 256 B (about 11.6 MiB) that
+ * every process loading this library holds on every device it uses until
+ * exit.
  * Limits: bf16 q/k, H = 64, d in {64, 128}, g <= 16 and k + g - 1 <= 256;
- * larger sizes return PIVOT_ERR_UNSUPPORTED_SHAPE without launching.
+ * larger sizes return PIVOT_ERR_UNSUPPORTED_SHAPE without launching.  At most
+ * 148 CTAs run (one per SM).
  * The first call on a device looks the array's device address up (once per
  * device, with that device current); make that first call before any stream
  * capture.  All calls share the one array and it keeps the last call's
  * contents: calls that overlap on the GPU (other streams, other host
  * threads) race and give undefined results, so order them.  Device-side
- * wait timeouts of this variant are not reported (there is no workspace for
- * pivot_last_device_status to read).  Allocates nothing. */
+ * waits are bounded by pivot_set_device_timeout_ns like every other call,
+ * but a wait that runs out is not reported (there is no workspace for
+ * pivot_last_device_status to read); the outputs are then undefined.
+ * pivot_last_cuda_error describes a PIVOT_ERR_CUDA return.  Allocates
+ * nothing. */
 PIVOT_API pivot_status pivot_reuse_noalloc(const void *q_I, const float *w_I, const void *k_I, int64_t L, int H,
                                            int d, pivot_dtype dt, int k, int g, int32_t *indices, float *scores_opt,
                                            pivot_stream_t stream);

@@ -3,8 +3,9 @@ memory (their device memory belongs to a pool or planner they do not
 control), with its scratch in a static device array instead of a caller
 workspace.  Checked through the C ABI against pivot_reuse, the entry point
 with a workspace, on two calls in a row (the array keeps the previous call's
-contents, so the second call checks that what must start cleared is cleared).
-This file is collected last on purpose."""
+contents, so the second call checks that what must start cleared is cleared),
+and against the CPU oracle on every group.  This file is collected last on
+purpose."""
 import ctypes
 
 import numpy as np
@@ -12,6 +13,7 @@ import pytest
 import torch
 
 import top_token_selection_proxy_b200 as P
+from parity import check_row, summarize
 from top_token_selection_proxy_b200 import inputs
 
 pytestmark = pytest.mark.gpu
@@ -53,15 +55,33 @@ def _same_rows(a_idx, a_sc, b_idx, b_sc):
                 assert abs(v - lo) <= TOL_ABS + TOL_REL * abs(lo), (t, s)
 
 
-def test_reuse_noalloc_matches_workspace_entry_point_twice():
+def _oracle_fails(orc, x, idx, sc, topk, g):
+    """Every member row against the oracle's Eq. (4)-(6): proxy scores over s <= t."""
+    L = x["q"].shape[0]
+    G = (L + g - 1) // g
+    mem = [list(range(i * g, min(i * g + g, L))) for i in range(G)]
+    qv, wv = orc.proxies(x["q"], x["w"], mem)
+    F = orc.scores_batch(qv, wv, x["k"], plen=np.array([m[-1] + 1 for m in mem]))
+    fails = []
+    for i, m in enumerate(mem):
+        for t in m:
+            fails += check_row(idx[t], sc[t], np.arange(t + 1), F[i, :t + 1], min(topk, t + 1), orc,
+                               f"noalloc reuse t={t}")
+    return fails
+
+
+@pytest.mark.parametrize("L,topk,g", [(3001, 120, 8), (4000, 249, 8)])
+def test_reuse_noalloc_matches_workspace_entry_point_twice(orc, L, topk, g):
+    """k + g - 1 = 127 (several tiles and cut-backs) and = 256, the largest selection the
+    static scratch takes (its sub-buffers run their cut-backs closest to full)."""
     from top_token_selection_proxy_b200 import build
 
     build.build()
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     lib = P.lib()
-    L, H, d, topk, g = 3001, 64, 128, 120, 8  # k + g - 1 = 127 <= 256; several tiles and cut-backs
-    x = inputs.random_prefill(L, H, d, inputs.BF16, seed=4242)
+    H, d = 64, 128
+    x = inputs.random_prefill(L, H, d, inputs.BF16, seed=4242 + topk)
     q, w, k = _dev(x["q"]), _dev(x["w"]), _dev(x["k"])
     ref_idx, ref_sc = P.reuse(q, w, k, topk, g, scores=True)
     torch.cuda.synchronize()
@@ -70,7 +90,10 @@ def test_reuse_noalloc_matches_workspace_entry_point_twice():
         st, idx, sc = _noalloc(lib, q, w, k, topk, g)
         assert st == 0, P.STATUS.get(st, st)
         torch.cuda.synchronize()
-        _same_rows(idx.cpu().numpy(), sc.cpu().numpy(), ref_idx, ref_sc)
+        idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+        _same_rows(idx, sc, ref_idx, ref_sc)
+        fails = _oracle_fails(orc, x, idx, sc, topk, g)
+        assert not fails, summarize(fails)
 
 
 def test_reuse_noalloc_rejects_sizes_beyond_its_scratch():

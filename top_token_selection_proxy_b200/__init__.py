@@ -353,6 +353,16 @@ def refine_streamed(q_host, w_host, k_host, topk: int, c: int, g: int, *, out_ho
     if w_host.shape != (L, H) or k_host.shape != (L, d) or out_host.shape != (L, topk):
         raise ValueError("expected q [L,H,d], w [L,H], k [L,d], out [L,topk]")
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if dev.type != "cuda" or dev.index is None:
+        raise ValueError("device must name one CUDA device, e.g. 'cuda:0'")
+    # the C calls take SMs, tensor maps and the launch from the calling thread's current
+    # device: make `dev` current for the whole call
+    with torch.cuda.device(dev):
+        return _refine_streamed_on(dev, q_host, w_host, k_host, topk, c, g, out_host, chunks, ws)
+
+
+def _refine_streamed_on(dev, q_host, w_host, k_host, topk, c, g, out_host, chunks, ws):
+    L, H, d = q_host.shape
     pl = _pipelines.get(dev.index)
     if pl is None or pl.shape != (L, H, d, topk):
         _drop_pipeline(dev.index)

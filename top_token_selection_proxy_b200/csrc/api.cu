@@ -518,6 +518,14 @@ pivot_status run_decode(int op, const void* q, const float* w, const void* kc, c
 
 }  // namespace
 
+// Library-internal hooks for the other host files (hidden: not part of the C ABI).
+namespace pivot {
+uint64_t device_timeout_ns() { return g_timeout_ns; }
+int debug_flags() { return g_debug_flags; }
+void clear_cuda_error() { g_cuda_err[0] = 0; }
+pivot_status record_cuda_error(cudaError_t e, const char* what) { return cuda_fail(e, what); }
+}  // namespace pivot
+
 extern "C" {
 
 size_t pivot_workspace_size(int op, int64_t L, int H, int d, int k, int c, int g, pivot_dtype dt) {

@@ -150,4 +150,10 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, const CU
                           int slices, cudaStream_t s);
 size_t decode_scan_smem_bytes(int D);
 
+// host-side library state shared by the entry-point files (defined in api.cu)
+uint64_t device_timeout_ns();     // bound on every device-side wait (pivot_set_device_timeout_ns)
+int debug_flags();                // pivot_set_debug_flags
+void clear_cuda_error();          // start of an entry point: pivot_last_cuda_error() reads ""
+pivot_status record_cuda_error(cudaError_t e, const char* what);  // remember e; returns PIVOT_ERR_CUDA
+
 }  // namespace pivot

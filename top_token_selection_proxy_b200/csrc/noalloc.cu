@@ -13,8 +13,11 @@
 // is an integration convenience, not part of the method.
 //
 // Limits: bf16 q/k, H = 64, d in {64, 128}, g <= 16, k + g - 1 <= 256, and
-// at most 128 CTAs (one per SM up to 128).  Scratch is
-//   256 B (status + counters) + 128 CTAs * 4 groups * 4 sub-buffers * 512 entries * 8 B = 8 MiB.
+// at most 148 CTAs (one per SM up to 148).  Each candidate sub-buffer gets the
+// same slack as on the workspace path (selection size + 384, rounded up to 64:
+// 640 entries for the largest selection of 256).  Scratch is
+//   256 B (status + counters) + 148 CTAs * 4 groups * 4 sub-buffers * 640 entries * 8 B
+//   = 12,124,416 B + 256 B (about 11.6 MiB).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -29,12 +32,13 @@ using namespace pivot;
 namespace {
 
 constexpr int kMaxSel = 256;                   // k + g - 1
-constexpr int kSubCap = 512;                   // entries per (group, lane quarter) sub-buffer: >= kMaxSel + 256
-constexpr int kMaxCtas = 128;
+constexpr int kSubCap = 640;                   // entries per (group, lane quarter) sub-buffer: kMaxSel + 384
+constexpr int kMaxCtas = 148;
 constexpr int kGroupsPerItem = 4;              // 256 / H with H = 64
 constexpr size_t kHdrBytes = 256;              // status word + counters
 constexpr size_t kSelBytes = (size_t)kMaxCtas * kGroupsPerItem * 4 * kSubCap * sizeof(uint64_t);
-constexpr size_t kStaticBytes = kHdrBytes + kSelBytes;  // 8 MiB + 256 B
+constexpr size_t kStaticBytes = kHdrBytes + kSelBytes;  // 12,124,416 B + 256 B
+static_assert(kSubCap >= kMaxSel + 384 && kSubCap % 64 == 0, "the workspace path's sub-buffer slack");
 
 // The scratch itself.  In host code this name is only a host-side stand-in:
 // the device address comes from cudaGetSymbolAddress below.
@@ -72,6 +76,7 @@ bool encode_keys(CUtensorMap* m, const void* base, int64_t rows, int d) {
 extern "C" PIVOT_API pivot_status pivot_reuse_noalloc(const void* q_I, const float* w_I, const void* k_I, int64_t L,
                                                       int H, int d, pivot_dtype dt, int k, int g, int32_t* indices,
                                                       float* scores_opt, pivot_stream_t stream) {
+  clear_cuda_error();
   if (!q_I || !w_I || !k_I || !indices || L <= 0 || k <= 0 || g <= 0) return PIVOT_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(q_I) & 15u) || (reinterpret_cast<uintptr_t>(k_I) & 15u))
     return PIVOT_ERR_INVALID_ARG;
@@ -80,13 +85,17 @@ extern "C" PIVOT_API pivot_status pivot_reuse_noalloc(const void* q_I, const flo
   if (k + g - 1 > kMaxSel) return PIVOT_ERR_UNSUPPORTED_SHAPE;  // beyond the static scratch
 
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return PIVOT_ERR_CUDA;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return record_cuda_error(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return record_cuda_error(cudaErrorInvalidDevice, "device ordinal beyond 63");
   void* base = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_addr[dev]) {  // first call on this device: look the array up once
       void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return PIVOT_ERR_CUDA;
+      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess) return record_cuda_error(e, "cudaGetSymbolAddress");
+      if (p == nullptr) return record_cuda_error(cudaErrorInvalidSymbol, "cudaGetSymbolAddress");
       g_addr[dev] = p;
     }
     base = g_addr[dev];
@@ -95,18 +104,20 @@ extern "C" PIVOT_API pivot_status pivot_reuse_noalloc(const void* q_I, const flo
   char* hdr = reinterpret_cast<char*>(base);
   // the array keeps the previous call's contents: the status word and the work
   // counter must start at zero (the candidate buffers are written before read)
-  if (cudaMemsetAsync(hdr, 0, kHdrBytes, s) != cudaSuccess) return PIVOT_ERR_CUDA;
+  e = cudaMemsetAsync(hdr, 0, kHdrBytes, s);
+  if (e != cudaSuccess) return record_cuda_error(e, "cudaMemsetAsync");
 
   int sms = 0;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-    return PIVOT_ERR_CUDA;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return record_cuda_error(e, "cudaDeviceGetAttribute");
+  if (sms <= 0) return record_cuda_error(cudaErrorInvalidValue, "multiprocessor count");
   const int n_sel = k + g - 1;
   const int64_t n_groups = (L + g - 1) / g;
   const int n_items = (int)((n_groups + kGroupsPerItem - 1) / kGroupsPerItem);
   const int grid = (int)std::min<int64_t>(std::min(sms, kMaxCtas), n_items);
 
   CUtensorMap kmap;
-  if (!encode_keys(&kmap, k_I, L, d)) return PIVOT_ERR_CUDA;
+  if (!encode_keys(&kmap, k_I, L, d)) return record_cuda_error(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
   ScanArgs a{};
   a.q = reinterpret_cast<const uint16_t*>(q_I);
   a.w = w_I;
@@ -127,7 +138,8 @@ extern "C" PIVOT_API pivot_status pivot_reuse_noalloc(const void* q_I, const flo
   a.sub_cap = kSubCap;
   a.counter = reinterpret_cast<unsigned int*>(hdr + 64);
   a.status = reinterpret_cast<int*>(hdr);
-  a.timeout_ns = 2000000000ull;
-  a.debug_flags = 0;
-  return launch_scan(a, &kmap, grid, s) == cudaSuccess ? PIVOT_OK : PIVOT_ERR_CUDA;
+  a.timeout_ns = device_timeout_ns();  // the bound pivot_set_device_timeout_ns sets for every call
+  a.debug_flags = 0;                   // the test hooks apply to the workspace entry points only
+  e = launch_scan(a, &kmap, grid, s);
+  return e == cudaSuccess ? PIVOT_OK : record_cuda_error(e, "scan kernel");
 }
