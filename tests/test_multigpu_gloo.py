@@ -87,15 +87,28 @@ def _zigzag_rank(rank: int, world: int, port: int, outdir: str) -> None:
     L, g, k, c = _zigzag_case(world)
     x = inputs.random_prefill(L, 4, 16, inputs.F32, seed=97)   # every rank draws the same sequence
     chunks = M.zigzag_chunks(L, g, world, rank)
-    k_local = torch.from_numpy(np.concatenate([x["k"][t0:t1] for t0, t1 in chunks]))
-    k_full = M.gather_keys(k_local, L, g, world).numpy()
+    # the rank holds only its chunks' rows; split_step gathers the keys and indexes each chunk
+    q_loc, w_loc = M.local_rows(x["q"], chunks), M.local_rows(x["w"], chunks)
+    k_loc = M.local_rows(torch.from_numpy(x["k"]), chunks)
+    seen = {}
+
+    def index_fn(q_rows, w_rows, k_prefix, t0, t1):
+        kp = k_prefix.numpy()
+        seen[t0] = bool(np.array_equal(kp, x["k"][:t1]))
+        # the chunk's groups from its own rows: a sequence whose rows before t0 are never read
+        # except as keys (their queries are zero-filled here)
+        qq = np.zeros((t1,) + x["q"].shape[1:], x["q"].dtype)
+        ww = np.zeros((t1,) + x["w"].shape[1:], x["w"].dtype)
+        qq[t0:t1], ww[t0:t1] = q_rows, w_rows
+        idx, val, _, _ = orc.refine(qq, ww, kp, k, c, g, g0=t0 // g, g1=t1 // g)
+        return idx, val
+
     rows = {}
-    for t0, t1 in chunks:  # the rank's groups, from the gathered keys
-        idx, val, _, _ = orc.refine(x["q"], x["w"], k_full, k, c, g, g0=t0 // g, g1=t1 // g)
+    for t0, t1, (idx, val) in M.split_step(index_fn, q_loc, w_loc, k_loc, L, g, world, rank):
         rows[t0] = (idx.tolist(), np.nan_to_num(val, nan=7.0).tolist())
     work = [M.chunk_work(L, g, c, t0, t1) for t0, t1 in chunks]
     with open(os.path.join(outdir, f"zz{rank}.json"), "w") as f:
-        json.dump({"keys_equal": bool(np.array_equal(k_full, x["k"])), "rows": rows, "work": sum(work)}, f)
+        json.dump({"keys_equal": all(seen.values()) and len(seen) == 2, "rows": rows, "work": sum(work)}, f)
     M.finish(world)
 
 

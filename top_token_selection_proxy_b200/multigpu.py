@@ -104,6 +104,32 @@ def gather_keys(k_local: torch.Tensor, L: int, g: int, world: int) -> torch.Tens
     return full
 
 
+def local_rows(a, chunks):
+    """This rank's rows of a per-position array (numpy or torch): its chunks, concatenated
+    in zigzag_chunks order."""
+    parts = [a[t0:t1] for t0, t1 in chunks]
+    if isinstance(a, torch.Tensor):
+        return torch.cat(parts).contiguous()
+    import numpy as np
+
+    return np.ascontiguousarray(np.concatenate(parts))
+
+
+def split_step(index_fn, q_local, w_local, k_local, L: int, g: int, world: int, rank: int):
+    """One step of one sequence indexed by `world` ranks: the all-gather of the key chunks
+    (the one exchange), then index_fn(q_rows, w_rows, k_prefix, t0, t1) on each of this
+    rank's zig-zag chunks, with that chunk's query / weight rows and the key prefix
+    [0, t1) it reads.  q_local / w_local / k_local hold the rank's chunks (local_rows).
+    Returns [(t0, t1, index_fn's result)]."""
+    k_full = gather_keys(k_local, L, g, world)
+    out, off = [], 0
+    for t0, t1 in zigzag_chunks(L, g, world, rank):
+        n = t1 - t0
+        out.append((t0, t1, index_fn(q_local[off:off + n], w_local[off:off + n], k_full[:t1], t0, t1)))
+        off += n
+    return out
+
+
 def finish(world: int) -> None:
     """Every rank calls this last: a final barrier, then leave the process group."""
     if world > 1 and dist.is_initialized():
@@ -112,4 +138,4 @@ def finish(world: int) -> None:
 
 
 __all__ = ["SEED_STRIDE", "env", "init", "rank_seed", "barrier", "max_over_ranks", "weak_scaling", "finish",
-           "zigzag_chunks", "chunk_work", "gather_keys"]
+           "zigzag_chunks", "chunk_work", "gather_keys", "local_rows", "split_step"]
