@@ -74,6 +74,11 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--no-extras", action="store_true", help="skip dense/Reuse/decode side measurements")
+    p.add_argument("--no-configs", action="store_true", help="skip the per-workload lines (tiny, 8K, 32K sweep, "
+                                                             "decode)")
+    p.add_argument("--split", action="store_true",
+                   help="one L=131072 sequence over all ranks (zig-zag group ranges + key all-gather; strong "
+                        "scaling) instead of one sequence per rank")
     p.add_argument("--profile-case", type=int, default=0, metavar="L",
                    help="profiling run: two PIVOT-Refine calls at sequence length L (H_I=64, d=128, k=2048, "
                         "c=4096, g=8) and exit; no timing, no JSON")
@@ -205,15 +210,211 @@ def cpu_oracle_sample(x, spec, runs=24):
     G = (spec.L + spec.g - 1) // spec.g
     per = max(1, cores)
     rows = 0
+    units_sampled = 0
     t0 = time.perf_counter()
     for j in range(runs):
         g0 = min(G - per, int((2 * j + 1) * G / (2 * runs)))
         orc.refine(x["q"], x["w"], x["k"], spec.k, spec.c, spec.g, g0=g0, g1=g0 + per)
         rows += per * spec.g
+        units_sampled += refine_units(spec, g0, g0 + per)
     dt = time.perf_counter() - t0
     desc = (f"oracle PIVOT-Refine (double precision, OpenMP over groups) on {runs} runs of {per} consecutive "
             f"groups ({rows} query rows) centred at {runs} evenly spaced positions of the L={spec.L} sequence")
-    return rows / dt, orc.threads(), desc, dt
+    return rows / dt, orc.threads(), desc, dt, units_sampled
+
+
+def refine_units(spec, g0, g1):
+    """Key-row products sum_i (P_i + |G_i| min(c, P_i)) of groups [g0, g1)."""
+    u = 0
+    for i in range(g0, g1):
+        P = min(i * spec.g + spec.g, spec.L)
+        u += P + (P - i * spec.g) * min(spec.c, P)
+    return u
+
+
+def prefill_work(spec, g=None):
+    """(scan FLOPs, refine FLOPs, Refine key-row products sum_i (P_i + |G_i| min(c, P_i))) of one
+    prefill sequence; FLOPs are 2*H*d per (query-or-proxy row, key) pair."""
+    L, H, d, c = spec.L, spec.H, spec.d, spec.c
+    g = spec.g if g is None else g
+    f_scan = f_ref = units = 0
+    for t0 in range(0, L, g):
+        P = min(t0 + g, L)
+        m = P - t0
+        f_scan += 2 * H * d * P
+        f_ref += 2 * m * min(c, P) * H * d
+        units += P + m * min(c, P)
+    return f_scan, f_ref, units
+
+
+def oracle_refine_timed(x, spec, groups):
+    """Wall time of the oracle's PIVOT-Refine over the given runs [(g0, g1)] of groups and the
+    key-row products they cover."""
+    from oracle import oracle as orc
+
+    L, g, c = spec.L, spec.g, spec.c
+    units = 0
+    t0 = time.perf_counter()
+    for g0, g1 in groups:
+        orc.refine(x["q"], x["w"], x["k"], spec.k, c, g, g0=g0, g1=g1)
+        for i in range(g0, g1):
+            P = min(i * g + g, L)
+            units += P + (P - i * g) * min(c, P)
+    return time.perf_counter() - t0, units
+
+
+def per_config_lines(to_dev_fn, dev, ws, flush, timed, tf_burst, hbm, cpu):
+    """Every workload of the build: GPU times of its paths with queries/s, us per group, roofline
+    fraction (scan [+ refine] FLOPs at the burst bf16 peak over the time) and x vs the dense
+    indexer on the same inputs; the CPU oracle timed whole on the tiny and 8K workloads, and on a
+    sample of groups, extrapolated to the whole sequence by key-row products, on the others."""
+    import numpy as np
+
+    import top_token_selection_proxy_b200 as P
+    from top_token_selection_proxy_b200 import inputs
+    from oracle import oracle as orc
+
+    out = []
+
+    def entry(spec, x, paths, cpu_mode):
+        q, w, k = to_dev_fn(x["q"], dev), to_dev_fn(x["w"], dev), to_dev_fn(x["k"], dev)
+        G = (spec.L + spec.g - 1) // spec.g
+        f_scan, f_ref, units = prefill_work(spec)
+        f_dense = 2 * spec.H * spec.d * spec.L * (spec.L + 1) // 2
+        ms = {}
+        if "dense" in paths:
+            ms["dense"] = timed(lambda: P.indexer_dense(q, w, k, spec.k, ws=ws), n=2)
+        if "reuse" in paths:
+            ms["reuse"] = timed(lambda: P.reuse(q, w, k, spec.k, spec.g, ws=ws))
+        if "refine" in paths:
+            ms["refine"] = timed(lambda: P.refine(q, w, k, spec.k, spec.c, spec.g, ws=ws))
+        flops = {"dense": f_dense, "reuse": f_scan, "refine": f_scan + f_ref}
+        e = {"workload": spec.name, "L": spec.L, "g": spec.g, "k": spec.k, "c": spec.c, "rho": spec.rho,
+             "dtype": "f32" if spec.dtype == inputs.F32 else "bf16"}
+        for name, t in ms.items():
+            e[name] = {"ms": t, "queries_per_s": spec.L / (t * 1e-3), "us_per_group": 1000.0 * t / G,
+                       "roofline_frac": (flops[name] / (tf_burst * 1e12)) / (t * 1e-3)}
+            if "dense" in ms and name != "dense":
+                e[name]["x_vs_dense"] = ms["dense"] / t
+        if cpu_mode == "whole" and cpu:
+            secs, u = oracle_refine_timed(x, spec, [(0, G)])
+            e["cpu_oracle_refine"] = {"seconds": secs, "queries_per_s": spec.L / secs, "cores": orc.threads(),
+                                      "kind": "oracle, timed whole"}
+        elif cpu_mode == "sample" and cpu:
+            runs = [(int(i), int(i) + 1) for i in inputs.sample_groups(G, spec.g, spec.k, spec.c, 16,
+                                                                       spec.seed + 2000)]
+            secs, u = oracle_refine_timed(x, spec, runs)
+            est = secs * units / u
+            e["cpu_oracle_refine"] = {"sample_seconds": secs, "sample_groups": len(runs),
+                                      "extrapolated_seconds": est, "queries_per_s": spec.L / est,
+                                      "cores": orc.threads(),
+                                      "kind": "oracle on 16 seeded groups, EXTRAPOLATED to the whole sequence "
+                                              "by key-row products sum_i (P_i + |G_i| min(c, P_i))"}
+        del q, w, k
+        return e
+
+    out.append(entry(inputs.TINY, inputs.make_prefill(inputs.TINY), ("dense", "reuse", "refine"), "whole"))
+    out.append(entry(inputs.PREFILL_8K, inputs.make_prefill(inputs.PREFILL_8K), ("dense", "reuse", "refine"),
+                     "whole"))
+    for rho in inputs.SWEEP_RHO:
+        x = inputs.make_prefill(inputs.sweep_32k(1, rho))  # one sequence per rho; the g axis sees the same inputs
+        dense_ms = None
+        for g in inputs.SWEEP_G:
+            spec = inputs.sweep_32k(g, rho)
+            e = entry(spec, x, ("dense", "reuse", "refine") if g == 1 else ("reuse", "refine"), "sample")
+            if g == 1:
+                dense_ms = e["dense"]["ms"]
+            else:
+                for name in ("reuse", "refine"):
+                    e[name]["x_vs_dense"] = dense_ms / e[name]["ms"]
+            out.append(e)
+        del x
+    ds = inputs.DECODE
+    xd = inputs.make_decode(ds)
+    dq, dw, dk = to_dev_fn(xd["q"], dev), to_dev_fn(xd["w"], dev), to_dev_fn(xd["k"], dev)
+    off = xd["offsets"]
+    key_bytes = int(off[-1]) * ds.d * 2
+    d_ms = {"refine": timed(lambda: P.refine_varlen(dq, dw, dk, off, ds.k, ds.c, ds.g, ws=ws)),
+            "reuse": timed(lambda: P.reuse_varlen(dq, dw, dk, off, ds.k, ds.g, ws=ws))}
+    rows = ds.B * ds.g
+    e = {"workload": ds.name, "B": ds.B, "g": ds.g, "k": ds.k, "c": ds.c, "key_bytes": key_bytes,
+         **{n: {"ms": t, "queries_per_s": rows / (t * 1e-3), "us_per_group": 1000.0 * t / ds.B,
+                "roofline_frac": (key_bytes / (hbm * 1e9)) / (t * 1e-3), "bound": "hbm"}
+            for n, t in d_ms.items()}}
+    if cpu:
+        t0 = time.perf_counter()
+        orc.decode(xd["q"], xd["w"], xd["k"], off, ds.k, ds.c, ds.g, 1)
+        secs = time.perf_counter() - t0
+        e["cpu_oracle_refine"] = {"seconds": secs, "queries_per_s": rows / secs, "cores": orc.threads(),
+                                  "kind": "oracle, timed whole (all 32 sequences)"}
+    out.append(e)
+    del dq, dw, dk
+    return out
+
+
+def run_split(args):
+    """One L=131072 sequence indexed by all ranks (PIVOT-Refine): each rank holds the rows of
+    its zig-zag chunks, the key chunks are all-gathered (NCCL; the one exchange), then every
+    rank runs the group-range call on its two chunks.  value = L / max-over-ranks step time."""
+    import numpy as np
+    import torch
+
+    import top_token_selection_proxy_b200 as P
+    from top_token_selection_proxy_b200 import build, inputs
+    from top_token_selection_proxy_b200 import multigpu as M
+
+    world, rank, local = M.env()
+    M.init("nccl", world)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if rank == 0:
+        build.build()
+    M.barrier(world)
+    P.lib()
+    spec = inputs.LONG_128K
+    x = inputs.make_prefill(spec)  # every rank draws the same sequence and keeps its chunks
+    chunks = M.zigzag_chunks(spec.L, spec.g, world, rank)
+    q_loc = to_dev(M.local_rows(x["q"], chunks), dev)
+    w_loc = to_dev(M.local_rows(x["w"], chunks), dev)
+    k_loc = to_dev(M.local_rows(x["k"], chunks), dev)
+    del x
+    ws = P.Workspace(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def index_fn(q_rows, w_rows, k_prefix, t0, t1):
+        return P.refine_range(q_rows, w_rows, k_prefix, spec.L, spec.k, spec.c, spec.g, t0 // spec.g,
+                              t1 // spec.g, ws=ws)[0]
+
+    def step():
+        return M.split_step(index_fn, q_loc, w_loc, k_loc, spec.L, spec.g, world, rank)
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    M.barrier(world)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    tot = 0.0
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+        torch.cuda.synchronize()
+        tot += ev[i][0].elapsed_time(ev[i][1])
+    M.barrier(world)
+    ms = M.max_over_ranks(tot, world, dev) / args.steps
+    status = M.max_over_ranks(float(P.last_device_status(ws)), world, dev)
+    if rank == 0:
+        print(json.dumps({"metric": METRIC, "value": spec.L / (ms / 1000.0), "unit": UNIT, "n_gpus": world,
+                          "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                          "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                          "config": {"workload": spec.name + "_refine_split", "L": spec.L, "H_I": spec.H,
+                                     "d": spec.d, "k": spec.k, "c": spec.c, "g": spec.g,
+                                     "parallelism": f"one sequence over {world} GPU(s): zig-zag group ranges, "
+                                                    "key all-gather",
+                                     "l2": "flushed before every step (256 MiB write)"},
+                          "gpu_launches": 3 * 2 * args.steps, "device_status": int(status)}), flush=True)
+    M.finish(world)
 
 
 def run_reference(args):
@@ -294,6 +495,9 @@ def main():
         return
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.split:
+        run_split(args)
         return
     import numpy as np
     import torch
@@ -412,6 +616,9 @@ def main():
         extras["workload_diagnostics"] = {"workload": inputs.PREFILL_8K.name,
                                           **diagnostics.summary(di.cpu().numpy(), kg, dfull.cpu().numpy())}
         del gq, gw, gk, di, dfull
+        if not args.no_configs:
+            hbm_, tfb_, _, _ = peaks()
+            extras["configs"] = per_config_lines(to_dev, dev, ws, flush, timed, tfb_, hbm_, not args.no_cpu)
 
     e2e = None
     M.barrier(world)  # every rank measures end to end (rank 0 arrives after its side measurements)
@@ -453,8 +660,12 @@ def main():
     G = (spec.L + spec.g - 1) // spec.g
     cpu = None
     if not args.no_cpu:
-        v, cores, desc, secs = cpu_oracle_sample(x, spec)
-        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc, "seconds": secs}
+        v, cores, desc, secs, u_s = cpu_oracle_sample(x, spec)
+        full = secs * refine_units(spec, 0, G) / u_s
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc, "seconds": secs,
+               "extrapolated_full_sequence_seconds": full,
+               "extrapolated_queries_per_s": spec.L / full,
+               "extrapolation": "EXTRAPOLATED from the sample by key-row products sum_i (P_i + |G_i| min(c, P_i))"}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",

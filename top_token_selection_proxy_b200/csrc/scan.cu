@@ -83,6 +83,12 @@ struct ScanTail {
   int est[4];               // group got a sampled threshold estimate in this attempt
   int retry;                // the attempt's estimate was too high: scan the item again
   uint32_t hist11[kHist11Words];    // radix-select histogram (11-bit digits)
+  // sample-tile histogram of each group's scores: 2048 bins of bits 30..20 of the order key
+  // (exponent and 3 mantissa bits of a positive score; every other key in bin 0), two
+  // 16-bit counts per word
+  uint32_t esth[4][1024];
+  uint32_t escan[4][4];     // per group, per warp partial sums of the bin search
+  int ebin[4];              // per group, the bin where the running count reaches r0
   uint64_t bot[16];
   SelSmem sel;
   // w-bar of the item's groups, permuted for the epilogue: row (b, m) holds heads
@@ -97,6 +103,7 @@ constexpr size_t scan_smem() {
   using C = ScanCfg<H, D>;
   return 1024 + C::B_BYTES + C::STAGES * C::A_BYTES + sizeof(ScanTail);
 }
+static_assert(scan_smem<64, 128>() <= 232448, "227 KB of dynamic shared memory per CTA");
 
 template <int H, int D>
 __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CUtensorMap kmap, const ScanArgs a) {
@@ -231,6 +238,7 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
         uint8_t* dst = sB + kb * (C::N * 128) + n * 128 + ((ch ^ (n & 7)) << 4);
         *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
+      for (int u = tid; u < 4 * 1024; u += C::THREADS) (&T.esth[0][0])[u] = 0u;
       for (int u = tid; u < C::NB * H; u += C::THREADS) {
         const int b = u / H, hj = u % H;
         int nm = T.nmem[b];
@@ -329,6 +337,8 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
       uint32_t qcnt = 0;
       uint64_t tau_r = 0;
       const int64_t e_r = T.e[grp_w];  // causal bound of this warp's group
+      // the estimate comes from the sample histogram when its 16-bit counts cannot overflow
+      const bool hist_est = ns > 0 && (int64_t)ns * C::BM < 65536;
       const int64_t s_begin = T.s_begin, s_end = T.s_end;
       auto seg_of = [&](int b, int q) { return selbase + (uint64_t)b * gstride + (uint64_t)q * scap; };
       auto publish_counts = [&]() {
@@ -393,7 +403,12 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
         if (ok && grp_w < nb_act) {
           const int64_t s = s_begin + (int64_t)tile_of(j, ns) * C::BM + q4 * 32 + my_lane;
           const bool valid = (s < s_end) && (s <= e_r);
-          const uint64_t p = pack_entry(score_key(sc), (uint32_t)s);
+          const uint32_t key = score_key(sc);
+          const uint64_t p = pack_entry(key, (uint32_t)s);
+          if (hist_est && j < ns && valid) {  // sample tile: count the score for the estimate
+            const uint32_t bin = key >= 0x80000000u ? (key >> 20) - 0x800u : 0u;
+            atomicAdd(&T.esth[grp_w][bin >> 1], (bin & 1u) ? 0x10000u : 1u);
+          }
           const bool pass = valid && p > tau_r;
           const uint32_t m = __ballot_sync(0xFFFFFFFFu, pass);
           if (pass) seg_of(grp_w, q4)[qcnt + __popc(m & lanemask_lt())] = p;
@@ -412,15 +427,59 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
           if (named_bar_or(1, C::NEPI, T.abort_flag != 0)) break;                   // uniform decision
           const uint32_t flags = T.cflags;
           publish_counts();
+          // keep the sample's best r0 (the sample's expected share of 1.5 * need, plus a
+          // margin); the threshold admits about 1.5 * need of the remaining keys
+          uint32_t r0 = (uint32_t)((3 * (int64_t)need * ns) / (2 * (int64_t)ntiles)) + 64u;
+          if (a.debug_flags & 4) r0 = 1;  // test hook: an estimate that is always too high
+          if (est_now && hist_est) {
+            // from the sample histogram: each group's 4 warps find the bin (from the top) where
+            // the count reaches r0; its lower edge is the estimate, below the r0-th best of the
+            // sample (so at least r0 sample entries stay), and each warp compacts its own
+            // sub-buffer against it -- no pass over the sub-buffers
+            const int gt = q4 * 32 + lane;  // thread within the group
+            uint32_t loc[16], sum = 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {  // bins 2047 - 16 gt - 2u - {0, 1}, descending
+              const uint32_t wv = T.esth[grp_w][1023 - 8 * gt - u];
+              loc[2 * u] = wv >> 16;
+              loc[2 * u + 1] = wv & 0xFFFFu;
+              sum += loc[2 * u] + loc[2 * u + 1];
+            }
+            uint32_t incl = warp_incl_scan(sum);
+            if (lane == 31) T.escan[grp_w][q4] = incl;
+            if (EG.tid < 4) T.ebin[EG.tid] = 0;
+            EG.sync();
+            for (int w = 0; w < q4; ++w) incl += T.escan[grp_w][w];
+            const uint32_t excl = incl - sum;
+            if (excl < r0 && r0 <= incl) {
+              uint32_t c = excl;
+#pragma unroll
+              for (int u = 0; u < 16; ++u) {
+                if (c + loc[u] >= r0) {
+                  T.ebin[grp_w] = 2047 - 16 * gt - u;
+                  break;
+                }
+                c += loc[u];
+              }
+            }
+            EG.sync();
+            const int eb = T.ebin[grp_w];  // 0 when the sample holds fewer than r0 scores above bin 0
+            const uint64_t th = eb > 0 ? (uint64_t)(((uint32_t)eb + 0x800u) << 20) << 32 : 0ull;
+            if (grp_w < nb_act && th > 0) {
+              qcnt = warp_compact_ge(seg_of(grp_w, q4), qcnt, th);
+              if (th - 1ull > tau_r) tau_r = th - 1ull;  // admit x >= th from now on
+            }
+            if (EG.tid < 4) T.est[EG.tid] = (EG.tid < nb_act && T.ebin[EG.tid] > 0) ? 1 : 0;
+            publish_counts();
+          }
           for (int b = 0; b < nb_act; ++b) {
-            if (est_now) {
-              // keep the sample's best r0 (the sample's expected share of 1.5 * need, plus
-              // a margin); the threshold admits about 1.5 * need of the remaining keys
-              uint32_t r0 = (uint32_t)((3 * (int64_t)need * ns) / (2 * (int64_t)ntiles)) + 64u;
-              if (a.debug_flags & 4) r0 = 1;  // test hook: an estimate that is always too high
+            const uint32_t tot = T.qcnt[b][0] + T.qcnt[b][1] + T.qcnt[b][2] + T.qcnt[b][3];
+            const bool over = T.qcnt[b][0] > scap - 256u || T.qcnt[b][1] > scap - 256u ||
+                              T.qcnt[b][2] > scap - 256u || T.qcnt[b][3] > scap - 256u;
+            if (est_now && !hist_est) {
               const uint64_t th = cut_back(b, r0, r0 + r0 / 4u);
               if (EG.tid == 0) T.est[b] = th > 0 ? 1 : 0;
-            } else if (flags & (1u << b)) {
+            } else if ((flags & (1u << b)) || (est_now && over && tot > need)) {
               // keep at most sub_cap - 128 in total (>= need + 128 since sub_cap >= need + 256):
               // then every sub-buffer has room for the 4 tiles until the next consensus
               cut_back(b, need, scap - 256u);
