@@ -629,7 +629,7 @@ def main():
         oh = torch.empty((spec.L, spec.k), dtype=torch.int32).pin_memory()
 
         def e2e_step():  # the public host-memory call: copies in, kernels and copies out overlap by chunks
-            P.refine_streamed(qh.view(torch.bfloat16), wh, kh.view(torch.bfloat16), spec.k, spec.c, spec.g,
+            P.refine_host(qh.view(torch.bfloat16), wh, kh.view(torch.bfloat16), spec.k, spec.c, spec.g,
                               out_host=oh, chunks=E2E_CHUNKS, ws=ws, device=dev)
 
         e2e_step()
@@ -645,7 +645,7 @@ def main():
         e2e = {"value": world * spec.L / (e_ms / 1000.0), "unit": UNIT, "ms_per_step": e_ms,
                "h2d_bytes_per_step": int(qh.numel() * 2 + wh.numel() * 4 + kh.numel() * 2),
                "d2h_bytes_per_step": int(oh.numel() * 4), "host_buffers": "pinned",
-               "api": f"refine_streamed, {E2E_CHUNKS} chunks of whole groups"}
+               "api": f"C ABI pivot_refine_host, {E2E_CHUNKS} runs of whole groups, copies overlapped with the kernels"}
 
     if rank != 0:
         M.finish(world)

@@ -150,6 +150,31 @@ PIVOT_API pivot_status pivot_refine_agg(const void *q_I, const float *w_I, const
                                         float *cand_scores_opt, void *ws, size_t ws_bytes,
                                         pivot_stream_t stream);
 
+/* PIVOT-Refine of one prefill sequence held in HOST memory (same computation as
+ * pivot_refine, Eq. (2), (4), (5), (7)-(9); the groups are independent given
+ * k_I, so the sequence is indexed in runs of whole groups).  q_host [L,H,d] bf16,
+ * w_host [L,H] fp32, k_host [L,d] bf16 and out_host [L,k] int32 are host
+ * pointers; they should be pinned (cudaHostAlloc / cudaHostRegister), otherwise
+ * the copies do not overlap.  The keys and weights are copied first, then the
+ * queries in `chunks` (1..64) runs of whole groups on a copy stream; run i is
+ * indexed on `stream` (pivot_refine_range) once its rows have landed, while
+ * run i+1 is copied in and run i-1's rows are copied back on a second copy
+ * stream.  ws is a DEVICE buffer of pivot_refine_host_workspace_size bytes
+ * (256-byte aligned) that holds the device copies and the refine workspace.
+ * Asynchronous: when the call returns the work is queued and `stream` is ordered
+ * after the last copy back, so synchronise `stream` before reading out_host or
+ * reusing the host buffers.  The first call on a device creates two copy
+ * streams and 130 events that live until the process exits; make that call
+ * before any stream capture.  Calls on one device enqueue one at a time (a
+ * mutex) and share the copy streams; give concurrent calls their own ws.
+ * Errors: PIVOT_ERR_INVALID_ARG (null pointer, chunks outside 1..64, c < k,
+ * misaligned ws), PIVOT_ERR_UNSUPPORTED_SHAPE, PIVOT_ERR_WORKSPACE_TOO_SMALL,
+ * PIVOT_ERR_CUDA (pivot_last_cuda_error says which call). */
+PIVOT_API size_t pivot_refine_host_workspace_size(int64_t L, int H, int d, int k, int c, int g);
+PIVOT_API pivot_status pivot_refine_host(const void *q_host, const float *w_host, const void *k_host, int64_t L,
+                                         int H, int d, int k, int c, int g, int chunks, int32_t *out_host, void *ws,
+                                         size_t ws_bytes, pivot_stream_t stream);
+
 /* Guardrail (PIVOT paper, "Efficiency Results (Figure 4)": PIVOT falls back to
  * dense DSA at short context to avoid overhead).  The pages give no criterion;
  * this library uses the work model of the prefill call, in key-row products

@@ -133,3 +133,24 @@ def test_decode_workspace_grows_with_the_cached_keys(lib):
         assert 0 < a and b - a >= 12 * 100000 - 8 * 256  # buffers start on 256-byte boundaries
     assert P.varlen_workspace_size(P.OP_REUSE, np.array([0, 3], dtype=np.int64), 64, 128, 8, 8, 4) == 0  # P_b < g
     assert P.varlen_workspace_size(P.OP_REUSE, np.array([5, 20], dtype=np.int64), 64, 128, 8, 8, 4) == 0  # off[0] != 0
+
+
+def test_host_entry_point_checks_arguments_before_any_cuda_call(lib):
+    """pivot_refine_host: argument and workspace checks happen on the host, before a stream,
+    event or copy is touched (so they also hold on a machine without a GPU)."""
+    buf = ctypes.create_string_buffer(4096 + 256)
+    ws = ctypes.c_void_p((ctypes.addressof(buf) + 255) // 256 * 256)
+    h = ctypes.cast(ctypes.create_string_buffer(64), ctypes.c_void_p)
+    L, H, d, k, c, g = 1024, 64, 128, 16, 32, 8
+    need = lib.pivot_refine_host_workspace_size(L, H, d, k, c, g)
+    # the device copies of q, w, k and the output rows, then the refine workspace
+    assert need >= L * H * d * 2 + L * H * 4 + L * d * 2 + L * k * 4 + \
+        lib.pivot_workspace_size(2, L, H, d, k, c, g, 0)
+    assert lib.pivot_refine_host_workspace_size(L, H, d, k, 8, g) == 0  # c < k
+    args = (h, h, h, L, H, d, k, c, g)
+    assert lib.pivot_refine_host(None, h, h, L, H, d, k, c, g, 8, h, ws, 4096, None) == 1
+    assert lib.pivot_refine_host(*args, 0, h, ws, 4096, None) == 1      # chunks outside 1..64
+    assert lib.pivot_refine_host(*args, 65, h, ws, 4096, None) == 1
+    mis = ctypes.c_void_p(ws.value + 16)
+    assert lib.pivot_refine_host(*args, 8, h, mis, 4096, None) == 1     # ws not 256-byte aligned
+    assert lib.pivot_refine_host(*args, 8, h, ws, 4096, None) == 3      # workspace too small

@@ -474,7 +474,7 @@ def test_group_ranges_reproduce_the_whole_sequence(orc):
 
 
 def test_streamed_refine_from_host_memory_matches_one_call(orc):
-    """refine_streamed (pinned host inputs, copies overlapped with group-range calls in
+    """refine_host (pivot_refine_host: pinned host inputs, copies overlapped with group-range calls in
     chunks) writes exactly the rows of one device-resident refine call, for a ragged
     length and chunk counts that do and do not divide the groups; twice in a row
     (buffer reuse, earlier output overwritten).  Its rows also pass the oracle's
@@ -492,7 +492,7 @@ def test_streamed_refine_from_host_memory_matches_one_call(orc):
     G = (6001 + g - 1) // g
     for chunks in (1, 3, 8, 8):
         oh.fill_(-7)
-        P.refine_streamed(qh, wh, kh, topk, c, g, out_host=oh, chunks=chunks)
+        P.refine_host(qh, wh, kh, topk, c, g, out_host=oh, chunks=chunks)
         torch.cuda.current_stream().synchronize()
         assert np.array_equal(np.sort(oh.numpy(), axis=1), want), f"chunks = {chunks}"
     fails = check_refine(orc, x, oh.numpy().copy(), None, cand, cand_sc, range(G), topk, c, g)

@@ -43,7 +43,7 @@ EXPORTS = (
     "pivot_set_device_timeout_ns", "pivot_set_debug_flags", "pivot_set_profile_events", "pivot_version",
     "pivot_reuse_noalloc", "pivot_guardrail_dense", "pivot_reuse_guarded", "pivot_refine_guarded",
     "pivot_reuse_agg", "pivot_refine_agg", "pivot_indexer_dense_range", "pivot_reuse_range",
-    "pivot_refine_range",
+    "pivot_refine_range", "pivot_refine_host_workspace_size", "pivot_refine_host",
 )
 
 # proxy aggregation (PIVOT paper, Ablation Studies, Proxy aggregation, Table 2)
@@ -82,6 +82,10 @@ def lib() -> ctypes.CDLL:
         L.pivot_refine_range.argtypes = [P, P, P, I64, I, I, I, I, I, I, I64, I64, P, P, P, P, P, SZ, P]
         L.pivot_reuse_agg.argtypes = [P, P, P, I64, I, I, I, I, I, I, P, P, P, SZ, P]
         L.pivot_refine_agg.argtypes = [P, P, P, I64, I, I, I, I, I, I, I, P, P, P, P, P, SZ, P]
+        L.pivot_refine_host_workspace_size.argtypes = [I64, I, I, I, I, I]
+        L.pivot_refine_host_workspace_size.restype = SZ
+        L.pivot_refine_host.argtypes = [P, P, P, I64, I, I, I, I, I, I, P, P, SZ, P]
+        L.pivot_refine_host.restype = I
         L.pivot_guardrail_dense.argtypes = [I, I64, I, I]
         L.pivot_guardrail_dense.restype = I
         L.pivot_reuse_guarded.argtypes = [P, P, P, I64, I, I, I, I, I, P, P, P, SZ, P, P]
@@ -303,48 +307,16 @@ def group_chunks(L: int, g: int, chunks: int):
     return [(i * g, min(L, (i + per) * g)) for i in range(0, G, per)]
 
 
-class _HostPipeline:
-    """Device copies and the two copy streams that refine_streamed reuses for one shape."""
+def refine_host(q_host, w_host, k_host, topk: int, c: int, g: int, *, out_host, chunks: int = 8,
+                ws: Optional[Workspace] = None, device=None, stream=None):
+    """PIVOT-Refine of one prefill sequence held in pinned host memory (pivot_refine_host).
 
-    def __init__(self, dev, L, H, d, topk):
-        self.shape = (L, H, d, topk)
-        self.q = torch.empty((L, H, d), dtype=torch.bfloat16, device=dev)
-        self.w = torch.empty((L, H), dtype=torch.float32, device=dev)
-        self.k = torch.empty((L, d), dtype=torch.bfloat16, device=dev)
-        self.out = torch.empty((L, topk), dtype=torch.int32, device=dev)
-        self.s_in = torch.cuda.Stream(dev)
-        self.s_out = torch.cuda.Stream(dev)
-
-
-_pipelines = {}  # device index -> the _HostPipeline of the last shape used there
-
-
-def _drop_pipeline(index) -> None:
-    pl = _pipelines.pop(index, None)
-    if pl is not None:  # its copies may still be in flight: let them finish before the buffers go
-        pl.s_in.synchronize()
-        pl.s_out.synchronize()
-
-
-def release_streamed_buffers() -> None:
-    """Free the device buffers refine_streamed keeps between calls (waits for its copies)."""
-    for index in list(_pipelines):
-        _drop_pipeline(index)
-
-
-def refine_streamed(q_host, w_host, k_host, topk: int, c: int, g: int, *, out_host, chunks: int = 8,
-                    ws: Optional[Workspace] = None, device=None):
-    """PIVOT-Refine of one prefill sequence held in pinned host memory.
-
-    q_host [L, H, d] bf16, w_host [L, H] fp32, k_host [L, d] bf16 and out_host [L, topk]
-    int32 are pinned CPU tensors.  Keys and weights are copied first, then the queries
-    in `chunks` runs of whole groups.  Run i is indexed with the group-range call on the
-    current stream while run i+1 is copied in (a second stream) and run i-1's rows are
-    copied out (a third), so the transfers overlap the kernels.  The rows equal those of
-    one `refine` call.  Device copies of the inputs are kept for the next call of the same
-    shape (one shape per device; release_streamed_buffers frees them).  Asynchronous: the
-    current stream is ordered after the last copy out, so synchronise it before reading
-    out_host."""
+    q_host [L, H, d] bf16, w_host [L, H] fp32, k_host [L, d] bf16 and out_host [L, topk] int32
+    are pinned CPU tensors.  The library copies the keys and weights, then the queries in
+    `chunks` runs of whole groups, indexes each run with the group-range call as soon as it
+    has landed and copies its rows back while later runs are still in flight.  The rows equal
+    those of one `refine` call.  Asynchronous: the stream is ordered after the last copy back,
+    so synchronise it before reading out_host."""
     for t, dt_ in ((q_host, torch.bfloat16), (w_host, torch.float32), (k_host, torch.bfloat16),
                    (out_host, torch.int32)):
         if t.is_cuda or not t.is_pinned() or not t.is_contiguous() or t.dtype != dt_:
@@ -355,41 +327,20 @@ def refine_streamed(q_host, w_host, k_host, topk: int, c: int, g: int, *, out_ho
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     if dev.type != "cuda" or dev.index is None:
         raise ValueError("device must name one CUDA device, e.g. 'cuda:0'")
-    # the C calls take SMs, tensor maps and the launch from the calling thread's current
-    # device: make `dev` current for the whole call
-    with torch.cuda.device(dev):
-        return _refine_streamed_on(dev, q_host, w_host, k_host, topk, c, g, out_host, chunks, ws)
-
-
-def _refine_streamed_on(dev, q_host, w_host, k_host, topk, c, g, out_host, chunks, ws):
-    L, H, d = q_host.shape
-    pl = _pipelines.get(dev.index)
-    if pl is None or pl.shape != (L, H, d, topk):
-        _drop_pipeline(dev.index)
-        pl = _pipelines[dev.index] = _HostPipeline(dev, L, H, d, topk)
-    W = _ws_for(ws, dev).get(workspace_size(OP_REFINE, L, H, d, topk, c, g, BF16))
-    cur = torch.cuda.current_stream(dev)
-    pl.s_in.wait_stream(cur)   # earlier work on the pipeline's buffers is done
-    pl.s_out.wait_stream(cur)
-    with torch.cuda.stream(pl.s_in):
-        pl.k.copy_(k_host, non_blocking=True)
-        pl.w.copy_(w_host, non_blocking=True)
-    for t0, t1 in group_chunks(L, g, chunks):
-        with torch.cuda.stream(pl.s_in):
-            pl.q[t0:t1].copy_(q_host[t0:t1], non_blocking=True)
-            landed = torch.cuda.Event()
-            landed.record(pl.s_in)
-        cur.wait_event(landed)
-        _check(lib().pivot_refine_range(_ptr(pl.q[t0:t1]), _ptr(pl.w[t0:t1]), _ptr(pl.k), L, H, d, BF16, topk, c, g,
-                                        t0 // g, (t1 + g - 1) // g, _ptr(pl.out[t0:t1]), None, None, None, _ptr(W),
-                                        W.numel(), ctypes.c_void_p(cur.cuda_stream)), "pivot_refine_range")
-        done = torch.cuda.Event()
-        done.record(cur)
-        pl.s_out.wait_event(done)
-        with torch.cuda.stream(pl.s_out):
-            out_host[t0:t1].copy_(pl.out[t0:t1], non_blocking=True)
-    cur.wait_stream(pl.s_out)
+    with torch.cuda.device(dev):  # the C call works on the calling thread's current device
+        nbytes = int(lib().pivot_refine_host_workspace_size(L, H, d, topk, c, g))
+        if nbytes == 0:
+            raise PivotError(2, "pivot_refine_host_workspace_size")
+        W = _ws_for(ws, dev).get(nbytes)
+        s = torch.cuda.current_stream(dev) if stream is None else stream
+        _check(lib().pivot_refine_host(_ptr(q_host), _ptr(w_host), _ptr(k_host), L, H, d, topk, c, g, chunks,
+                                       _ptr(out_host), _ptr(W), W.numel(), ctypes.c_void_p(s.cuda_stream)),
+               "pivot_refine_host")
     return out_host
+
+
+# the earlier name of refine_host
+refine_streamed = refine_host
 
 
 def guardrail_dense(op: int, L: int, c: int, g: int) -> bool:
@@ -515,7 +466,7 @@ __all__ = [
     "indexer_dense", "reuse", "refine", "reuse_varlen", "refine_varlen", "last_device_status",
     "guardrail_dense", "reuse_guarded", "refine_guarded", "AGGREGATION",
     "indexer_dense_range", "reuse_range", "refine_range",
-    "group_chunks", "refine_streamed", "release_streamed_buffers",
+    "group_chunks", "refine_host", "refine_streamed",
     "set_device_timeout_ns", "set_debug_flags", "KernelTimer", "OP_DENSE", "OP_REUSE", "OP_REFINE", "BF16", "F32",
     "STATUS",
 ]

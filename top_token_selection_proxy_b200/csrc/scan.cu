@@ -189,7 +189,10 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
     const int ntiles = T.ntiles;
 
     // ---------------------------------------------------------------- Eq. (4): pool proxies into B
+    // the members' q rows are read once: evict-first in L2, so they do not push the groups'
+    // selection sub-buffers out to DRAM
     {
+      const uint64_t qpol = l2_policy_evict_first();
       constexpr int XC = D / 8;  // 16-byte chunks per row
       for (int u = tid; u < C::NB * H * XC; u += C::THREADS) {
         const int xc = u % XC;
@@ -209,8 +212,9 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
           uint4 vv[8];
 #pragma unroll
           for (int u = 0; u < 8; ++u)
-            vv[u] = (m0 + u < nm) ? __ldg(reinterpret_cast<const uint4*>(a.q + ((r0 + m0 + u) * H + hj) * (int64_t)D) + xc)
-                                  : make_uint4(0u, 0u, 0u, 0u);
+            vv[u] = (m0 + u < nm)
+                        ? ldg_hint(reinterpret_cast<const uint4*>(a.q + ((r0 + m0 + u) * H + hj) * (int64_t)D) + xc, qpol)
+                        : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
           for (int u = 0; u < 8; ++u) {
             if (m0 + u < nm) {
@@ -539,15 +543,17 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
             group_minmax64<C::NEPI>(lo, hi, T.sel, EG);
             th = radix11_threshold<C::NEPI>(buf, n, need, need, T.hist11, T.sel, EG, lo, hi);
           }
-          const uint32_t m = compact_ge<C::NEPI>(buf, buf, n, th, T.sel, EG);
           const int64_t grp = T.grp0 + b;
+          // dense rows and candidate sets are written straight from the entries >= th (exactly
+          // `need` of them, or all when fewer); Reuse emission works on the compacted set
           if (a.mode == EMIT_DENSE) {
-            emit_row<C::NEPI>(buf, m, 0xFFFFFFFFu, 0ull, a.out_idx + grp * a.topk,
+            emit_row<C::NEPI>(buf, n, 0xFFFFFFFFu, th - 1ull, a.out_idx + grp * a.topk,
                           a.out_scores ? a.out_scores + grp * a.topk : nullptr, (uint32_t)a.topk, T.sel, EG);
           } else if (a.mode == EMIT_CAND) {
-            emit_row<C::NEPI>(buf, m, 0xFFFFFFFFu, 0ull, a.cand + grp * a.n_sel,
+            emit_row<C::NEPI>(buf, n, 0xFFFFFFFFu, th - 1ull, a.cand + grp * a.n_sel,
                           a.cand_scores ? a.cand_scores + grp * a.n_sel : nullptr, need, T.sel, EG);
           } else {  // EMIT_REUSE
+            const uint32_t m = compact_ge<C::NEPI>(buf, buf, n, th, T.sel, EG);
             emit_reuse<C::NEPI>(buf, m, a.topk, T.mrow0[b], T.nmem[b], T.mrow0[b], a.out_idx, a.out_scores, T.sel,
                             T.bot, EG);
           }
