@@ -90,6 +90,7 @@ struct ScanTail {
   uint32_t escan[4][4];     // per group, per warp partial sums of the bin search
   int ebin[4];              // per group, the bin where the running count reaches r0
   uint64_t bot[16];
+  uint32_t ecount;          // final selection: entries written so far
   SelSmem sel;
   // w-bar of the item's groups, permuted for the epilogue: row (b, m) holds heads
   // 8j + 2m, 8j + 2m + 1 (j = 0..7) of group b in 16 floats, rows 20 floats apart
@@ -496,6 +497,9 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
       // ---------------------------------------------------------------- final exact selection + emit
       if (EG.tid == 0) T.retry = 0;
       if (!named_bar_or(1, C::NEPI, T.abort_flag != 0)) {
+        // each group's entries are >= tau + 1: tau is the group's admission threshold (entries
+        // kept by a cut-back are >= the new tau + 1, later ones are above it)
+        if (lane == 0 && q4 == 0) T.tau[grp_w] = tau_r;
         publish_counts();
         // every entry left lies above the group's estimate (if it has one): with fewer
         // than `need` of them the estimate was too high and the top-need is not complete
@@ -514,11 +518,13 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
             publish_counts();
             n = T.qcnt[b][0] + T.qcnt[b][1] + T.qcnt[b][2] + T.qcnt[b][3];
           }
-          // gather the four sub-buffers into shared memory (each segment starts 16-byte aligned)
+          // gather the four sub-buffers into shared memory (each segment starts 16-byte aligned),
+          // keeping the largest entry for the selection's range
           uint32_t off = 0;
+          uint64_t hi = 0ull;
           for (int q = 0; q < 4; ++q) {
             const uint32_t nq = T.qcnt[b][q];
-            group_copy<C::NEPI>(sbuf + off, seg_of(b, q), nq, EG);
+            hi = group_copy_max<C::NEPI>(sbuf + off, seg_of(b, q), nq, hi, EG);
             off += (nq + 1u) & ~1u;
             if (nq & 1u) {  // pad to keep the next segment aligned: a zero entry sorts below everything
               if (EG.tid == 0) sbuf[off - 1] = 0ull;
@@ -532,26 +538,20 @@ __global__ void __launch_bounds__(576, 1) scan_kernel(const __grid_constant__ CU
           // largest is a real entry (n_real > need), found within the entries' range
           uint64_t th = 1ull;
           if (n_real > need) {
-            uint64_t lo = ~0ull, hi = 0ull;
-            for (uint32_t i = EG.tid; i < n; i += C::NEPI) {
-              const uint64_t e = buf[i];
-              if (e != 0ull) {
-                lo = e < lo ? e : lo;
-                hi = e > hi ? e : hi;
-              }
-            }
-            group_minmax64<C::NEPI>(lo, hi, T.sel, EG);
+            uint64_t lo = T.tau[b] + 1ull;
+            group_minmax64<C::NEPI>(lo, hi, T.sel, EG);  // (lo is the same in every thread)
             th = radix11_threshold<C::NEPI>(buf, n, need, need, T.hist11, T.sel, EG, lo, hi);
           }
           const int64_t grp = T.grp0 + b;
           // dense rows and candidate sets are written straight from the entries >= th (exactly
           // `need` of them, or all when fewer); Reuse emission works on the compacted set
           if (a.mode == EMIT_DENSE) {
-            emit_row<C::NEPI>(buf, n, 0xFFFFFFFFu, th - 1ull, a.out_idx + grp * a.topk,
-                          a.out_scores ? a.out_scores + grp * a.topk : nullptr, (uint32_t)a.topk, T.sel, EG);
+            emit_ge_warps<C::NEPI>(buf, n, th, a.out_idx + grp * a.topk,
+                                   a.out_scores ? a.out_scores + grp * a.topk : nullptr, (uint32_t)a.topk, &T.ecount,
+                                   EG);
           } else if (a.mode == EMIT_CAND) {
-            emit_row<C::NEPI>(buf, n, 0xFFFFFFFFu, th - 1ull, a.cand + grp * a.n_sel,
-                          a.cand_scores ? a.cand_scores + grp * a.n_sel : nullptr, need, T.sel, EG);
+            emit_ge_warps<C::NEPI>(buf, n, th, a.cand + grp * a.n_sel,
+                                   a.cand_scores ? a.cand_scores + grp * a.n_sel : nullptr, need, &T.ecount, EG);
           } else {  // EMIT_REUSE
             const uint32_t m = compact_ge<C::NEPI>(buf, buf, n, th, T.sel, EG);
             emit_reuse<C::NEPI>(buf, m, a.topk, T.mrow0[b], T.nmem[b], T.mrow0[b], a.out_idx, a.out_scores, T.sel,

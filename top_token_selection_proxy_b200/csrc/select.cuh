@@ -259,6 +259,33 @@ __device__ __forceinline__ void group_copy(uint64_t* dst, const uint64_t* src, u
   }
 }
 
+// group_copy that also returns max(hi, the largest entry copied) to every thread's own
+// view (each thread sees the maximum of what it copied; reduce across the group after).
+template <int NT>
+__device__ __forceinline__ uint64_t group_copy_max(uint64_t* dst, const uint64_t* src, uint32_t n, uint64_t hi,
+                                                   const Group<NT>& G) {
+  constexpr int U = 4;
+  for (uint32_t base = 0; base < n; base += NT * 2 * U) {
+    ulonglong2 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t i = base + (u * NT + G.tid) * 2;
+      v[u].x = v[u].y = 0ull;
+      if (i + 1 < n) v[u] = *reinterpret_cast<const ulonglong2*>(src + i);
+      else if (i < n) v[u].x = src[i];
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t i = base + (u * NT + G.tid) * 2;
+      if (i + 1 < n) *reinterpret_cast<ulonglong2*>(dst + i) = v[u];
+      else if (i < n) dst[i] = v[u].x;
+      hi = v[u].x > hi ? v[u].x : hi;
+      hi = v[u].y > hi ? v[u].y : hi;
+    }
+  }
+  return hi;
+}
+
 // Inclusive warp scan of v.
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v) {
   const int l = lane_id();
@@ -452,6 +479,43 @@ __device__ uint32_t emit_row(const uint64_t* buf, uint32_t n, uint32_t t_max, ui
     if (row_scores) row_scores[i] = -__int_as_float(0x7f800000);
   }
   return m;
+}
+
+// Write the indices (and optionally scores) of the entries of buf[0..n) that are >= th
+// (th >= 1, so zero pads never qualify) to row[0..) in arbitrary order and pad the rest
+// of row[0..width) with -1.  Each warp appends its qualifying entries with one shared
+// atomic per 32 entries (no group-wide prefix passes); *count is shared scratch.
+template <int NT>
+__device__ uint32_t emit_ge_warps(const uint64_t* buf, uint32_t n, uint64_t th, int32_t* row, float* row_scores,
+                                  uint32_t width, uint32_t* count, const Group<NT>& G) {
+  if (G.tid == 0) *count = 0u;
+  G.sync();
+  const uint32_t lane = G.tid & 31, lt = lanemask_lt();
+  for (uint32_t i0 = G.tid & ~31u; i0 < n; i0 += NT) {
+    const uint32_t i = i0 + lane;
+    const uint64_t x = i < n ? buf[i] : 0ull;
+    const bool take = x >= th;
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, take);
+    if (m == 0u) continue;
+    const int leader = __ffs(m) - 1;
+    uint32_t base = 0;
+    if ((int)lane == leader) base = atomicAdd(count, (uint32_t)__popc(m));
+    base = __shfl_sync(0xFFFFFFFFu, base, leader);
+    if (take) {
+      const uint32_t pos = base + __popc(m & lt);
+      if (pos < width) {
+        row[pos] = (int32_t)entry_idx(x);
+        if (row_scores) row_scores[pos] = entry_score(x);
+      }
+    }
+  }
+  G.sync();
+  const uint32_t got = *count < width ? *count : width;
+  for (uint32_t p = got + G.tid; p < width; p += NT) {
+    row[p] = -1;
+    if (row_scores) row_scores[p] = -__int_as_float(0x7f800000);
+  }
+  return got;
 }
 
 // Eq. (6) emit for one group after its exact top-(k+g-1) sits in buf[0..m):
