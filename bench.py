@@ -40,10 +40,10 @@ E2E_CHUNKS = 8  # runs of groups the end-to-end call pipelines its copies over
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum); valid only while
 # the sources the scan kernel is built from hash to `sources_sha256`.
 SCAN_TRAFFIC = {
-    "bytes": 2764699392 + 1645043200,
+    "bytes": 2490000000 + 939570000,  # 2.49 GB + 939.57 MB, as ncu printed them
     "sources": ("scan.cu", "select.cuh", "ptx.cuh", "kernels.cuh", "headsum.cuh"),
-    "sources_sha256": "e958954c05d754c3c30a335dba5fca923bc87f6193ecc7998d18a5747895ab10",
-    "profile": "profiles/dram_traffic_prefill_L131072_g8_refine.md",
+    "sources_sha256": "b9a771ddbd4a63fd3e34c0656affa93674bd6a8de341415357dbbc1033e210a7",
+    "profile": "profiles/kernels_prefill_L131072_g8_refine_1pass.md",
 }
 
 
