@@ -588,9 +588,23 @@ def main():
         off = xd["offsets"]
         dref = timed(lambda: P.refine_varlen(dq, dw, dk, off, ds.k, ds.c, ds.g, ws=ws))
         dreu = timed(lambda: P.reuse_varlen(dq, dw, dk, off, ds.k, ds.g, ws=ws))
+
+        def decode_phases(f, n=3):
+            """Median (proxies + scan, selection + emit, re-scoring + row select) of n calls."""
+            ph = []
+            for _ in range(n):
+                flush.fill_(1)
+                with timer:
+                    f()
+                torch.cuda.synchronize()
+                ph.append(timer.ms())
+            return {name: statistics.median(x[i] for x in ph)
+                    for i, name in enumerate(("scan", "select_emit", "refine_rowselect"))}
+
+        dph = decode_phases(lambda: P.refine_varlen(dq, dw, dk, off, ds.k, ds.c, ds.g, ws=ws))
         key_bytes = int(off[-1]) * ds.d * 2
         hbm, _, _, _ = peaks()
-        extras["decode"] = {"workload": ds.name, "refine_ms": dref, "reuse_ms": dreu,
+        extras["decode"] = {"workload": ds.name, "refine_ms": dref, "reuse_ms": dreu, "refine_kernels_ms": dph,
                             "key_bytes": key_bytes, "refine_hbm_frac": key_bytes / (dref * 1e-3) / (hbm * 1e9)}
         del dq, dw, dk
         # guardrail: the guarded Refine call against both of its paths on short prefills

@@ -268,7 +268,9 @@ PIVOT_API void pivot_set_debug_flags(int flags);
  * by the caller), every following call records them on its stream:
  * events[0] before its first kernel, events[1] after the scan kernel,
  * events[2] after the refine kernel and events[3] after the last kernel
- * (unused slots are recorded at the same point as the previous one).
+ * (unused slots are recorded at the same point as the previous one).  A
+ * decode-batch call records events[1] after its proxies and scan, events[2]
+ * after its selection and emit, events[3] after its last kernel.
  * Pass NULL to stop.  Not thread-safe; a process-wide setting. */
 PIVOT_API void pivot_set_profile_events(void **events, int n);
 

@@ -389,14 +389,22 @@ def _varlen_common(q, w, kc, offsets, g):
     B = off_h.numel() - 1
     if q.dim() != 3 or q.shape[0] != B * g or w.shape != (B * g, q.shape[1]) or kc.shape[1] != q.shape[2]:
         raise ValueError("expected q [B*g,H,d], w [B*g,H], k_cache [sum P, d]")
-    off_d = off_h.to(q.device)
-    return B, q.shape[1], q.shape[2], _dt(q), off_h, off_d
+    return B, q.shape[1], q.shape[2], _dt(q), off_h
+
+
+def _offsets_dev(off_h, device, stream):
+    """The offsets on the device, copied on the call's stream from pinned memory without
+    blocking the host (the launches that follow are queued behind the copy)."""
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    with torch.cuda.stream(s):
+        return off_h.pin_memory().to(device, non_blocking=True)
 
 
 def reuse_varlen(q, w, k_cache, offsets, topk: int, g: int, *, scores: bool = False,
                  ws: Optional[Workspace] = None, stream=None):
     """Eq. (3)-(6) for a batch of MTP decode groups.  Returns (indices [B*g,topk], scores|None)."""
-    B, H, d, dt, off_h, off_d = _varlen_common(q, w, k_cache, offsets, g)
+    B, H, d, dt, off_h = _varlen_common(q, w, k_cache, offsets, g)
+    off_d = _offsets_dev(off_h, q.device, stream)
     idx = torch.empty((B * g, topk), dtype=torch.int32, device=q.device)
     sc = torch.empty((B * g, topk), dtype=torch.float32, device=q.device) if scores else None
     nbytes = varlen_workspace_size(OP_REUSE, off_h, H, d, topk, topk, g, dt)
@@ -410,7 +418,8 @@ def reuse_varlen(q, w, k_cache, offsets, topk: int, g: int, *, scores: bool = Fa
 def refine_varlen(q, w, k_cache, offsets, topk: int, c: int, g: int, *, scores: bool = False, cand: bool = False,
                   ws: Optional[Workspace] = None, stream=None):
     """Eq. (3)-(5),(7)-(9) for a batch of MTP decode groups."""
-    B, H, d, dt, off_h, off_d = _varlen_common(q, w, k_cache, offsets, g)
+    B, H, d, dt, off_h = _varlen_common(q, w, k_cache, offsets, g)
+    off_d = _offsets_dev(off_h, q.device, stream)
     idx = torch.empty((B * g, topk), dtype=torch.int32, device=q.device)
     sc = torch.empty((B * g, topk), dtype=torch.float32, device=q.device) if scores else None
     cd = torch.empty((B, c), dtype=torch.int32, device=q.device) if cand else None
@@ -438,7 +447,9 @@ def set_debug_flags(flags: int) -> None:
 
 class KernelTimer:
     """Records CUDA events between the library's kernel launches (on the call's
-    stream): times of the scan kernel, the refine kernel and the row select."""
+    stream): times of the scan kernel, the refine kernel and the row select of a
+    prefill call; of the proxies + scan, the selection + emit, and the re-scoring +
+    row select of a decode call."""
 
     def __init__(self):
         self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
@@ -456,7 +467,7 @@ class KernelTimer:
         lib().pivot_set_profile_events(None, 0)
 
     def ms(self):
-        """(scan, refine, rowselect) milliseconds of the last call (after a sync)."""
+        """The three phase times (ms) of the last call, in the order above (after a sync)."""
         e = self.ev
         return e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])
 

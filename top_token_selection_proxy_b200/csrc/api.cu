@@ -174,7 +174,7 @@ struct DecodeWs {
   uint32_t* keys;
   uint64_t* sscratch;
   float* fscratch;
-  int scan_grid, slices, simt_grid;
+  int scan_grid, simt_grid;
   int64_t simt_per_block, simt_member_off;
   size_t bytes;
 };
@@ -199,17 +199,14 @@ DecodeWs carve_decode(void* base, int op, int B, const int64_t* off, int H, int 
     DecodeArgs& a = w.d;
     a.n_sets = n_sets;
     w.scan_grid = (int)std::min<int64_t>(sms, n_sets);
-    w.slices = (int)((pmax + kDecodeSlice - 1) / kDecodeSlice);
     a.proxy = cv.take<uint16_t>((size_t)B * H * d);
     a.wbar = cv.take<float>((size_t)B * kWbarStride);
     a.set_off = cv.take<int32_t>((size_t)B + 1);
     a.scores = cv.take<uint32_t>((size_t)total);
     a.ties = cv.take<uint64_t>((size_t)total);
+    a.ties2 = cv.take<uint64_t>((size_t)total);
     a.hist1 = cv.take<uint32_t>((size_t)B * 2048);
-    a.hist2 = cv.take<uint32_t>((size_t)B * 2048);
     a.sel = cv.take<uint64_t>((size_t)B * n_sel);
-    a.cnt = cv.take<uint32_t>((size_t)B);
-    a.tcnt = cv.take<uint32_t>((size_t)B);
     if (op == PIVOT_OP_REFINE) {
       if (!user_cand) w.cand = cv.take<int32_t>((size_t)B * c);
       w.keys = cv.take<uint32_t>((size_t)B * g * c);
@@ -444,7 +441,7 @@ pivot_status run_decode(int op, const void* q, const float* w, const void* kc, c
     return e == cudaSuccess ? PIVOT_OK : cuda_fail(e, "simt kernel");
   }
 
-  if ((int64_t)B * W.slices > 0x7FFFFFFFLL) return PIVOT_ERR_UNSUPPORTED_SHAPE;  // selection grid
+  if ((int64_t)B * kSelCl > 0x7FFFFFFFLL) return PIVOT_ERR_UNSUPPORTED_SHAPE;  // selection grid
   const int n_sel = sel_size(op, k, c, g);
   int32_t* cand = cand_opt ? cand_opt : W.cand;
   DecodeArgs a = W.d;
@@ -467,9 +464,17 @@ pivot_status run_decode(int op, const void* q, const float* w, const void* kc, c
   CUtensorMap kmap, pmap;  // 128-key tiles of the cache; the 64-row proxy of a sequence
   if (!make_kmap(&kmap, kc, off_host[B], d, 128) || !make_kmap(&pmap, a.proxy, (int64_t)B * H, d, H))
     return cuda_fail(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
-  e = launch_decode(a, &kmap, &pmap, W.scan_grid, W.slices, s);
-  if (e != cudaSuccess) return cuda_fail(e, "decode kernels");
-  if (op == PIVOT_OP_REUSE) return PIVOT_OK;
+  prof(0, s);
+  e = launch_decode_scan(a, &kmap, &pmap, W.scan_grid, s);
+  if (e != cudaSuccess) return cuda_fail(e, "decode scan");
+  prof(1, s);
+  e = launch_decode_select(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "decode selection");
+  prof(2, s);
+  if (op == PIVOT_OP_REUSE) {
+    prof(3, s);
+    return PIVOT_OK;
+  }
 
   RefineArgs r{};
   r.q = reinterpret_cast<const uint16_t*>(q);
@@ -513,7 +518,9 @@ pivot_status run_decode(int op, const void* q, const float* w, const void* kc, c
   rs.out_idx = indices;
   rs.out_scores = scores;
   e = launch_rowselect(rs, (int)std::min<int64_t>(8 * num_sms(), rs.n_rows), s);
-  return e == cudaSuccess ? PIVOT_OK : cuda_fail(e, "rowselect kernel");
+  if (e != cudaSuccess) return cuda_fail(e, "rowselect kernel");
+  prof(3, s);
+  return PIVOT_OK;
 }
 
 }  // namespace

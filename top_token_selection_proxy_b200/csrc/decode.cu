@@ -16,13 +16,13 @@
 //      blocks exactly as the prefill scan reads (group, lane quarter).  The
 //      epilogue writes each key's order key and counts its top 11 bits in a
 //      per-sequence histogram;
-//   3. select (two passes over the order keys, many CTAs per sequence): the
-//      histogram's threshold bin, then the next 11 bits inside that bin;
-//      keys above the thresholds are appended as winners, keys in the final
-//      bin pair as ties;
-//   4. emit (one CTA per sequence): the best of the ties by the full (score,
-//      index) order complete the exact selection; the candidate row (Refine)
-//      or the g member rows (Reuse) are written from it.
+//   3. select + emit (one thread-block cluster per sequence, one launch): the
+//      histogram's threshold bin, then the next 11 bits inside that bin, counted
+//      in the CTAs' shared memory and summed through distributed shared memory;
+//      the best of the last bin's keys by the full (score, index) order complete
+//      the exact selection, and the candidate row (Refine) or the g member rows
+//      (Reuse) are written from it.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
 #include <cstddef>
@@ -38,7 +38,6 @@ namespace {
 
 constexpr int kDH = 64;          // heads (the tensor-core shape)
 constexpr int kSetTiles = kDecodeSetKeys / 128;  // key tiles per accumulator: one per 64-column slot
-constexpr int kSelThreads = 256;
 
 template <int D>
 struct DScanCfg {
@@ -83,7 +82,7 @@ __host__ __device__ constexpr int prep_blocks_per_seq(int D) { return (kDH * (D 
 
 // Blocks b*PB .. b*PB+PB-1: sequence b's proxy (Eq. 4: the fp32 mean of its g
 // query rows, summed in member order, rounded to bf16), w-bar (written in the
-// epilogue's permuted layout) and zeroed selection state.  Last block:
+// epilogue's permuted layout) and its zeroed digit histogram.  Last block:
 // set_off[b] = sum over b' < b of ceil(P_b' / kDecodeSetKeys).
 __global__ void __launch_bounds__(256) dprep_kernel(const DecodeArgs a) {
   const int tid = threadIdx.x;
@@ -111,14 +110,7 @@ __global__ void __launch_bounds__(256) dprep_kernel(const DecodeArgs a) {
     return;
   }
   const int b = blockIdx.x / PB, part = blockIdx.x % PB;
-  for (int i = part * 256 + tid; i < 4096; i += PB * 256) {
-    if (i < 2048) a.hist1[(int64_t)b * 2048 + i] = 0u;
-    else a.hist2[(int64_t)b * 2048 + i - 2048] = 0u;
-  }
-  if (part == 0 && tid == 0) {
-    a.cnt[b] = 0u;
-    a.tcnt[b] = 0u;
-  }
+  for (int i = part * 256 + tid; i < 2048; i += PB * 256) a.hist1[(int64_t)b * 2048 + i] = 0u;
   const int XC = a.D / 8;  // 16-byte chunks per row
   const int g = a.g;       // <= 16
   const int64_t r0 = (int64_t)b * g;
@@ -410,7 +402,22 @@ __global__ void __launch_bounds__(576, 1) dscan_kernel(const __grid_constant__ C
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
-// ------------------------------------------------------------------ 3. select
+// ------------------------------------------------------------------ 3. select + emit
+// One thread-block cluster of kSelCl CTAs per sequence, one launch for the exact
+// selection of n = min(n_sel, P) keys by the order (score desc, index asc):
+//   level 1  T1 = the bin of the scan's top-11-bit histogram where the count from the
+//            top reaches n.  Each CTA reads its share of the sequence's order keys once
+//            (16-byte loads): keys above T1 are selected, keys in T1 are listed as
+//            level-1 ties and their next 11 bits are counted in the CTA's histogram;
+//   level 2  the CTAs' histograms are summed through distributed shared memory; T2 is
+//            the bin where the count reaches the rest of n; the level-1 ties are split
+//            over the CTAs: above T2 selected, in T2 listed as level-2 ties;
+//   final    CTA 0 takes the best of the level-2 ties by the full (score, index) order
+//            and writes the candidate row (Refine) or the g member rows (Reuse).
+// The list counters sit in CTA 0's shared memory (one remote atomic per warp and chunk).
+// Selected entries go straight into CTA 0's shared memory when n_sel fits its stage
+// (kSelStage entries), else to the workspace; the ties lists have room for every key
+// of the sequence, so no list can overflow.
 namespace {
 
 struct BinThr {
@@ -419,9 +426,11 @@ struct BinThr {
   uint32_t at;     // entries in bin T
 };
 
-// Over a 2048-bin histogram hg (global) with `total` entries: the bin T where the
-// count from the top first reaches `need` (need <= total).  All threads call.
-__device__ BinThr hist_threshold(const uint32_t* hg, uint32_t need, uint32_t total, uint32_t* wtot, int* scal) {
+// Over 2048 counts read by ld(bin) with `total` entries: the bin T where the count from
+// the top first reaches need (need <= total).  All NT threads of the block call it.
+template <int NT, typename Ld>
+__device__ BinThr bin_threshold(Ld&& ld, uint32_t need, uint32_t total, uint32_t* wtot, int* scal) {
+  constexpr int BPT = 2048 / NT;
   BinThr r{-1, total, 0u};
   if (need >= total) return r;
   const int t = threadIdx.x;
@@ -430,10 +439,10 @@ __device__ BinThr hist_threshold(const uint32_t* hg, uint32_t need, uint32_t tot
     scal[1] = (int)total;
     scal[2] = 0;
   }
-  uint32_t loc[8], sum = 0;
+  uint32_t loc[BPT], sum = 0;
 #pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    loc[u] = hg[2047 - 8 * t - u];
+  for (int u = 0; u < BPT; ++u) {
+    loc[u] = ld(2047 - BPT * t - u);
     sum += loc[u];
   }
   const uint32_t incl = warp_incl_scan(sum);
@@ -444,9 +453,9 @@ __device__ BinThr hist_threshold(const uint32_t* hg, uint32_t need, uint32_t tot
   if (excl < need && need <= excl + sum) {
     uint32_t c = excl;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < BPT; ++u) {
       if (c + loc[u] >= need) {
-        scal[0] = 2047 - 8 * t - u;
+        scal[0] = 2047 - BPT * t - u;
         scal[1] = (int)c;
         scal[2] = (int)loc[u];
         break;
@@ -462,130 +471,221 @@ __device__ BinThr hist_threshold(const uint32_t* hg, uint32_t need, uint32_t tot
   return r;
 }
 
-}  // namespace
+constexpr int kSelV4 = 4;  // 16-byte loads of order keys per thread and level-1 chunk (16 keys)
 
-// Block b * slices + z handles keys [z * kDecodeSlice, (z + 1) * kDecodeSlice) of sequence b.
-// level 1: winners = digit1 > T1; counts digit2 of the keys in bin T1.
-// level 2: winners = digit1 == T1 && digit2 > T2; ties = (T1, T2).
-// Every thread holds its 32 keys in registers; the block claims room for all
-// of its winners (and ties) with one atomic per counter.
-__global__ void __launch_bounds__(kSelThreads) dselect_kernel(const DecodeArgs a, int slices, int level) {
-  constexpr int U = kDecodeSlice / kSelThreads;
-  static_assert(U == 32, "one bit per key of a thread");
-  __shared__ uint32_t h[kHist11Words];
-  __shared__ uint32_t wtot[8];
-  __shared__ uint32_t wcnt[2][8];
-  __shared__ uint32_t base_s[2];
-  __shared__ int scal[4];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int b = (int)(blockIdx.x / (unsigned)slices);
-  const int64_t P = a.key_off[b + 1] - a.key_off[b];
-  const int64_t s0 = (int64_t)(blockIdx.x % (unsigned)slices) * kDecodeSlice;
-  if (s0 >= P) return;
-  const int64_t s1 = min64(P, s0 + kDecodeSlice);
-  const uint32_t need = (uint32_t)min64(a.n_sel, P);
-  const uint32_t* keys = a.scores + a.key_off[b];
-  const BinThr t1 = hist_threshold(a.hist1 + (int64_t)b * 2048, need, (uint32_t)P, wtot, scal);
-  if (level == 2 && t1.T < 0) return;  // level 1 took every key
-  BinThr t2{-1, 0u, 0u};
-  if (level == 2) t2 = hist_threshold(a.hist2 + (int64_t)b * 2048, need - t1.above, t1.at, wtot, scal);
-  if (level == 1) {
-    for (int i = tid; i < kHist11Words; i += kSelThreads) h[i] = 0u;
-    __syncthreads();
-  }
-  uint32_t v[U];
-#pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const int64_t s = s0 + u * kSelThreads + tid;
-    v[u] = s < s1 ? keys[s] : 0u;
-  }
-  uint32_t win = 0u, tie = 0u;
-#pragma unroll
-  for (int u = 0; u < U; ++u) {
-    const bool valid = s0 + u * kSelThreads + tid < s1;
-    const int d1 = (int)(v[u] >> 21), d2 = (int)((v[u] >> 10) & 2047u);
-    if (level == 1) {
-      if (valid && d1 > t1.T) win |= 1u << u;
-      if (valid && d1 == t1.T) atomicAdd(&h[h11((uint32_t)d2)], 1u);
-    } else if (valid && d1 == t1.T) {
-      if (d2 > t2.T) win |= 1u << u;
-      if (d2 == t2.T) tie |= 1u << u;
-    }
-  }
+struct SelClSmem {
+  uint4 keys[kSelV4][kSelClThreads];  // each thread's keys of the current chunk (read back only by it)
+  uint32_t h2[kHist11Words];     // this CTA's counts of the second digit of its level-1 ties
+  uint32_t comb[2048 / kSelCl];  // cluster sums of this CTA's slice of the second-digit bins
+  uint32_t ctr[4];               // (CTA 0) list lengths: selected, level-1 ties, level-2 ties
+  uint32_t wtot[kSelClThreads / 32];
+  int scal[4];
+  SelSmem S;
+  uint64_t bot[16];
+};
+
+// Warp-aggregated append of each thread's candidates (bit u of win / tie; entry(u) is the
+// packed entry) to the selected list sl (counter cs) and a ties list tl (counter ct); the
+// counters may be another CTA's shared memory.  Positions at or past cap_s / cap_t are
+// dropped and reported.  The whole warp calls.
+template <int U, typename E>
+__device__ __forceinline__ bool append2(E&& entry, uint32_t win, uint32_t tie, uint64_t* sl, uint32_t* cs,
+                                        uint32_t cap_s, uint64_t* tl, uint32_t* ct, uint32_t cap_t) {
+  const int lane = threadIdx.x & 31;
   const uint32_t nw = __popc(win), nt = __popc(tie);
   const uint32_t iw = warp_incl_scan(nw), it = warp_incl_scan(nt);
+  const uint32_t tw = __shfl_sync(0xFFFFFFFFu, iw, 31), tt = __shfl_sync(0xFFFFFFFFu, it, 31);
+  if (tw == 0u && tt == 0u) return false;
+  uint32_t bw = 0, bt = 0;
   if (lane == 31) {
-    wcnt[0][warp] = iw;
-    wcnt[1][warp] = it;
+    if (tw) bw = atomicAdd(cs, tw);
+    if (tt) bt = atomicAdd(ct, tt);
   }
-  __syncthreads();
-  if (tid == 0) {
-    uint32_t tw = 0, tt = 0;
-    for (int x = 0; x < kSelThreads / 32; ++x) {
-      tw += wcnt[0][x];
-      tt += wcnt[1][x];
-    }
-    base_s[0] = tw ? atomicAdd(&a.cnt[b], tw) : 0u;
-    base_s[1] = tt ? atomicAdd(&a.tcnt[b], tt) : 0u;
-  }
-  __syncthreads();
-  uint32_t pw = base_s[0] + iw - nw, pt = base_s[1] + it - nt;
-  for (int x = 0; x < warp; ++x) {
-    pw += wcnt[0][x];
-    pt += wcnt[1][x];
-  }
-  uint64_t* sel = a.sel + (int64_t)b * a.n_sel;
-  uint64_t* ties = a.ties + a.key_off[b];
-  bool over = false;  // counts that do not match the stored keys (an aborted scan)
+  bw = __shfl_sync(0xFFFFFFFFu, bw, 31);
+  bt = __shfl_sync(0xFFFFFFFFu, bt, 31);
+  uint32_t pw = bw + iw - nw, pt = bt + it - nt;
+  bool over = false;
 #pragma unroll
   for (int u = 0; u < U; ++u) {
-    const uint32_t s = (uint32_t)(s0 + u * kSelThreads + tid);
     if (win & (1u << u)) {
-      if (pw < need) sel[pw] = pack_entry(v[u], s);
+      if (pw < cap_s) sl[pw] = entry(u);
       else over = true;
       ++pw;
     }
     if (tie & (1u << u)) {
-      if (pt < (uint32_t)P) ties[pt] = pack_entry(v[u], s);
+      if (pt < cap_t) tl[pt] = entry(u);
       else over = true;
       ++pt;
     }
   }
-  if (over) atomicOr(a.status, DEV_ERR_BOUNDS);
-  if (level == 1 && t1.T >= 0) {
-    __syncthreads();
-    for (int i = tid; i < 2048; i += kSelThreads) {
-      const uint32_t c = h[h11(i)];
-      if (c) atomicAdd(&a.hist2[(int64_t)b * 2048 + i], c);
-    }
-  }
+  return over;
 }
 
-// ------------------------------------------------------------------ 4. emit
-__global__ void __launch_bounds__(kSelThreads) demit_kernel(const DecodeArgs a) {
-  __shared__ SelSmem S;
-  __shared__ uint64_t bot[16];
-  const Group<kSelThreads> G{(int)threadIdx.x, 0};
-  for (int b = blockIdx.x; b < a.B; b += gridDim.x) {
-    const int64_t P = a.key_off[b + 1] - a.key_off[b];
-    const uint32_t need = (uint32_t)min64(a.n_sel, P);
-    uint64_t* sel = a.sel + (int64_t)b * a.n_sel;
-    const uint32_t nw = min(a.cnt[b], need);
-    uint32_t m = nw;
-    if (nw < need) {  // the best (need - nw) ties, by the full (score, index) order
-      const uint64_t* ties = a.ties + a.key_off[b];
-      const uint32_t nt = min(a.tcnt[b], (uint32_t)P), need3 = need - nw;
-      const uint64_t th = radix_threshold<kSelThreads>(ties, nt, need3, need3, S, G);
-      m += compact_ge<kSelThreads>(ties, sel + nw, nt, th, S, G);
+}  // namespace
+
+__global__ void __launch_bounds__(kSelClThreads) dselect_cluster_kernel(const DecodeArgs a) {
+  namespace cg = cooperative_groups;
+  constexpr int NT = kSelClThreads, SL = 2048 / kSelCl;
+  constexpr int V4 = kSelV4;
+  __shared__ SelClSmem sm;
+  extern __shared__ uint64_t stage[];  // kSelStage entries; CTA 0's holds the selected entries
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int b = (int)(blockIdx.x / kSelCl);
+  const int tid = threadIdx.x;
+  const int64_t kbase = a.key_off[b];
+  const int64_t P = a.key_off[b + 1] - kbase;
+  const uint32_t need = (uint32_t)min64(a.n_sel, P);
+  uint64_t* X = a.ties + kbase;   // level-1 ties
+  uint64_t* Y = a.ties2 + kbase;  // level-2 ties
+  const bool staged = a.n_sel <= kSelStage;
+  uint64_t* sel = staged ? cluster.map_shared_rank(stage, 0) : a.sel + (int64_t)b * a.n_sel;
+  uint32_t* ctr = cluster.map_shared_rank(sm.ctr, 0);
+
+  // this CTA's share [s0, s1) of the order keys: up to 3 keys on each side by plain loads,
+  // the 16-byte-aligned middle [a0, a1) by vector loads; its first chunk is prefetched
+  // into L2 while the level-1 threshold is found
+  const int64_t s0 = P * rank / kSelCl, s1 = P * (rank + 1) / kSelCl;
+  const uint32_t* keys = a.scores + kbase;
+  const int64_t a0 = min64(s1, s0 + ((4 - ((kbase + s0) & 3)) & 3));
+  const int64_t a1 = max64(a0, s1 - ((kbase + s1) & 3));
+  const int64_t nvec = (a1 - a0) >> 2;
+  const uint4* kv = reinterpret_cast<const uint4*>(keys + a0);
+#pragma unroll
+  for (int j = 0; j < V4; ++j)
+    if (j * NT + tid < nvec) prefetch_l2(kv + j * NT + tid);
+
+  for (int i = tid; i < kHist11Words; i += NT) sm.h2[i] = 0u;
+  if (tid < 4) sm.ctr[tid] = 0u;
+  const uint32_t* hg1 = a.hist1 + (int64_t)b * 2048;
+  const BinThr t1 = bin_threshold<NT>([&](int i) { return hg1[i]; }, need, (uint32_t)P, sm.wtot, sm.scal);
+  __syncthreads();
+  cluster.sync();  // (0) CTA 0's counters are zero before any append
+  bool over = false;
+
+  // ---- level 1: a key is selected when its top 11 bits exceed T1 (every key when T1 < 0),
+  // a level-1 tie when they equal T1
+  const bool all1 = t1.T < 0;
+  const uint32_t top1 = all1 ? 0u : (((uint32_t)t1.T << 21) | 0x1FFFFFu);  // selected: key > top1
+  // append the candidates (bits of win | tie) of each thread: warp-aggregated positions, one
+  // remote counter update per warp and list; each thread then writes only its own few entries
+  auto place = [&](uint32_t win, uint32_t tie, auto&& key_of, auto&& pos_of) {
+    const int lane = tid & 31;
+    const uint32_t nw = __popc(win), nt = __popc(tie);
+    const uint32_t iw = warp_incl_scan(nw), it = warp_incl_scan(nt);
+    const uint32_t tw = __shfl_sync(0xFFFFFFFFu, iw, 31), tt = __shfl_sync(0xFFFFFFFFu, it, 31);
+    if (tw == 0u && tt == 0u) return;
+    uint32_t bw = 0, bt = 0;
+    if (lane == 31) {
+      if (tw) bw = atomicAdd(&ctr[0], tw);
+      if (tt) bt = atomicAdd(&ctr[1], tt);
     }
-    G.sync();
-    if (a.mode == EMIT_CAND) {
-      emit_row<kSelThreads>(sel, m, 0xFFFFFFFFu, 0ull, a.cand + (int64_t)b * a.n_sel,
-                            a.cand_scores ? a.cand_scores + (int64_t)b * a.n_sel : nullptr, (uint32_t)a.n_sel, S, G);
-    } else {
-      emit_reuse<kSelThreads>(sel, m, a.topk, P - a.g, a.g, (int64_t)b * a.g, a.out_idx, a.out_scores, S, bot, G);
+    uint32_t pw = __shfl_sync(0xFFFFFFFFu, bw, 31) + iw - nw, pt = __shfl_sync(0xFFFFFFFFu, bt, 31) + it - nt;
+    for (uint32_t c = win | tie; c; c &= c - 1u) {
+      const int u = __ffs(c) - 1;
+      const uint32_t v = key_of(u);
+      const uint64_t e = pack_entry(v, (uint32_t)pos_of(u));
+      if ((win >> u) & 1u) {
+        if (pw < need) sel[pw] = e;
+        else over = true;
+        ++pw;
+      } else {
+        if (pt < (uint32_t)P) X[pt] = e;
+        else over = true;
+        ++pt;
+        atomicAdd(&sm.h2[h11((v >> 10) & 2047u)], 1u);  // second digit of the tie
+      }
     }
-    G.sync();
+  };
+  {
+    const int nh = (int)(a0 - s0);
+    const int64_t s = tid < nh ? s0 + tid : a1 + (tid - nh);
+    const bool valid = tid < 8 && (tid < nh || s < s1);
+    const uint32_t v = valid ? keys[s] : 0u;
+    const uint32_t win = (valid && (all1 || v > top1)) ? 1u : 0u;
+    const uint32_t tie = (valid && (int)(v >> 21) == t1.T) ? 1u : 0u;
+    place(win, tie, [&](int) { return v; }, [&](int) { return s; });
+  }
+  uint32_t* kst = reinterpret_cast<uint32_t*>(&sm.keys[0][0]);
+  for (int64_t v0 = 0; v0 < nvec; v0 += (int64_t)NT * V4) {
+    uint4 x[V4];
+#pragma unroll
+    for (int j = 0; j < V4; ++j) {
+      const int64_t vi = v0 + j * NT + tid;
+      x[j] = vi < nvec ? kv[vi] : make_uint4(0u, 0u, 0u, 0u);
+    }
+    uint32_t win = 0u, tie = 0u;
+#pragma unroll
+    for (int j = 0; j < V4; ++j) {
+      const bool valid = v0 + j * NT + tid < nvec;
+      const uint32_t c4[4] = {x[j].x, x[j].y, x[j].z, x[j].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (valid && (all1 || c4[e] > top1)) win |= 1u << (4 * j + e);
+        if (valid && (int)(c4[e] >> 21) == t1.T) tie |= 1u << (4 * j + e);
+      }
+    }
+    if (win | tie) {
+#pragma unroll
+      for (int j = 0; j < V4; ++j) sm.keys[j][tid] = x[j];
+    }
+    place(win, tie, [&](int u) { return kst[((u >> 2) * NT + tid) * 4 + (u & 3)]; },
+          [&](int u) { return a0 + 4 * (v0 + (u >> 2) * NT + tid) + (u & 3); });
+  }
+  __syncthreads();
+  cluster.sync();  // (1) the level-1 lists and every CTA's second-digit histogram are complete
+
+  if (tid < SL) {
+    uint32_t c = 0;
+    for (int r = 0; r < kSelCl; ++r) c += cluster.map_shared_rank(sm.h2, r)[h11((uint32_t)(rank * SL + tid))];
+    sm.comb[tid] = c;
+  }
+  const uint32_t NW1 = ctr[0], at1 = min(ctr[1], (uint32_t)P);
+  cluster.sync();  // (2) the combined second-digit histogram is complete; the counts are read
+  BinThr t2{-1, 0u, 0u};
+  if (t1.T >= 0 && NW1 < need)
+    t2 = bin_threshold<NT>([&](int i) { return cluster.map_shared_rank(sm.comb, i / SL)[i % SL]; }, need - NW1, at1,
+                           sm.wtot, sm.scal);
+
+  // ---- level 2 over this CTA's portion [q0, q1) of the level-1 ties
+  {
+    constexpr int U = 8;
+    const uint32_t q0 = (uint32_t)((uint64_t)at1 * rank / kSelCl),
+                   q1 = (uint32_t)((uint64_t)at1 * (rank + 1) / kSelCl);
+    for (uint32_t c0 = q0; c0 < q1; c0 += NT * U) {
+      uint64_t x[U];
+      uint32_t win = 0u, tie = 0u;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint32_t i = c0 + u * NT + tid;
+        x[u] = i < q1 ? X[i] : 0ull;
+        const int d2 = (int)((x[u] >> 42) & 2047u);
+        if (i < q1 && d2 > t2.T) win |= 1u << u;
+        if (i < q1 && d2 == t2.T) tie |= 1u << u;
+      }
+      over |= append2<U>([&](int u) { return x[u]; }, win, tie, sel, &ctr[0], need, Y, &ctr[2], (uint32_t)P);
+    }
+  }
+  if (over) atomicOr(a.status, DEV_ERR_BOUNDS);
+  __syncthreads();
+  cluster.sync();  // (3) the selected list and the level-2 ties are complete
+  if (rank != 0) return;
+
+  const Group<NT> G{tid, 0};
+  uint64_t* buf = staged ? stage : sel;
+  const uint32_t nw = min(sm.ctr[0], need);
+  uint32_t m = nw;
+  if (nw < need) {  // the best (need - nw) level-2 ties by the full (score, index) order
+    const uint32_t nt = min(sm.ctr[2], (uint32_t)P), need3 = need - nw;
+    const uint64_t th = radix_threshold<NT>(Y, nt, need3, need3, sm.S, G);
+    m += compact_ge<NT>(Y, buf + nw, nt, th, sm.S, G);
+  }
+  G.sync();
+  if (a.mode == EMIT_CAND) {
+    emit_row<NT>(buf, m, 0xFFFFFFFFu, 0ull, a.cand + (int64_t)b * a.n_sel,
+                 a.cand_scores ? a.cand_scores + (int64_t)b * a.n_sel : nullptr, (uint32_t)a.n_sel, sm.S, G);
+  } else {
+    emit_reuse<NT>(buf, m, a.topk, P - a.g, a.g, (int64_t)b * a.g, a.out_idx, a.out_scores, sm.S, sm.bot, G);
   }
 }
 
@@ -596,8 +696,8 @@ size_t decode_scan_smem_bytes(int D) {
   return 0;
 }
 
-cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, const CUtensorMap* pmap, int scan_grid,
-                          int slices, cudaStream_t s) {
+cudaError_t launch_decode_scan(const DecodeArgs& a, const CUtensorMap* kmap, const CUtensorMap* pmap, int scan_grid,
+                               cudaStream_t s) {
   if (a.H != kDH || (a.D != 64 && a.D != 128)) return cudaErrorInvalidValue;
   const int64_t prep_grid = (int64_t)a.B * prep_blocks_per_seq(a.D) + 1;
   if (prep_grid > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
@@ -614,14 +714,25 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, const CU
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     k<<<scan_grid, DScanCfg<64>::THREADS, smem, s>>>(*kmap, *pmap, a);
   }
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const unsigned sg = (unsigned)slices * (unsigned)a.B;
-  dselect_kernel<<<sg, kSelThreads, 0, s>>>(a, slices, 1);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  dselect_kernel<<<sg, kSelThreads, 0, s>>>(a, slices, 2);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  demit_kernel<<<a.B < 1184 ? a.B : 1184, kSelThreads, 0, s>>>(a);
   return cudaGetLastError();
+}
+
+cudaError_t launch_decode_select(const DecodeArgs& a, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)a.B * kSelCl);
+  cfg.blockDim = dim3(kSelClThreads);
+  cfg.dynamicSmemBytes = kSelStage * sizeof(uint64_t);
+  cudaFuncSetAttribute(dselect_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)cfg.dynamicSmemBytes);
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = kSelCl;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, dselect_cluster_kernel, a);
 }
 
 }  // namespace pivot

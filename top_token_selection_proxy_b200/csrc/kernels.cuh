@@ -106,7 +106,9 @@ struct SimtArgs {
 
 // MTP decode groups: one group of g draft rows per sequence (decode.cu).
 constexpr int kDecodeSetKeys = 512;  // keys per scan set (4 tiles of 128, one per accumulator slot)
-constexpr int kDecodeSlice = 8192;   // keys per selection block
+constexpr int kSelCl = 8;            // CTAs of the decode selection's cluster (one per sequence)
+constexpr int kSelClThreads = 512;   // threads per CTA of that cluster
+constexpr int kSelStage = 4096;      // selected entries the cluster keeps in shared memory
 constexpr int kWbarStride = 80;      // floats per sequence of the permuted w-bar table (4 rows of 20)
 struct DecodeArgs {
   const uint16_t* q;        // bf16 bits [B*g, H, D]
@@ -123,11 +125,9 @@ struct DecodeArgs {
   int32_t* set_off;         // [B+1] first scan set of each sequence
   uint32_t* scores;         // [sum P] order keys of the proxy scores (Eq. 5)
   uint32_t* hist1;          // [B, 2048] counts of the order keys' top 11 bits
-  uint32_t* hist2;          // [B, 2048] counts of the next 11 bits inside the level-1 threshold bin
-  uint64_t* sel;            // [B, n_sel] packed selected entries
-  uint32_t* cnt;            // [B] entries in sel
-  uint64_t* ties;           // [sum P] packed entries of the final threshold bin pair
-  uint32_t* tcnt;           // [B]
+  uint64_t* sel;            // [B, n_sel] packed selected entries (when n_sel > kSelStage)
+  uint64_t* ties;           // [sum P] packed entries: level-1 lists, then the level-2 ties
+  uint64_t* ties2;          // [sum P] packed entries: level-2 lists
   // outputs
   int32_t* cand;            // [B, n_sel] (Refine)
   float* cand_scores;       // or null
@@ -144,10 +144,11 @@ cudaError_t launch_refine(const RefineArgs& a, const CUtensorMap* gather_kmap, c
 size_t refine_smem_bytes(int H, int D, int mc);
 cudaError_t launch_simt(const SimtArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_rowselect(const RowSelArgs& a, int grid, cudaStream_t s);
-// prep, scan, two selection passes and emit of a decode batch; scan_grid <= n_sets,
-// slices = ceil(max P_b / kDecodeSlice)
-cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap* kmap, const CUtensorMap* pmap, int scan_grid,
-                          int slices, cudaStream_t s);
+// MTP decode batch: prep + scan (order keys and digit histogram; scan_grid <= n_sets), then
+// the selection and emit (one cluster of kSelCl CTAs per sequence).
+cudaError_t launch_decode_scan(const DecodeArgs& a, const CUtensorMap* kmap, const CUtensorMap* pmap, int scan_grid,
+                               cudaStream_t s);
+cudaError_t launch_decode_select(const DecodeArgs& a, cudaStream_t s);
 size_t decode_scan_smem_bytes(int D);
 
 // host-side library state shared by the entry-point files (defined in api.cu)
