@@ -156,9 +156,11 @@ PIVOT_API pivot_status pivot_refine_agg(const void *q_I, const float *w_I, const
  * w_host [L,H] fp32, k_host [L,d] bf16 and out_host [L,k] int32 are host
  * pointers; they should be pinned (cudaHostAlloc / cudaHostRegister), otherwise
  * the copies do not overlap.  The keys and weights are copied first, then the
- * queries in `chunks` (1..64) runs of whole groups on a copy stream; run i is
- * indexed on `stream` (pivot_refine_range) once its rows have landed, while
- * run i+1 is copied in and run i-1's rows are copied back on a second copy
+ * queries in `chunks` (1..64) runs of whole groups on a copy stream, from the
+ * sequence's end to its start (the groups with the longest prefixes first, so
+ * the run indexed last is the cheapest); each run is indexed on `stream`
+ * (pivot_refine_range) once its rows have landed, while the next run is
+ * copied in and the previous run's rows are copied back on a second copy
  * stream.  ws is a DEVICE buffer of pivot_refine_host_workspace_size bytes
  * (256-byte aligned) that holds the device copies and the refine workspace.
  * Asynchronous: when the call returns the work is queued and `stream` is ordered

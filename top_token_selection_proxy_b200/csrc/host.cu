@@ -3,9 +3,12 @@
 // queries in runs of whole groups on a copy stream; each run is indexed with the
 // group-range call on the caller's stream as soon as it has landed, and its rows
 // are copied back on a second copy stream while later runs are still being
-// copied in or indexed.  Every step is ordered by events; nothing synchronises
-// the host.  (Group ranges: the groups of Eq. (2) are independent given k_I, so a
-// run's rows equal the same rows of one whole-sequence call.)
+// copied in or indexed.  The runs go from the sequence's end to its start: a
+// group's work grows with its causal prefix, so the heaviest runs overlap the
+// copies of the rest and the run indexed last, whose kernels and copy back are
+// not overlapped, is the cheapest.  Every step is ordered by events; nothing
+// synchronises the host.  (Group ranges: the groups of Eq. (2) are independent
+// given k_I, so a run's rows equal the same rows of one whole-sequence call.)
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -117,8 +120,9 @@ PIVOT_API pivot_status pivot_refine_host(const void* q_host, const float* w_host
   if ((e = cudaMemcpyAsync(k_dev, k_host, (size_t)L * d * 2, cudaMemcpyHostToDevice, p.s_in)) != cudaSuccess ||
       (e = cudaMemcpyAsync(w_dev, w_host, (size_t)L * wrow, cudaMemcpyHostToDevice, p.s_in)) != cudaSuccess)
     return record_cuda_error(e, "copy in");
-  int i = 0;
-  for (int64_t g0 = 0; g0 < G; g0 += per, ++i) {
+  const int n_runs = (int)((G + per - 1) / per);
+  for (int i = 0; i < n_runs; ++i) {
+    const int64_t g0 = (int64_t)(n_runs - 1 - i) * per;  // the last run first
     const int64_t g1 = std::min<int64_t>(G, g0 + per);
     const int64_t t0 = g0 * g, t1 = std::min<int64_t>(g1 * g, L);
     if ((e = cudaMemcpyAsync(q_dev + t0 * qrow, reinterpret_cast<const char*>(q_host) + t0 * qrow,
