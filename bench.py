@@ -40,7 +40,7 @@ E2E_CHUNKS = 8  # runs of groups the end-to-end call pipelines its copies over
 # ncu capture (dram__bytes_read.sum + dram__bytes_write.sum); valid only while
 # the sources the scan kernel is built from hash to `sources_sha256`.
 SCAN_TRAFFIC = {
-    "bytes": 2490000000 + 939570000,  # 2.49 GB + 939.57 MB, as ncu printed them
+    "bytes": 2500000000 + 949310000,  # 2.50 GB + 949.31 MB, as ncu printed them
     "sources": ("scan.cu", "select.cuh", "ptx.cuh", "kernels.cuh", "headsum.cuh"),
     "sources_sha256": "01067b0f47c43dbd8642eb4c13f6d200454e8682689443f487d82ec41c4fb143",
     "profile": "profiles/kernels_prefill_L131072_g8_refine_1pass.md",
