@@ -79,6 +79,10 @@ def parse():
     p.add_argument("--split", action="store_true",
                    help="one L=131072 sequence over all ranks (zig-zag group ranges + key all-gather; strong "
                         "scaling) instead of one sequence per rank")
+    p.add_argument("--split-decode", action="store_true",
+                   help="the MTP decode batch with every prefix split over all ranks (key shards, all-gather of "
+                        "the shards' selections, merge; Refine re-scores held candidates and sums; strong "
+                        "scaling)")
     p.add_argument("--profile-case", type=int, default=0, metavar="L",
                    help="profiling run: two PIVOT-Refine calls at sequence length L (H_I=64, d=128, k=2048, "
                         "c=4096, g=8) and exit; no timing, no JSON")
@@ -417,6 +421,65 @@ def run_split(args):
     M.finish(world)
 
 
+def run_split_decode(args):
+    """The MTP decode batch with every sequence's prefix split over the ranks (PIVOT-Refine): each
+    rank holds one contiguous key shard per sequence; a step is the shard selections, one
+    all-gather of them (NCCL), the merge, the re-scoring of the candidates each rank holds, one
+    element-wise sum of the member scores (NCCL) and the member top-k.  value = the batch's
+    queries / max-over-ranks step time."""
+    import torch
+
+    import top_token_selection_proxy_b200 as P
+    from top_token_selection_proxy_b200 import build, inputs
+    from top_token_selection_proxy_b200 import multigpu as M
+
+    world, rank, local = M.env()
+    M.init("nccl", world)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if rank == 0:
+        build.build()
+    M.barrier(world)
+    P.lib()
+    ds = inputs.DECODE
+    x = inputs.make_decode(ds)  # every rank draws the same batch and keeps its shards' keys
+    k_shard, shard_off, pos_base = M.shard_of(x["k"], x["offsets"], world, rank)
+    q, w, ks = to_dev(x["q"], dev), to_dev(x["w"], dev), to_dev(k_shard, dev)
+    fns = M.device_split_fns(P.OP_REFINE, q, w, ks, shard_off, pos_base, x["offsets"], ds.k, ds.c, ds.g)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        return M.decode_split_step(fns[0], fns[1], world, fns[2], fns[3])
+
+    for _ in range(max(args.warmup, 0)):
+        step()
+    torch.cuda.synchronize()
+    M.barrier(world)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    tot = 0.0
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+        torch.cuda.synchronize()
+        tot += ev[i][0].elapsed_time(ev[i][1])
+    M.barrier(world)
+    ms = M.max_over_ranks(tot, world, dev) / args.steps
+    if rank == 0:
+        print(json.dumps({"metric": "decode queries/s, prefixes split over GPUs", "value": ds.B * ds.g / (ms / 1e3),
+                          "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                          "ms_per_step": ms, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+                          "dtype": "bf16", "data": "synthetic",
+                          "config": {"workload": ds.name + "_refine_prefix_split", "B": ds.B, "g": ds.g,
+                                     "k": ds.k, "c": ds.c,
+                                     "parallelism": f"every prefix over {world} GPU(s): key shards, all-gather of "
+                                                    "the shard selections, sum of the member scores",
+                                     "l2": "flushed before every step (256 MiB write)"},
+                          "gpu_launches": 6 * args.steps}), flush=True)
+    M.finish(world)
+
+
 def run_reference(args):
     """Reference arm: the CPU oracle as it stands, on bounded samples of the workload."""
     world, rank, _ = dist_env()
@@ -498,6 +561,9 @@ def main():
         return
     if args.split:
         run_split(args)
+        return
+    if args.split_decode:
+        run_split_decode(args)
         return
     import numpy as np
     import torch

@@ -208,8 +208,8 @@ PIVOT_API pivot_status pivot_refine_guarded(const void *q_I, const float *w_I, c
  * host copy of the key offsets (key_offsets_host[0] = 0, non-decreasing,
  * every P_b = key_offsets_host[b+1] - key_offsets_host[b] >= g).  On the
  * tensor-core path (bf16, H = 64, d in {64, 128}) it grows with the batch's
- * keys: 12 bytes per cached key (a 32-bit score key and room for a packed tie
- * entry) plus per-sequence proxies, histograms and the selection. */
+ * keys: 20 bytes per cached key (a 32-bit score key and room for two packed
+ * selection lists) plus per-sequence proxies, histograms and the selection. */
 PIVOT_API size_t pivot_varlen_workspace_size(int op, int B, const int64_t *key_offsets_host, int H, int d, int k, int c,
                                    int g, pivot_dtype dt);
 
@@ -219,8 +219,8 @@ PIVOT_API size_t pivot_varlen_workspace_size(int op, int B, const int64_t *key_o
  * key_offsets[b] .. key_offsets[b+1]-1), key_offsets_dev / key_offsets_host
  * [B+1] (same values, device and host copies) -> indices [B*g,k] of
  * positions local to each sequence.  Asynchronous on `stream`.  Returns
- * PIVOT_ERR_UNSUPPORTED_SHAPE when B * ceil(max P_b / 8192) exceeds 2^31 - 1
- * (the selection grid).  A device-side wait that runs out (PIVOT_ERR_DEVICE_TIMEOUT
+ * PIVOT_ERR_UNSUPPORTED_SHAPE when 8 * B exceeds 2^31 - 1 (the selection
+ * grid: one 8-CTA cluster per sequence).  A device-side wait that runs out (PIVOT_ERR_DEVICE_TIMEOUT
  * from pivot_last_device_status) leaves the outputs undefined; the selection
  * then never writes past its buffers and may also flag PIVOT_ERR_DEVICE_BOUNDS. */
 PIVOT_API pivot_status pivot_reuse_varlen(const void *q, const float *w, const void *k_cache, const int64_t *key_offsets_dev,
@@ -235,6 +235,66 @@ PIVOT_API pivot_status pivot_refine_varlen(const void *q, const float *w, const 
                                  int d, pivot_dtype dt, int k, int c, int g, int32_t *indices, float *scores_opt,
                                  int32_t *cand_opt, float *cand_scores_opt, void *ws, size_t ws_bytes,
                                  pivot_stream_t stream);
+
+/* ---- One long decode prefix split over ranks (one exchange, then one merge).
+ * Eq. (3), (5)-(7) select over a group's whole prefix, and the exact top-n of
+ * a set is inside the union of the exact top-n of its parts.  So rank r of R
+ * holds, for every sequence b, one contiguous shard of its cached keys: rows
+ * shard_offsets[b] .. shard_offsets[b+1]-1 of k_shard (at least one row), which
+ * are the prefix positions pos_base[b] .. of a prefix of P_b = plen_offsets[b+1]
+ * - plen_offsets[b] keys (P_b >= g).  Every rank holds all q [B*g,H,d] and w
+ * [B*g,H] rows.  Steps:
+ *   1. pivot_decode_shard_select (each rank): the shard's exact top-n, n = k+g-1
+ *      (Reuse) or c (Refine), as packed entries [B, n] uint64 (order key << 32 |
+ *      (0xFFFFFFFF - prefix position); 0 pads a shard with fewer keys);
+ *   2. exchange: all-gather of the entries into [R, B, n] (rank order free);
+ *   3. pivot_decode_merge (every rank): Reuse rows [B*g, k], or the candidate set
+ *      C [B, c] (prefix positions) and, for this rank, C in its shard's rows;
+ *   Refine adds:
+ *   4. pivot_decode_shard_rescore (each rank): Eq. (8) member score keys [B*g, c]
+ *      (uint32) of the candidates this rank holds, 0 for the others;
+ *   5. exchange: element-wise sum of the keys over the ranks (every candidate is
+ *      held by exactly one rank);
+ *   6. pivot_decode_rowselect: Eq. (9), indices [B*g, k] of prefix positions.
+ * The results equal pivot_reuse_varlen / pivot_refine_varlen on the whole prefix.
+ * Tensor-core shape only (bf16, H = 64, d in {64, 128}), else
+ * PIVOT_ERR_UNSUPPORTED_SHAPE.  All pointers are device pointers except the
+ * *_host offsets; all calls are asynchronous on `stream`. */
+
+/* Step 1.  ws: pivot_decode_shard_workspace_size bytes (0: unsupported shape or
+ * offsets).  op is PIVOT_OP_REUSE (c ignored) or PIVOT_OP_REFINE. */
+PIVOT_API size_t pivot_decode_shard_workspace_size(int op, int B, const int64_t *shard_offsets_host, int H, int d,
+                                                   int k, int c, int g);
+PIVOT_API pivot_status pivot_decode_shard_select(int op, const void *q, const float *w, const void *k_shard,
+                                                 const int64_t *shard_offsets_dev, const int64_t *shard_offsets_host,
+                                                 const int64_t *pos_base_dev, int B, int H, int d, pivot_dtype dt,
+                                                 int k, int c, int g, uint64_t *entries, void *ws, size_t ws_bytes,
+                                                 pivot_stream_t stream);
+
+/* Step 3.  entries [R, B, n] from step 2.  Reuse writes indices [B*g, k] (and
+ * scores_opt); Refine writes cand [B, c] (and cand_scores_opt), and cand_local_opt
+ * [B, c] (-1 where another rank holds the key) when pos_base_dev and
+ * shard_offsets_dev describe this rank's shard.  ws: the bytes below. */
+PIVOT_API size_t pivot_decode_merge_workspace_size(int op, int R, int B, int k, int c, int g);
+PIVOT_API pivot_status pivot_decode_merge(int op, const uint64_t *entries, int R, const int64_t *plen_offsets_dev,
+                                          const int64_t *plen_offsets_host, int B, int k, int c, int g,
+                                          int32_t *indices, float *scores_opt, int32_t *cand, float *cand_scores_opt,
+                                          const int64_t *pos_base_dev, const int64_t *shard_offsets_dev,
+                                          int32_t *cand_local_opt, void *ws, size_t ws_bytes, pivot_stream_t stream);
+
+/* Step 4.  cand_local [B, c] from step 3; keys [B*g, c]; ws: at least 256 bytes
+ * (step 1's workspace will do). */
+PIVOT_API pivot_status pivot_decode_shard_rescore(const void *q, const float *w, const void *k_shard,
+                                                  const int64_t *shard_offsets_dev, const int64_t *shard_offsets_host,
+                                                  const int64_t *pos_base_dev, const int64_t *plen_offsets_dev, int B,
+                                                  int H, int d, pivot_dtype dt, int k, int c, int g,
+                                                  const int32_t *cand_local, uint32_t *keys, void *ws,
+                                                  size_t ws_bytes, pivot_stream_t stream);
+
+/* Step 6.  keys [B*g, c] summed over the ranks, cand [B, c] from step 3. */
+PIVOT_API pivot_status pivot_decode_rowselect(const uint32_t *keys, const int32_t *cand,
+                                              const int64_t *plen_offsets_dev, int B, int k, int c, int g,
+                                              int32_t *indices, float *scores_opt, pivot_stream_t stream);
 
 /* Synchronises `stream`, then reads the device status word that the last
  * call using workspace `ws` left: PIVOT_OK, PIVOT_ERR_DEVICE_TIMEOUT or

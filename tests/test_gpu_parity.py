@@ -14,6 +14,7 @@ import torch
 import top_token_selection_proxy_b200 as P
 from parity import check_row, summarize
 from top_token_selection_proxy_b200 import inputs
+from top_token_selection_proxy_b200 import multigpu as MG
 
 pytestmark = pytest.mark.gpu
 
@@ -317,12 +318,17 @@ def test_long_128k_refine_reuse_dense_sampled(orc, long_inputs):
     assert not fails, summarize(fails)
 
 
-def _decode_batch_fails(orc, s, x):
-    """Every sequence's C row and Reuse rows, and every Refine row, against the oracle."""
+def _decode_batch_fails(orc, s, x, run=None):
+    """Every sequence's C row and Reuse rows, and every Refine row, against the oracle.  run(q, w,
+    k_cache, offsets) -> (Reuse indices, scores, Refine indices, scores, C, C scores) on the device
+    (default: the batch calls)."""
     off = x["offsets"]
     q, w, kc = dev(x["q"]), dev(x["w"]), dev(x["k"])
-    u_idx, u_sc = P.reuse_varlen(q, w, kc, off, s.k, s.g, scores=True)
-    r_idx, r_sc, r_c, r_cs = P.refine_varlen(q, w, kc, off, s.k, s.c, s.g, scores=True, cand=True)
+    if run is None:
+        u_idx, u_sc = P.reuse_varlen(q, w, kc, off, s.k, s.g, scores=True)
+        r_idx, r_sc, r_c, r_cs = P.refine_varlen(q, w, kc, off, s.k, s.c, s.g, scores=True, cand=True)
+    else:
+        u_idx, u_sc, r_idx, r_sc, r_c, r_cs = run(q, w, kc, off)
     torch.cuda.synchronize()
     u_idx, u_sc, r_idx, r_sc, r_c, r_cs = map(host, (u_idx, u_sc, r_idx, r_sc, r_c, r_cs))
     B, g = s.B, s.g
@@ -389,6 +395,41 @@ def test_decode_duplicate_keys_lowest_index_wins(orc):
         lowest_copies(r_c[b], r_cs[b], b, Pb - 1, f"C_{b}")
         for r in range(s.g):
             lowest_copies(u_idx[b * s.g + r], u_sc[b * s.g + r], b, Pb - s.g + r, f"reuse b={b} r={r}")
+
+
+def _split_run(s, world):
+    """The decode step with every prefix split over `world` ranks, run rank after rank on this GPU."""
+    def run(q, w, kc, off):
+        u_idx, u_sc = MG.decode_split_emulated(P.OP_REUSE, q, w, kc, off, world, s.k, s.c, s.g, scores=True)
+        r_idx, r_sc, r_c, r_cs = MG.decode_split_emulated(P.OP_REFINE, q, w, kc, off, world, s.k, s.c, s.g,
+                                                         scores=True)
+        return u_idx, u_sc, r_idx, r_sc, r_c, r_cs
+    return run
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_decode_prefix_split_small_ragged(orc, world):
+    """One long prefix over ranks (C ABI pivot_decode_shard_select / _merge / _shard_rescore /
+    _rowselect): prefixes of 4 to 3000 keys in 2 or 3 shards, some at or under c and k + g - 1;
+    every C row, Reuse row and Refine row against the oracle."""
+    s = inputs.DecodeSpec("small", B=5, p_lo=4, p_hi=3000, H=64, d=128, k=64, c=128, g=4, seed=21)
+    fails, _ = _decode_batch_fails(orc, s, inputs.make_decode(s), run=_split_run(s, world))
+    assert not fails, summarize(fails)
+
+
+def test_decode_prefix_split_full_batch_matches_one_call(orc):
+    """The full decode batch split over 3 ranks writes exactly the rows of the one-call decode
+    (the same scores and the same exact selections), and its rows pass the oracle."""
+    s = inputs.DECODE
+    x = inputs.make_decode(s)
+    fails, got = _decode_batch_fails(orc, s, x, run=_split_run(s, 3))
+    assert not fails, summarize(fails)
+    q, w, kc = dev(x["q"]), dev(x["w"]), dev(x["k"])
+    off = x["offsets"]
+    u_idx, _ = P.reuse_varlen(q, w, kc, off, s.k, s.g)
+    r_idx, _, r_c, _ = P.refine_varlen(q, w, kc, off, s.k, s.c, s.g, cand=True)
+    for a, b_ in ((got[0], u_idx), (got[2], r_idx), (got[4], r_c)):
+        assert np.array_equal(np.sort(a, axis=1), np.sort(host(b_), axis=1))
 
 
 def test_decode_small_ragged(orc):

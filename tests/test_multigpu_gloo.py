@@ -152,3 +152,148 @@ def test_zigzag_layout():
         assert max(works) <= 1.12 * min(works)
     with pytest.raises(ValueError):
         M.zigzag_chunks(100, 8, 2, 0)
+
+
+# ---------------------------------------------------------------- one long decode prefix over ranks
+
+
+def _split_case():
+    """A small decode batch whose prefixes are split over the ranks (P_b >= 3 for world 3)."""
+    return inputs.DecodeSpec("split", B=3, p_lo=40, p_hi=300, H=4, d=16, k=8, c=24, g=4, seed=83, dtype=inputs.F32)
+
+
+def _oracle_split_fns(x, rank, world, variant, orc):
+    """The split step's four functions on the CPU: the oracle's scores (Eq. 5 for the proxies,
+    Eq. 8 for the members) with the selections written out in numpy.  Entries travel as
+    (score, position) tensors; a candidate's member scores are 0 on the ranks that do not hold it."""
+    import numpy as np
+
+    s = _split_case()
+    off = x["offsets"]
+    B, g, k, c = s.B, s.g, s.k, s.c
+    plen = np.diff(off)
+    mem = [list(range(b * g, b * g + g)) for b in range(B)]
+    qv, wv = orc.proxies(x["q"], x["w"], mem)
+    F = orc.scores_batch(qv, wv, x["k"], plen=plen, key_base=off[:-1])
+    cuts = M.decode_shards(plen, world, rank)
+    n = k + g - 1 if variant == 0 else c
+
+    def top(sc, ix, m):  # the m best by (score desc, position asc)
+        keep = ix >= 0
+        sc, ix = sc[keep], ix[keep]
+        o = np.lexsort((ix, -sc))[:m]
+        return sc[o], ix[o]
+
+    def select_fn():  # this rank's shard of every prefix: its exact top-n
+        sc = np.full((B, n), -np.inf)
+        ix = np.full((B, n), -1, np.int64)
+        for b, (lo, hi) in enumerate(cuts):
+            f, p = top(F[b, lo:hi], np.arange(lo, hi), n)
+            sc[b, :f.size], ix[b, :p.size] = f, p
+        return torch.from_numpy(sc), torch.from_numpy(ix)
+
+    def merge_fn(gathered):
+        sc, ix = gathered[0].numpy(), gathered[1].numpy()  # [R, B, n]
+        if variant == 0:  # Reuse rows: member t keeps the k best of the selection's entries <= t
+            rows = []
+            for b in range(B):
+                f, p = top(sc[:, b].ravel(), ix[:, b].ravel(), min(n, plen[b]))
+                for r in range(g):
+                    e = p <= plen[b] - g + r
+                    rows.append(sorted(top(f[e], p[e], k)[1].tolist()))
+            return rows
+        C = np.full((B, c), -1, np.int64)
+        CL = np.full((B, c), -1, np.int64)
+        for b in range(B):
+            p = top(sc[:, b].ravel(), ix[:, b].ravel(), min(c, plen[b]))[1]
+            C[b, :p.size] = p
+            lo, hi = cuts[b]
+            held = (p >= lo) & (p < hi)
+            CL[b, :p.size][held] = p[held] - lo
+        return C, CL
+
+    def rescore_fn(merged):
+        C, CL = merged
+        qm, wm = orc.query_rows(x["q"], x["w"], list(range(B * g)))
+        key_rows = np.full((B * g, c), -1, np.int64)
+        for b in range(B):
+            held = CL[b] >= 0
+            for r in range(g):
+                key_rows[b * g + r, held] = C[b, held]
+        Ms = orc.scores_batch(qm, wm, x["k"], key_rows=key_rows, key_base=np.repeat(off[:-1], g))
+        held = key_rows >= 0
+        return torch.from_numpy(np.where(held, Ms, 0.0)), torch.from_numpy(held.astype(np.int64))
+
+    def rowselect_fn(summed, merged):
+        C = merged[0]
+        Ms, cnt = summed[0].numpy(), summed[1].numpy()
+        rows, once = [], True
+        for b in range(B):
+            valid = C[b] >= 0
+            once &= bool((cnt[b * g:(b + 1) * g][:, valid] == 1).all())
+            for r in range(g):
+                e = valid & (C[b] <= plen[b] - g + r)
+                rows.append(sorted(top(Ms[b * g + r][e], C[b][e], k)[1].tolist()))
+        return rows, once
+
+    if variant == 0:
+        return select_fn, merge_fn, None, None
+    return select_fn, merge_fn, rescore_fn, rowselect_fn
+
+
+def _decode_split_rank(rank: int, world: int, port: int, outdir: str) -> None:
+    from oracle import oracle as orc
+
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port), "WORLD_SIZE": str(world),
+                       "RANK": str(rank), "LOCAL_RANK": str(rank)})
+    M.init("gloo", world, timeout_s=60.0)
+    x = inputs.make_decode(_split_case())  # every rank draws the same batch and keeps its shards' keys
+    out = {}
+    for variant in (0, 1):
+        sel, merge, rescore, rowsel = _oracle_split_fns(x, rank, world, variant, orc)
+        res = M.decode_split_step(sel, merge, world, rescore, rowsel)
+        out[variant] = {"rows": res} if variant == 0 else {"rows": res[0], "held_once": res[1]}
+    with open(os.path.join(outdir, f"ds{rank}.json"), "w") as f:
+        json.dump(out, f)
+    M.finish(world)
+
+
+@pytest.mark.timeout(300)
+@pytest.mark.parametrize("world", [2, 3])
+def test_decode_prefix_split_over_ranks(tmp_path, orc, world):
+    """One all-gather of the shards' exact top-n and a merge give every rank the Reuse rows of the
+    whole prefixes; Refine's per-rank re-scoring of held candidates and one element-wise sum give
+    its rows.  Both equal the oracle's decode on the unsplit batch."""
+    import numpy as np
+
+    mp.spawn(_decode_split_rank, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    res = [json.load(open(tmp_path / f"ds{r}.json")) for r in range(world)]
+    s = _split_case()
+    x = inputs.make_decode(s)
+    for variant in (0, 1):
+        idx = orc.decode(x["q"], x["w"], x["k"], x["offsets"], s.k, s.c, s.g, variant)[0]
+        want = [sorted(int(v) for v in row if v >= 0) for row in idx]
+        for r in res:
+            assert r[str(variant)]["rows"] == want, f"variant {variant}: split rows differ from the whole prefix"
+            if variant == 1:
+                assert r["1"]["held_once"], "every candidate is held by exactly one rank"
+
+
+def test_decode_shards_partition_every_prefix():
+    import numpy as np
+
+    plen = [3, 7, 100, 4097]
+    for world in (1, 2, 3):
+        cover = [np.zeros(P, int) for P in plen]
+        for rank in range(world):
+            for b, (lo, hi) in enumerate(M.decode_shards(plen, world, rank)):
+                assert hi - lo >= 1
+                cover[b][lo:hi] += 1
+        assert all((cv == 1).all() for cv in cover)
+    with pytest.raises(ValueError):
+        M.decode_shards([2], 3, 0)
+    k = np.arange(20 * 2).reshape(20, 2)
+    off = np.array([0, 8, 20])
+    ks, so, pb = M.shard_of(k, off, 2, 1)
+    assert so.tolist() == [0, 4, 10] and pb.tolist() == [4, 6]
+    assert np.array_equal(ks, np.concatenate([k[4:8], k[14:20]]))

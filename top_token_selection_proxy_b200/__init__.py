@@ -44,6 +44,9 @@ EXPORTS = (
     "pivot_reuse_noalloc", "pivot_guardrail_dense", "pivot_reuse_guarded", "pivot_refine_guarded",
     "pivot_reuse_agg", "pivot_refine_agg", "pivot_indexer_dense_range", "pivot_reuse_range",
     "pivot_refine_range", "pivot_refine_host_workspace_size", "pivot_refine_host",
+    "pivot_decode_shard_workspace_size", "pivot_decode_shard_select", "pivot_decode_merge_workspace_size",
+    "pivot_decode_merge",
+    "pivot_decode_shard_rescore", "pivot_decode_rowselect",
 )
 
 # proxy aggregation (PIVOT paper, Ablation Studies, Proxy aggregation, Table 2)
@@ -90,6 +93,17 @@ def lib() -> ctypes.CDLL:
         L.pivot_guardrail_dense.restype = I
         L.pivot_reuse_guarded.argtypes = [P, P, P, I64, I, I, I, I, I, P, P, P, SZ, P, P]
         L.pivot_refine_guarded.argtypes = [P, P, P, I64, I, I, I, I, I, I, P, P, P, P, P, SZ, P, P]
+        L.pivot_decode_shard_workspace_size.argtypes = [I, I, P, I, I, I, I, I]
+        L.pivot_decode_shard_workspace_size.restype = SZ
+        L.pivot_decode_shard_select.argtypes = [I, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, SZ, P]
+        L.pivot_decode_merge_workspace_size.argtypes = [I, I, I, I, I, I]
+        L.pivot_decode_merge_workspace_size.restype = SZ
+        L.pivot_decode_merge.argtypes = [I, P, I, P, P, I, I, I, I, P, P, P, P, P, P, P, P, SZ, P]
+        L.pivot_decode_shard_rescore.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, P, P, SZ, P]
+        L.pivot_decode_rowselect.argtypes = [P, P, P, I, I, I, I, P, P, P]
+        for f in ("pivot_decode_shard_select", "pivot_decode_merge", "pivot_decode_shard_rescore",
+                  "pivot_decode_rowselect"):
+            getattr(L, f).restype = I
         for f in ("pivot_indexer_dense", "pivot_reuse", "pivot_refine", "pivot_reuse_varlen",
                   "pivot_refine_varlen", "pivot_last_device_status", "pivot_reuse_guarded",
                   "pivot_refine_guarded", "pivot_reuse_agg", "pivot_refine_agg", "pivot_indexer_dense_range",
@@ -432,6 +446,95 @@ def refine_varlen(q, w, k_cache, offsets, topk: int, c: int, g: int, *, scores: 
     return idx, sc, cd, cs
 
 
+# ---------------------------------------------------------------- one long decode prefix over ranks
+# The C ABI's four steps (pivot_decode_shard_select, _merge, _shard_rescore, _rowselect); the
+# exchanges between them (an all-gather of the shard entries, an element-wise sum of the member
+# score keys) belong to the caller: multigpu.decode_split_step runs them over torch.distributed.
+
+
+def _offsets_pair(offsets, device, stream):
+    h = torch.as_tensor(offsets, dtype=torch.int64).cpu().contiguous()
+    return h, _offsets_dev(h, device, stream)
+
+
+def decode_shard_select(op: int, q, w, k_shard, shard_offsets, pos_base, topk: int, c: int, g: int, *,
+                        ws: Optional[Workspace] = None, stream=None):
+    """Step 1: this rank's key shard of every sequence -> its exact top-n (n = k+g-1 for
+    OP_REUSE, c for OP_REFINE) as packed int64 entries [B, n] with prefix positions (0 pads)."""
+    _need_cuda(q, w, k_shard)
+    sh, sd = _offsets_pair(shard_offsets, q.device, stream)
+    pb = torch.as_tensor(pos_base, dtype=torch.int64).to(q.device)
+    B = sh.numel() - 1
+    H, d = q.shape[1], q.shape[2]
+    n = topk + g - 1 if op == OP_REUSE else c
+    ent = torch.empty((B, n), dtype=torch.int64, device=q.device)
+    nbytes = int(lib().pivot_decode_shard_workspace_size(op, B, _ptr(sh), H, d, topk, c, g))
+    if nbytes == 0:
+        raise PivotError(1, "decode_shard_select", "unsupported shape or offsets")
+    W = _ws_for(ws, q.device).get(nbytes)
+    _check(lib().pivot_decode_shard_select(op, _ptr(q), _ptr(w), _ptr(k_shard), _ptr(sd), _ptr(sh), _ptr(pb), B, H,
+                                           d, _dt(q), topk, c, g, _ptr(ent), _ptr(W), W.numel(), _stream(stream)),
+           "pivot_decode_shard_select")
+    return ent
+
+
+def decode_merge(op: int, entries, plen_offsets, topk: int, c: int, g: int, *, shard_offsets=None, pos_base=None,
+                 scores: bool = False, ws: Optional[Workspace] = None, stream=None):
+    """Step 3: entries [R, B, n] of all ranks -> OP_REUSE: (indices [B*g, k], scores|None);
+    OP_REFINE: (C [B, c], C scores|None, C in this rank's shard rows [B, c] | None)."""
+    _need_cuda(entries)
+    R, B, n = entries.shape
+    ph, pd = _offsets_pair(plen_offsets, entries.device, stream)
+    dev = entries.device
+    local = shard_offsets is not None
+    sd = _offsets_pair(shard_offsets, dev, stream)[1] if local else None
+    pb = torch.as_tensor(pos_base, dtype=torch.int64).to(dev) if local else None
+    nbytes = int(lib().pivot_decode_merge_workspace_size(op, R, B, topk, c, g))
+    W = _ws_for(ws, dev).get(nbytes)
+    idx = sc = cand = csc = cl = None
+    if op == OP_REUSE:
+        idx = torch.empty((B * g, topk), dtype=torch.int32, device=dev)
+        sc = torch.empty((B * g, topk), dtype=torch.float32, device=dev) if scores else None
+    else:
+        cand = torch.empty((B, c), dtype=torch.int32, device=dev)
+        csc = torch.empty((B, c), dtype=torch.float32, device=dev) if scores else None
+        cl = torch.empty((B, c), dtype=torch.int32, device=dev) if local else None
+    _check(lib().pivot_decode_merge(op, _ptr(entries), R, _ptr(pd), _ptr(ph), B, topk, c, g, _ptr(idx), _ptr(sc),
+                                    _ptr(cand), _ptr(csc), _ptr(pb), _ptr(sd), _ptr(cl), _ptr(W), W.numel(),
+                                    _stream(stream)), "pivot_decode_merge")
+    return (idx, sc) if op == OP_REUSE else (cand, csc, cl)
+
+
+def decode_shard_rescore(q, w, k_shard, shard_offsets, pos_base, plen_offsets, cand_local, topk: int, c: int,
+                         g: int, *, ws: Optional[Workspace] = None, stream=None):
+    """Step 4: Eq. (8) member score keys [B*g, c] (int32 bits of the uint32 keys) of the candidates
+    this rank's shard holds; 0 for the others."""
+    _need_cuda(q, w, k_shard, cand_local)
+    sh, sd = _offsets_pair(shard_offsets, q.device, stream)
+    pd = _offsets_pair(plen_offsets, q.device, stream)[1]
+    pb = torch.as_tensor(pos_base, dtype=torch.int64).to(q.device)
+    B = sh.numel() - 1
+    H, d = q.shape[1], q.shape[2]
+    keys = torch.empty((B * g, c), dtype=torch.int32, device=q.device)
+    W = _ws_for(ws, q.device).get(256)
+    _check(lib().pivot_decode_shard_rescore(_ptr(q), _ptr(w), _ptr(k_shard), _ptr(sd), _ptr(sh), _ptr(pb), _ptr(pd),
+                                            B, H, d, _dt(q), topk, c, g, _ptr(cand_local), _ptr(keys), _ptr(W),
+                                            W.numel(), _stream(stream)), "pivot_decode_shard_rescore")
+    return keys
+
+
+def decode_rowselect(keys, cand, plen_offsets, topk: int, c: int, g: int, *, scores: bool = False, stream=None):
+    """Step 6: Eq. (9) on the rank-summed keys -> (indices [B*g, k], scores|None)."""
+    _need_cuda(keys, cand)
+    B = cand.shape[0]
+    pd = _offsets_pair(plen_offsets, keys.device, stream)[1]
+    idx = torch.empty((B * g, topk), dtype=torch.int32, device=keys.device)
+    sc = torch.empty((B * g, topk), dtype=torch.float32, device=keys.device) if scores else None
+    _check(lib().pivot_decode_rowselect(_ptr(keys), _ptr(cand), _ptr(pd), B, topk, c, g, _ptr(idx), _ptr(sc),
+                                        _stream(stream)), "pivot_decode_rowselect")
+    return idx, sc
+
+
 def last_device_status(ws: Workspace, stream=None) -> int:
     """Synchronise the stream and return the device status code of the last call on ``ws``."""
     return int(lib().pivot_last_device_status(_ptr(ws.buf), _stream(stream)))
@@ -478,6 +581,7 @@ __all__ = [
     "guardrail_dense", "reuse_guarded", "refine_guarded", "AGGREGATION",
     "indexer_dense_range", "reuse_range", "refine_range",
     "group_chunks", "refine_host", "refine_streamed",
+    "decode_shard_select", "decode_merge", "decode_shard_rescore", "decode_rowselect",
     "set_device_timeout_ns", "set_debug_flags", "KernelTimer", "OP_DENSE", "OP_REUSE", "OP_REFINE", "BF16", "F32",
     "STATUS",
 ]

@@ -523,6 +523,38 @@ pivot_status run_decode(int op, const void* q, const float* w, const void* kc, c
   return PIVOT_OK;
 }
 
+// ---------------------------------------------------------------- decode split (one long prefix over ranks)
+// Shard offsets: like key offsets, but a shard may hold any number >= 1 of a sequence's keys.
+pivot_status check_shard_offsets(int B, const int64_t* off) {
+  if (B <= 0 || !off || off[0] != 0) return PIVOT_ERR_INVALID_ARG;
+  for (int b = 0; b < B; ++b)
+    if (off[b + 1] - off[b] < 1) return PIVOT_ERR_INVALID_ARG;
+  if (off[B] >= (int64_t)0x7FFFFFF0) return PIVOT_ERR_UNSUPPORTED_SHAPE;
+  return PIVOT_OK;
+}
+
+size_t merge_ws_bytes(int op, int R, int B, int k, int c, int g) {
+  const size_t n_sel = (size_t)sel_size(op, k, c, g);
+  return kHdr + align_up((size_t)B * R * n_sel * 8, 256) + align_up((size_t)B * n_sel * 8, 256);
+}
+
+DecodeArgs shard_args(const DecodeWs& W, int op, const void* q, const float* w, const int64_t* off_dev, int B, int H,
+                      int d, int k, int c, int g) {
+  DecodeArgs a = W.d;
+  a.q = reinterpret_cast<const uint16_t*>(q);
+  a.w = w;
+  a.key_off = off_dev;
+  a.B = B;
+  a.H = H;
+  a.D = d;
+  a.g = g;
+  a.n_sel = sel_size(op, k, c, g);
+  a.topk = k;
+  a.status = W.status;
+  a.timeout_ns = g_timeout_ns;
+  return a;
+}
+
 }  // namespace
 
 // Library-internal hooks for the other host files (hidden: not part of the C ABI).
@@ -587,6 +619,169 @@ pivot_status pivot_refine_varlen(const void* q, const float* w, const void* k_ca
   return run_decode(PIVOT_OP_REFINE, q, w, k_cache, key_offsets_dev, key_offsets_host, B, H, d, dt, k, c, g,
                     indices, scores_opt, cand_opt, cand_scores_opt, ws, ws_bytes,
                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t pivot_decode_shard_workspace_size(int op, int B, const int64_t* shard_offsets_host, int H, int d, int k, int c,
+                                         int g) {
+  if (op != PIVOT_OP_REUSE && op != PIVOT_OP_REFINE) return 0;
+  if (op == PIVOT_OP_REUSE) c = k;
+  if (check_common(1, H, d, PIVOT_BF16, k, c, g, op) != PIVOT_OK || !tc_shape(H, d, PIVOT_BF16) ||
+      check_shard_offsets(B, shard_offsets_host) != PIVOT_OK)
+    return 0;
+  return carve_decode(nullptr, op, B, shard_offsets_host, H, d, k, c, g, PIVOT_BF16, false).bytes;
+}
+
+pivot_status pivot_decode_shard_select(int op, const void* q, const float* w, const void* k_shard,
+                                       const int64_t* shard_offsets_dev, const int64_t* shard_offsets_host,
+                                       const int64_t* pos_base_dev, int B, int H, int d, pivot_dtype dt, int k, int c,
+                                       int g, uint64_t* entries, void* ws, size_t ws_bytes, pivot_stream_t stream) {
+  g_cuda_err[0] = 0;
+  if (op != PIVOT_OP_REUSE && op != PIVOT_OP_REFINE) return PIVOT_ERR_INVALID_ARG;
+  if (op == PIVOT_OP_REUSE) c = k;
+  pivot_status st = check_common(1, H, d, dt, k, c, g, op);
+  if (st != PIVOT_OK) return st;
+  if ((st = check_shard_offsets(B, shard_offsets_host)) != PIVOT_OK) return st;
+  if (!q || !w || !k_shard || !shard_offsets_dev || !pos_base_dev || !entries || !ws) return PIVOT_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_shard) || !aligned16(ws)) return PIVOT_ERR_INVALID_ARG;
+  if (!tc_shape(H, d, dt)) return PIVOT_ERR_UNSUPPORTED_SHAPE;
+  const DecodeWs need = carve_decode(nullptr, op, B, shard_offsets_host, H, d, k, c, g, dt, false);
+  if (ws_bytes < need.bytes) return PIVOT_ERR_WORKSPACE_TOO_SMALL;
+  const DecodeWs W = carve_decode(ws, op, B, shard_offsets_host, H, d, k, c, g, dt, false);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(ws, 0, kHdr, s);
+  if (e != cudaSuccess) return cuda_fail(e, "memset");
+  DecodeArgs a = shard_args(W, op, q, w, shard_offsets_dev, B, H, d, k, c, g);
+  a.mode = EMIT_ENTRIES;
+  a.pos_base = pos_base_dev;
+  a.entries = entries;
+  CUtensorMap kmap, pmap;
+  if (!make_kmap(&kmap, k_shard, shard_offsets_host[B], d, 128) || !make_kmap(&pmap, a.proxy, (int64_t)B * H, d, H))
+    return cuda_fail(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+  if ((e = launch_decode_scan(a, &kmap, &pmap, W.scan_grid, s)) != cudaSuccess) return cuda_fail(e, "decode scan");
+  if ((e = launch_decode_select(a, s)) != cudaSuccess) return cuda_fail(e, "decode selection");
+  return PIVOT_OK;
+}
+
+size_t pivot_decode_merge_workspace_size(int op, int R, int B, int k, int c, int g) {
+  if ((op != PIVOT_OP_REUSE && op != PIVOT_OP_REFINE) || R < 1 || B < 1 || k < 1 || g < 1) return 0;
+  if (op == PIVOT_OP_REUSE) c = k;
+  if (c < k) return 0;
+  return merge_ws_bytes(op, R, B, k, c, g);
+}
+
+pivot_status pivot_decode_merge(int op, const uint64_t* entries, int R, const int64_t* plen_offsets_dev,
+                                const int64_t* plen_offsets_host, int B, int k, int c, int g, int32_t* indices,
+                                float* scores_opt, int32_t* cand, float* cand_scores_opt,
+                                const int64_t* pos_base_dev, const int64_t* shard_offsets_dev,
+                                int32_t* cand_local_opt, void* ws, size_t ws_bytes, pivot_stream_t stream) {
+  g_cuda_err[0] = 0;
+  if (op != PIVOT_OP_REUSE && op != PIVOT_OP_REFINE) return PIVOT_ERR_INVALID_ARG;
+  if (op == PIVOT_OP_REUSE) c = k;
+  if (R < 1 || k < 1 || c < k || g < 1 || g > 16) return PIVOT_ERR_INVALID_ARG;
+  pivot_status st = check_offsets(B, plen_offsets_host, g);
+  if (st != PIVOT_OK) return st;
+  if (!entries || !plen_offsets_dev || !ws || !aligned16(ws)) return PIVOT_ERR_INVALID_ARG;
+  if (op == PIVOT_OP_REUSE ? !indices : !cand) return PIVOT_ERR_INVALID_ARG;
+  if (cand_local_opt && (!pos_base_dev || !shard_offsets_dev)) return PIVOT_ERR_INVALID_ARG;
+  if ((int64_t)R * sel_size(op, k, c, g) >= (int64_t)0x7FFFFFF0) return PIVOT_ERR_UNSUPPORTED_SHAPE;
+  if (ws_bytes < merge_ws_bytes(op, R, B, k, c, g)) return PIVOT_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(ws, 0, kHdr, s);
+  if (e != cudaSuccess) return cuda_fail(e, "memset");
+  Carve cv{reinterpret_cast<char*>(ws)};
+  cv.take<char>(kHdr);
+  MergeArgs m{};
+  m.entries = entries;
+  m.R = R;
+  m.B = B;
+  m.g = g;
+  m.n_sel = sel_size(op, k, c, g);
+  m.topk = k;
+  m.mode = op == PIVOT_OP_REUSE ? EMIT_REUSE : EMIT_CAND;
+  m.plen_off = plen_offsets_dev;
+  m.gather = cv.take<uint64_t>((size_t)B * R * m.n_sel);
+  m.sel = cv.take<uint64_t>((size_t)B * m.n_sel);
+  m.out_idx = indices;
+  m.out_scores = scores_opt;
+  m.cand = cand;
+  m.cand_scores = cand_scores_opt;
+  m.pos_base = pos_base_dev;
+  m.shard_off = shard_offsets_dev;
+  m.cand_local = cand_local_opt;
+  e = launch_decode_merge(m, s);
+  return e == cudaSuccess ? PIVOT_OK : cuda_fail(e, "decode merge");
+}
+
+pivot_status pivot_decode_shard_rescore(const void* q, const float* w, const void* k_shard,
+                                        const int64_t* shard_offsets_dev, const int64_t* shard_offsets_host,
+                                        const int64_t* pos_base_dev, const int64_t* plen_offsets_dev, int B, int H,
+                                        int d, pivot_dtype dt, int k, int c, int g, const int32_t* cand_local,
+                                        uint32_t* keys, void* ws, size_t ws_bytes, pivot_stream_t stream) {
+  g_cuda_err[0] = 0;
+  pivot_status st = check_common(1, H, d, dt, k, c, g, PIVOT_OP_REFINE);
+  if (st != PIVOT_OK) return st;
+  if ((st = check_shard_offsets(B, shard_offsets_host)) != PIVOT_OK) return st;
+  if (!q || !w || !k_shard || !shard_offsets_dev || !pos_base_dev || !plen_offsets_dev || !cand_local || !keys || !ws)
+    return PIVOT_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_shard) || !aligned16(ws)) return PIVOT_ERR_INVALID_ARG;
+  if (!tc_shape(H, d, dt)) return PIVOT_ERR_UNSUPPORTED_SHAPE;
+  if (ws_bytes < kHdr) return PIVOT_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(ws, 0, kHdr, s);
+  if (e != cudaSuccess) return cuda_fail(e, "memset");
+  RefineArgs r{};
+  r.q = reinterpret_cast<const uint16_t*>(q);
+  r.w = w;
+  r.k = reinterpret_cast<const uint16_t*>(k_shard);
+  r.L = 0;
+  r.H = H;
+  r.D = d;
+  r.g = g;
+  r.c = c;
+  r.topk = k;
+  r.mc = 512 / H;
+  r.n_groups = B;
+  {
+    const int chunks = (g + r.mc - 1) / r.mc, tiles = (c + 127) / 128;
+    r.cparts = std::max(1, std::min(tiles, num_sms() / std::max(1, B * chunks)));
+    r.n_items = B * chunks * r.cparts;
+  }
+  r.cand = cand_local;
+  r.key_off = shard_offsets_dev;
+  r.pos_base = pos_base_dev;
+  r.plen_off = plen_offsets_dev;
+  r.keys = keys;
+  char* hdr = reinterpret_cast<char*>(ws);
+  r.counter = reinterpret_cast<unsigned*>(hdr + kCounterOff) + 1;
+  r.status = reinterpret_cast<int*>(hdr + kStatusOff);
+  r.timeout_ns = g_timeout_ns;
+  CUtensorMap gmap, qmap;
+  if (!make_kmap(&gmap, k_shard, shard_offsets_host[B], d, 1) || !make_kmap(&qmap, q, (int64_t)B * g * H, d, 256))
+    return cuda_fail(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+  e = launch_refine(r, &gmap, &qmap, std::min(num_sms(), r.n_items), s);
+  return e == cudaSuccess ? PIVOT_OK : cuda_fail(e, "refine kernel");
+}
+
+pivot_status pivot_decode_rowselect(const uint32_t* keys, const int32_t* cand, const int64_t* plen_offsets_dev,
+                                    int B, int k, int c, int g, int32_t* indices, float* scores_opt,
+                                    pivot_stream_t stream) {
+  g_cuda_err[0] = 0;
+  if (!keys || !cand || !plen_offsets_dev || !indices || B < 1 || k < 1 || c < k || g < 1)
+    return PIVOT_ERR_INVALID_ARG;
+  RowSelArgs rs{};
+  rs.keys = keys;
+  rs.cand = cand;
+  rs.n_rows = (int64_t)B * g;
+  rs.L = 0;
+  rs.key_off = plen_offsets_dev;
+  rs.g = g;
+  rs.c = c;
+  rs.topk = k;
+  rs.out_idx = indices;
+  rs.out_scores = scores_opt;
+  const cudaError_t e =
+      launch_rowselect(rs, (int)std::min<int64_t>(8 * num_sms(), rs.n_rows), reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PIVOT_OK : cuda_fail(e, "rowselect kernel");
 }
 
 pivot_status pivot_last_device_status(const void* ws, pivot_stream_t stream) {

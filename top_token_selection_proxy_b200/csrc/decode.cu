@@ -684,8 +684,59 @@ __global__ void __launch_bounds__(kSelClThreads) dselect_cluster_kernel(const De
   if (a.mode == EMIT_CAND) {
     emit_row<NT>(buf, m, 0xFFFFFFFFu, 0ull, a.cand + (int64_t)b * a.n_sel,
                  a.cand_scores ? a.cand_scores + (int64_t)b * a.n_sel : nullptr, (uint32_t)a.n_sel, sm.S, G);
-  } else {
+  } else if (a.mode == EMIT_REUSE) {
     emit_reuse<NT>(buf, m, a.topk, P - a.g, a.g, (int64_t)b * a.g, a.out_idx, a.out_scores, sm.S, sm.bot, G);
+  } else {  // EMIT_ENTRIES: this key shard's selection, positions made global, 0 pads
+    const uint32_t base = a.pos_base ? (uint32_t)a.pos_base[b] : 0u;
+    uint64_t* e = a.entries + (int64_t)b * a.n_sel;
+    for (uint32_t i = tid; i < (uint32_t)a.n_sel; i += NT)
+      e[i] = i < m ? pack_entry((uint32_t)(buf[i] >> 32), entry_idx(buf[i]) + base) : 0ull;
+  }
+}
+
+// ------------------------------------------------------------------ decode split: merge
+// One CTA per sequence: the ranks' shard selections (each the exact top-n of its keys, so
+// their union holds the exact top-n of the whole prefix) are gathered, the top n = min(n_sel,
+// P_b) are selected by the full (score, index) order, and the candidate row (Refine) or the
+// g member rows (Reuse, members at positions P_b - g .. P_b - 1) are written.
+__global__ void __launch_bounds__(512) dmerge_kernel(const MergeArgs a) {
+  constexpr int NT = 512;
+  __shared__ SelSmem S;
+  __shared__ uint32_t hist11[kHist11Words];
+  __shared__ uint64_t bot[16];
+  const Group<NT> G{(int)threadIdx.x, 0};
+  for (int b = blockIdx.x; b < a.B; b += gridDim.x) {
+    const int64_t P = a.plen_off[b + 1] - a.plen_off[b];
+    const uint32_t need = (uint32_t)min64(a.n_sel, P);
+    const uint32_t n = (uint32_t)a.R * (uint32_t)a.n_sel;
+    uint64_t* buf = a.gather + (int64_t)b * n;
+    for (int r = 0; r < a.R; ++r) {  // (n_sel may be odd: plain 8-byte copies)
+      const uint64_t* src = a.entries + ((int64_t)r * a.B + b) * a.n_sel;
+      for (int i = G.tid; i < a.n_sel; i += NT) buf[(int64_t)r * a.n_sel + i] = src[i];
+    }
+    G.sync();
+    // the need-th largest; zero pads never pass (a threshold of 0 means "every entry")
+    uint64_t th = radix11_threshold<NT>(buf, n, need, need, hist11, S, G);
+    if (th == 0ull) th = 1ull;
+    uint64_t* sel = a.sel + (int64_t)b * a.n_sel;
+    const uint32_t m = compact_ge<NT>(buf, sel, n, th, S, G);
+    G.sync();
+    if (a.mode == EMIT_CAND) {
+      int32_t* row = a.cand + (int64_t)b * a.n_sel;
+      emit_row<NT>(sel, m, 0xFFFFFFFFu, 0ull, row, a.cand_scores ? a.cand_scores + (int64_t)b * a.n_sel : nullptr,
+                   (uint32_t)a.n_sel, S, G);
+      G.sync();
+      if (a.cand_local) {  // C in the rows of this rank's key shard, -1 where another rank holds the key
+        const int64_t base = a.pos_base[b], len = a.shard_off[b + 1] - a.shard_off[b];
+        for (int i = G.tid; i < a.n_sel; i += NT) {
+          const int64_t v = row[i];
+          a.cand_local[(int64_t)b * a.n_sel + i] = (v >= base && v < base + len) ? (int32_t)(v - base) : -1;
+        }
+      }
+    } else {
+      emit_reuse<NT>(sel, m, a.topk, P - a.g, a.g, (int64_t)b * a.g, a.out_idx, a.out_scores, S, bot, G);
+    }
+    G.sync();
   }
 }
 
@@ -714,6 +765,11 @@ cudaError_t launch_decode_scan(const DecodeArgs& a, const CUtensorMap* kmap, con
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     k<<<scan_grid, DScanCfg<64>::THREADS, smem, s>>>(*kmap, *pmap, a);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_merge(const MergeArgs& a, cudaStream_t s) {
+  dmerge_kernel<<<a.B < 1184 ? a.B : 1184, 512, 0, s>>>(a);
   return cudaGetLastError();
 }
 

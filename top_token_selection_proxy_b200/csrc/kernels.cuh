@@ -13,7 +13,8 @@ namespace pivot {
 enum EmitMode : int {
   EMIT_DENSE = 0,   // g == 1: row t = top-k of the query's own scores (Eq. 1)
   EMIT_REUSE = 1,   // Eq. 6: each member t takes the proxy top-k under s <= t
-  EMIT_CAND = 2     // Eq. 7: write the proxy top-c candidate set C_i
+  EMIT_CAND = 2,    // Eq. 7: write the proxy top-c candidate set C_i
+  EMIT_ENTRIES = 3  // decode split: a key shard's exact top-n as packed entries (global positions)
 };
 
 // Device status word bits (written with atomicOr, read by pivot_last_device_status).
@@ -62,6 +63,8 @@ struct RefineArgs {
   int n_items;           // n_groups * ceil(g / mc) * cparts
   const int32_t* cand;   // [n_groups, c]  (-1 padded)
   const int64_t* key_off;  // decode: [B+1]; null for prefill
+  const int64_t* pos_base;  // decode, optional: [B] global position of each sequence's first key row
+  const int64_t* plen_off;  // decode, optional: [B+1] offsets giving the full prefix lengths (members' positions)
   uint32_t* keys;        // [rows, c] member score keys (0 = not eligible)
   unsigned int* counter;
   int* status;
@@ -117,8 +120,9 @@ struct DecodeArgs {
   int B, H, D, g;
   int n_sel;                // k+g-1 (Reuse) or c (Refine)
   int topk;
-  int mode;                 // EMIT_CAND or EMIT_REUSE
+  int mode;                 // EMIT_CAND, EMIT_REUSE or EMIT_ENTRIES
   int64_t n_sets;           // sum over b of ceil(P_b / kDecodeSetKeys)
+  const int64_t* pos_base;  // EMIT_ENTRIES: [B] global position of each sequence's first key here
   // workspace
   uint16_t* proxy;          // [B*H, D] bf16 bits: the pooled proxies (Eq. 4)
   float* wbar;              // [B, kWbarStride] w-bar, permuted for the epilogue
@@ -133,8 +137,25 @@ struct DecodeArgs {
   float* cand_scores;       // or null
   int32_t* out_idx;         // [B*g, topk] (Reuse)
   float* out_scores;        // or null
+  uint64_t* entries;        // [B, n_sel] (EMIT_ENTRIES; 0 pads)
   int* status;
   uint64_t timeout_ns;
+};
+
+// Decode split: the top-n of the ranks' exchanged shard entries, then the emit.
+struct MergeArgs {
+  const uint64_t* entries;  // [R, B, n_sel] packed entries with global positions (0 pads)
+  int R, B, g, n_sel, topk, mode;  // mode: EMIT_REUSE or EMIT_CAND
+  const int64_t* plen_off;  // [B+1] offsets whose differences are the full prefix lengths P_b
+  uint64_t* gather;         // workspace [B, R * n_sel]
+  uint64_t* sel;            // workspace [B, n_sel]
+  int32_t* out_idx;         // Reuse: [B*g, topk]
+  float* out_scores;
+  int32_t* cand;            // Refine: [B, n_sel] global positions
+  float* cand_scores;
+  const int64_t* pos_base;  // optional: this rank's shard ([B] first global position, shard_off [B+1])
+  const int64_t* shard_off;
+  int32_t* cand_local;      // optional: [B, n_sel] C in this rank's shard rows (-1: held elsewhere)
 };
 // launchers (return cudaError_t of the launch)
 cudaError_t launch_scan(const ScanArgs& a, const CUtensorMap* kmap, int grid, cudaStream_t s);
@@ -149,6 +170,7 @@ cudaError_t launch_rowselect(const RowSelArgs& a, int grid, cudaStream_t s);
 cudaError_t launch_decode_scan(const DecodeArgs& a, const CUtensorMap* kmap, const CUtensorMap* pmap, int scan_grid,
                                cudaStream_t s);
 cudaError_t launch_decode_select(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_decode_merge(const MergeArgs& a, cudaStream_t s);
 size_t decode_scan_smem_bytes(int D);
 
 // host-side library state shared by the entry-point files (defined in api.cu)

@@ -152,7 +152,9 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(const __grid_constant__ 
           const int r0 = mc * C::MC;
           int64_t P, nmem_g;
           if (decode) {
-            P = a.key_off[grp + 1] - a.key_off[grp];
+            // a key shard (pos_base / plen_off): the candidate ids are rows of this shard, the
+            // members' positions and the candidate count follow the full prefix
+            P = a.plen_off ? a.plen_off[grp + 1] - a.plen_off[grp] : a.key_off[grp + 1] - a.key_off[grp];
             nmem_g = a.g;
             I.key_base = a.key_off[grp];
             I.qrow0 = grp * a.g + r0;
@@ -438,6 +440,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(const __grid_constant__ 
       if (named_bar_or(2, C::NEPI, !valid || T.abort_flag != 0)) break;
       const int32_t* cand = a.cand + I.grp * (int64_t)a.c;
       const int ntiles = nm > 0 ? I.ntiles : 0, nhalf = I.nhalf, tile0 = I.tile0, n_c = I.n_c;
+      const int64_t pos0 = (valid && a.pos_base) ? a.pos_base[I.grp] : 0;  // global position of key row 0 here
       if (tid < nm * H) T.wperm[wperm_index(tid / H, tid % H)] = wv;
       named_bar_sync(2, C::NEPI);
       bool stop = false;
@@ -480,7 +483,7 @@ __global__ void __launch_bounds__(640, 1) refine_kernel(const __grid_constant__ 
           // Eq. (8) with the member's causal mask s <= t; key 0 marks "not eligible"
           if (mv && slot < a.c) {
             const int64_t t = I.t0 + r;
-            const bool valid = (sidx >= 0) && ((int64_t)sidx <= t);
+            const bool valid = (sidx >= 0) && ((int64_t)sidx + pos0 <= t);
             out_keys[(I.orow0 + r) * (int64_t)a.c + slot] = valid ? score_key(sc) : 0u;
           }
         }
