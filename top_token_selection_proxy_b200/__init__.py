@@ -327,8 +327,9 @@ def refine_host(q_host, w_host, k_host, topk: int, c: int, g: int, *, out_host, 
 
     q_host [L, H, d] bf16, w_host [L, H] fp32, k_host [L, d] bf16 and out_host [L, topk] int32
     are pinned CPU tensors.  The library copies the keys and weights, then the queries in
-    `chunks` runs of whole groups, indexes each run with the group-range call as soon as it
-    has landed and copies its rows back while later runs are still in flight.  The rows equal
+    `chunks` runs of whole groups (from the sequence's end to its start, heaviest first),
+    indexes each run with the group-range call as soon as it has landed and copies its rows
+    back while later runs are still in flight.  The rows equal
     those of one `refine` call.  Asynchronous: the stream is ordered after the last copy back,
     so synchronise it before reading out_host."""
     for t, dt_ in ((q_host, torch.bfloat16), (w_host, torch.float32), (k_host, torch.bfloat16),
