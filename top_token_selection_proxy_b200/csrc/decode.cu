@@ -413,7 +413,9 @@ __global__ void __launch_bounds__(576, 1) dscan_kernel(const __grid_constant__ C
 //            the bin where the count reaches the rest of n; the level-1 ties are split
 //            over the CTAs: above T2 selected, in T2 listed as level-2 ties;
 //   final    CTA 0 takes the best of the level-2 ties by the full (score, index) order
-//            and writes the candidate row (Refine) or the g member rows (Reuse).
+//            and writes the candidate row (Refine), the g member rows (Reuse), or, for
+//            one key shard of a prefix split over GPUs, the selection itself as packed
+//            entries with prefix positions (merged after the exchange, dmerge_kernel).
 // The list counters sit in CTA 0's shared memory (one remote atomic per warp and chunk).
 // Selected entries go straight into CTA 0's shared memory when n_sel fits its stage
 // (kSelStage entries), else to the workspace; the ties lists have room for every key
