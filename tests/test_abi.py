@@ -70,6 +70,51 @@ def test_invalid_arguments_rejected_before_launch(lib):
     assert lib.pivot_varlen_workspace_size(1, 2, off.ctypes.data_as(ctypes.c_void_p), 64, 128, 8, 8, 4, 0) == 0
 
 
+def test_decode_split_entry_points_validate_on_the_host(lib):
+    """The split decode's calls (one long prefix over GPUs) size their workspaces and reject bad
+    arguments before any device work."""
+    vp = ctypes.c_void_p
+    shard = np.array([0, 1, 5, 9], np.int64)  # a shard may hold a single key of a sequence
+    empty = np.array([0, 0, 4, 9], np.int64)  # ... but not none
+    sz = lambda op, off, H=64, d=128: lib.pivot_decode_shard_workspace_size(op, 3, off.ctypes.data_as(vp), H, d,
+                                                                            8, 16, 4)
+    assert sz(P.OP_REUSE, shard) > 0 and sz(P.OP_REFINE, shard) > 0
+    assert sz(P.OP_REFINE, empty) == 0
+    assert sz(P.OP_DENSE, shard) == 0                      # Reuse or Refine only
+    assert sz(P.OP_REFINE, shard, H=32) == 0              # tensor-core shape only
+    m = [lib.pivot_decode_merge_workspace_size(P.OP_REFINE, R, 3, 8, 16, 4) for R in (1, 2, 4)]
+    assert 0 < m[0] < m[1] < m[2]
+    assert lib.pivot_decode_merge_workspace_size(P.OP_REFINE, 0, 3, 8, 16, 4) == 0
+    assert lib.pivot_decode_merge_workspace_size(P.OP_REFINE, 2, 3, 8, 4, 4) == 0  # c < k
+    buf = ctypes.create_string_buffer(1 << 16)
+    ptr = ctypes.c_void_p((ctypes.addressof(buf) + 255) // 256 * 256)
+    plen = np.array([0, 9, 20, 40], np.int64)
+    short = np.array([0, 3, 20, 40], np.int64)  # P_0 = 3 < g = 4
+    pl, sh = plen.ctypes.data_as(vp), short.ctypes.data_as(vp)
+    # merge: null entries, a prefix shorter than g, Reuse without its output, workspace too small
+    assert lib.pivot_decode_merge(P.OP_REUSE, None, 2, ptr, pl, 3, 8, 8, 4, ptr, None, None, None, None, None,
+                                  None, ptr, 1 << 15, None) == 1
+    assert lib.pivot_decode_merge(P.OP_REUSE, ptr, 2, ptr, sh, 3, 8, 8, 4, ptr, None, None, None, None, None,
+                                  None, ptr, 1 << 15, None) == 1
+    assert lib.pivot_decode_merge(P.OP_REUSE, ptr, 2, ptr, pl, 3, 8, 8, 4, None, None, None, None, None, None,
+                                  None, ptr, 1 << 15, None) == 1
+    assert lib.pivot_decode_merge(P.OP_REFINE, ptr, 2, ptr, pl, 3, 8, 16, 4, None, None, ptr, None, None, None,
+                                  ptr, ptr, 1 << 15, None) == 1  # a local C needs this rank's shard
+    assert lib.pivot_decode_merge(P.OP_REFINE, ptr, 2, ptr, pl, 3, 8, 16, 4, None, None, ptr, None, None, None,
+                                  None, ptr, 256, None) == 3
+    sp = shard.ctypes.data_as(vp)
+    # shard select: dense is not a decode op; fp32 has no tensor-core path; null entries
+    assert lib.pivot_decode_shard_select(P.OP_DENSE, ptr, ptr, ptr, ptr, sp, ptr, 3, 64, 128, P.BF16, 8, 16, 4,
+                                         ptr, ptr, 1 << 15, None) == 1
+    assert lib.pivot_decode_shard_select(P.OP_REFINE, ptr, ptr, ptr, ptr, sp, ptr, 3, 64, 128, P.F32, 8, 16, 4,
+                                         ptr, ptr, 1 << 15, None) == 2
+    assert lib.pivot_decode_shard_select(P.OP_REFINE, ptr, ptr, ptr, ptr, sp, ptr, 3, 64, 128, P.BF16, 8, 16, 4,
+                                         None, ptr, 1 << 15, None) == 1
+    assert lib.pivot_decode_shard_rescore(ptr, ptr, ptr, ptr, sp, ptr, ptr, 3, 64, 128, P.BF16, 8, 16, 4, None,
+                                          ptr, ptr, 1 << 15, None) == 1
+    assert lib.pivot_decode_rowselect(ptr, ptr, ptr, 3, 8, 4, 4, ptr, None, None) == 1  # c < k
+
+
 def test_workspace_too_small_rejected(lib):
     buf = ctypes.create_string_buffer(4096)
     ptr = ctypes.c_void_p((ctypes.addressof(buf) + 15) // 16 * 16)
