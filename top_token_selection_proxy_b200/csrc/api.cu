@@ -644,6 +644,7 @@ pivot_status pivot_decode_shard_select(int op, const void* q, const float* w, co
   if (!q || !w || !k_shard || !shard_offsets_dev || !pos_base_dev || !entries || !ws) return PIVOT_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_shard) || !aligned16(ws)) return PIVOT_ERR_INVALID_ARG;
   if (!tc_shape(H, d, dt)) return PIVOT_ERR_UNSUPPORTED_SHAPE;
+  if ((int64_t)B * kSelCl > 0x7FFFFFFFLL) return PIVOT_ERR_UNSUPPORTED_SHAPE;  // selection grid
   const DecodeWs need = carve_decode(nullptr, op, B, shard_offsets_host, H, d, k, c, g, dt, false);
   if (ws_bytes < need.bytes) return PIVOT_ERR_WORKSPACE_TOO_SMALL;
   const DecodeWs W = carve_decode(ws, op, B, shard_offsets_host, H, d, k, c, g, dt, false);
