@@ -259,7 +259,14 @@ PIVOT_API pivot_status pivot_refine_varlen(const void *q, const float *w, const 
  * The results equal pivot_reuse_varlen / pivot_refine_varlen on the whole prefix.
  * Tensor-core shape only (bf16, H = 64, d in {64, 128}), else
  * PIVOT_ERR_UNSUPPORTED_SHAPE.  All pointers are device pointers except the
- * *_host offsets; all calls are asynchronous on `stream`. */
+ * *_host offsets; all calls are asynchronous on `stream`; the caller owns every
+ * buffer.  Errors (returned before any device work): PIVOT_ERR_INVALID_ARG
+ * (an op other than Reuse / Refine, null pointers, a shard without a key, a
+ * prefix shorter than g, c < k, a local C without this rank's shard, a
+ * misaligned q / k_shard / ws), PIVOT_ERR_UNSUPPORTED_SHAPE,
+ * PIVOT_ERR_WORKSPACE_TOO_SMALL, PIVOT_ERR_CUDA (pivot_last_cuda_error says
+ * which call).  Steps 1 and 4 use the library-wide bounded device waits
+ * (pivot_last_device_status on their workspace reports a timeout). */
 
 /* Step 1.  ws: pivot_decode_shard_workspace_size bytes (0: unsupported shape or
  * offsets).  op is PIVOT_OP_REUSE (c ignored) or PIVOT_OP_REFINE. */
