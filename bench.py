@@ -42,7 +42,7 @@ E2E_CHUNKS = 8  # runs of groups the end-to-end call pipelines its copies over
 SCAN_TRAFFIC = {
     "bytes": 2500000000 + 949310000,  # 2.50 GB + 949.31 MB, as ncu printed them
     "sources": ("scan.cu", "select.cuh", "ptx.cuh", "kernels.cuh", "headsum.cuh"),
-    "sources_sha256": "01067b0f47c43dbd8642eb4c13f6d200454e8682689443f487d82ec41c4fb143",
+    "sources_sha256": "09345fcff2aee30e9689cf7e53448ce1ce41b74bdae9b8721d517af192714fca",
     "profile": "profiles/kernels_prefill_L131072_g8_refine_1pass.md",
 }
 
