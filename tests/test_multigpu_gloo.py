@@ -297,3 +297,37 @@ def test_decode_shards_partition_every_prefix():
     ks, so, pb = M.shard_of(k, off, 2, 1)
     assert so.tolist() == [0, 4, 10] and pb.tolist() == [4, 6]
     assert np.array_equal(ks, np.concatenate([k[4:8], k[14:20]]))
+
+
+def test_decode_split_step_single_rank_passes_through():
+    """With one rank the exchanges are a leading axis of 1 and the identity, and the step runs
+    select -> merge (Reuse), or select -> merge -> rescore -> row select (Refine), in that order."""
+    calls = []
+
+    def select_fn():
+        calls.append("select")
+        return torch.arange(6).reshape(2, 3), torch.zeros(2, 3)
+
+    def merge_fn(g_):
+        calls.append("merge")
+        assert g_[0].shape == (1, 2, 3) and g_[1].shape == (1, 2, 3)
+        return "C", "C_local", None
+
+    def rescore_fn(merged):
+        calls.append("rescore")
+        assert merged[1] == "C_local"
+        return torch.ones(4, 5, dtype=torch.int32)
+
+    def rowselect_fn(keys, merged):
+        calls.append("rowselect")
+        assert torch.equal(keys, torch.ones(4, 5, dtype=torch.int32)) and merged[0] == "C"
+        return "rows"
+
+    assert M.decode_split_step(select_fn, merge_fn, 1) == ("C", "C_local", None)
+    assert calls == ["select", "merge"]
+    calls.clear()
+    assert M.decode_split_step(select_fn, merge_fn, 1, rescore_fn, rowselect_fn) == "rows"
+    assert calls == ["select", "merge", "rescore", "rowselect"]
+    k = torch.arange(20 * 2).reshape(20, 2)
+    ks, so, pb = M.shard_of(k, [0, 8, 20], 2, 0)
+    assert torch.equal(ks, torch.cat([k[0:4], k[8:14]])) and so.tolist() == [0, 4, 10] and pb.tolist() == [0, 0]
