@@ -453,9 +453,30 @@ def refine_varlen(q, w, k_cache, offsets, topk: int, c: int, g: int, *, scores: 
 # score keys) belong to the caller: multigpu.decode_split_step runs them over torch.distributed.
 
 
+class DeviceOffsets:
+    """int64 offsets (or per-sequence positions) kept on the host and on one device, so that repeated
+    calls pass them without copying; any of the decode split calls accepts one where it takes offsets
+    or positions."""
+
+    def __init__(self, values, device):
+        self.host = torch.as_tensor(values, dtype=torch.int64).cpu().contiguous()
+        self.dev = self.host.to(device)
+
+
 def _offsets_pair(offsets, device, stream):
+    if isinstance(offsets, DeviceOffsets):
+        return offsets.host, offsets.dev
     h = torch.as_tensor(offsets, dtype=torch.int64).cpu().contiguous()
     return h, _offsets_dev(h, device, stream)
+
+
+def _positions_dev(values, device, stream):
+    """Per-sequence int64 values on the device (copied from pinned memory without blocking)."""
+    if isinstance(values, DeviceOffsets):
+        return values.dev
+    if isinstance(values, torch.Tensor) and values.is_cuda:
+        return values
+    return _offsets_pair(values, device, stream)[1]
 
 
 def decode_shard_select(op: int, q, w, k_shard, shard_offsets, pos_base, topk: int, c: int, g: int, *,
@@ -464,7 +485,7 @@ def decode_shard_select(op: int, q, w, k_shard, shard_offsets, pos_base, topk: i
     OP_REUSE, c for OP_REFINE) as packed int64 entries [B, n] with prefix positions (0 pads)."""
     _need_cuda(q, w, k_shard)
     sh, sd = _offsets_pair(shard_offsets, q.device, stream)
-    pb = torch.as_tensor(pos_base, dtype=torch.int64).to(q.device)
+    pb = _positions_dev(pos_base, q.device, stream)
     B = sh.numel() - 1
     H, d = q.shape[1], q.shape[2]
     n = topk + g - 1 if op == OP_REUSE else c
@@ -489,7 +510,7 @@ def decode_merge(op: int, entries, plen_offsets, topk: int, c: int, g: int, *, s
     dev = entries.device
     local = shard_offsets is not None
     sd = _offsets_pair(shard_offsets, dev, stream)[1] if local else None
-    pb = torch.as_tensor(pos_base, dtype=torch.int64).to(dev) if local else None
+    pb = _positions_dev(pos_base, dev, stream) if local else None
     nbytes = int(lib().pivot_decode_merge_workspace_size(op, R, B, topk, c, g))
     W = _ws_for(ws, dev).get(nbytes)
     idx = sc = cand = csc = cl = None
@@ -513,7 +534,7 @@ def decode_shard_rescore(q, w, k_shard, shard_offsets, pos_base, plen_offsets, c
     _need_cuda(q, w, k_shard, cand_local)
     sh, sd = _offsets_pair(shard_offsets, q.device, stream)
     pd = _offsets_pair(plen_offsets, q.device, stream)[1]
-    pb = torch.as_tensor(pos_base, dtype=torch.int64).to(q.device)
+    pb = _positions_dev(pos_base, q.device, stream)
     B = sh.numel() - 1
     H, d = q.shape[1], q.shape[2]
     keys = torch.empty((B * g, c), dtype=torch.int32, device=q.device)
@@ -582,7 +603,7 @@ __all__ = [
     "guardrail_dense", "reuse_guarded", "refine_guarded", "AGGREGATION",
     "indexer_dense_range", "reuse_range", "refine_range",
     "group_chunks", "refine_host", "refine_streamed",
-    "decode_shard_select", "decode_merge", "decode_shard_rescore", "decode_rowselect",
+    "decode_shard_select", "decode_merge", "decode_shard_rescore", "decode_rowselect", "DeviceOffsets",
     "set_device_timeout_ns", "set_debug_flags", "KernelTimer", "OP_DENSE", "OP_REUSE", "OP_REFINE", "BF16", "F32",
     "STATUS",
 ]

@@ -205,8 +205,13 @@ def device_split_fns(op: int, q, w, k_shard, shard_off, pos_base, plen_off, topk
                      scores: bool = False):
     """The four steps on this rank's GPU through the library (the C ABI's pivot_decode_* calls).
     Reuse's merge returns (indices, scores|None); Refine's returns (C, C scores|None, C in this
-    rank's shard rows) and its row select (indices, scores|None)."""
+    rank's shard rows) and its row select (indices, scores|None).  The offsets and shard positions
+    go to the device once, here."""
     import top_token_selection_proxy_b200 as P
+
+    shard_off = P.DeviceOffsets(shard_off, q.device)
+    pos_base = P.DeviceOffsets(pos_base, q.device)
+    plen_off = P.DeviceOffsets(plen_off, q.device)
 
     def select_fn():
         return P.decode_shard_select(op, q, w, k_shard, shard_off, pos_base, topk, c, g)
