@@ -338,8 +338,9 @@ def per_config_lines(to_dev_fn, dev, ws, flush, timed, tf_burst, hbm, cpu):
     dq, dw, dk = to_dev_fn(xd["q"], dev), to_dev_fn(xd["w"], dev), to_dev_fn(xd["k"], dev)
     off = xd["offsets"]
     key_bytes = int(off[-1]) * ds.d * 2
-    d_ms = {"refine": timed(lambda: P.refine_varlen(dq, dw, dk, off, ds.k, ds.c, ds.g, ws=ws)),
-            "reuse": timed(lambda: P.reuse_varlen(dq, dw, dk, off, ds.k, ds.g, ws=ws))}
+    offd = P.DeviceOffsets(off, dev)  # the batch's offsets stay on the device, like its keys
+    d_ms = {"refine": timed(lambda: P.refine_varlen(dq, dw, dk, offd, ds.k, ds.c, ds.g, ws=ws)),
+            "reuse": timed(lambda: P.reuse_varlen(dq, dw, dk, offd, ds.k, ds.g, ws=ws))}
     rows = ds.B * ds.g
     e = {"workload": ds.name, "B": ds.B, "g": ds.g, "k": ds.k, "c": ds.c, "key_bytes": key_bytes,
          **{n: {"ms": t, "queries_per_s": rows / (t * 1e-3), "us_per_group": 1000.0 * t / ds.B,
@@ -652,8 +653,9 @@ def main():
         xd = inputs.make_decode(ds)
         dq, dw, dk = to_dev(xd["q"], dev), to_dev(xd["w"], dev), to_dev(xd["k"], dev)
         off = xd["offsets"]
-        dref = timed(lambda: P.refine_varlen(dq, dw, dk, off, ds.k, ds.c, ds.g, ws=ws))
-        dreu = timed(lambda: P.reuse_varlen(dq, dw, dk, off, ds.k, ds.g, ws=ws))
+        offd = P.DeviceOffsets(off, dev)  # the batch's offsets stay on the device, like its keys
+        dref = timed(lambda: P.refine_varlen(dq, dw, dk, offd, ds.k, ds.c, ds.g, ws=ws))
+        dreu = timed(lambda: P.reuse_varlen(dq, dw, dk, offd, ds.k, ds.g, ws=ws))
 
         def decode_phases(f, n=3):
             """Median (proxies + scan, selection + emit, re-scoring + row select) of n calls."""
@@ -667,7 +669,7 @@ def main():
             return {name: statistics.median(x[i] for x in ph)
                     for i, name in enumerate(("scan", "select_emit", "refine_rowselect"))}
 
-        dph = decode_phases(lambda: P.refine_varlen(dq, dw, dk, off, ds.k, ds.c, ds.g, ws=ws))
+        dph = decode_phases(lambda: P.refine_varlen(dq, dw, dk, offd, ds.k, ds.c, ds.g, ws=ws))
         key_bytes = int(off[-1]) * ds.d * 2
         hbm, _, _, _ = peaks()
         extras["decode"] = {"workload": ds.name, "refine_ms": dref, "reuse_ms": dreu, "refine_kernels_ms": dph,

@@ -400,7 +400,7 @@ def refine_guarded(q, w, k, topk: int, c: int, g: int, *, scores: bool = False, 
 
 def _varlen_common(q, w, kc, offsets, g):
     _need_cuda(q, w, kc)
-    off_h = torch.as_tensor(offsets, dtype=torch.int64).cpu().contiguous()
+    off_h = offsets.host if isinstance(offsets, DeviceOffsets) else torch.as_tensor(offsets, dtype=torch.int64).cpu().contiguous()
     B = off_h.numel() - 1
     if q.dim() != 3 or q.shape[0] != B * g or w.shape != (B * g, q.shape[1]) or kc.shape[1] != q.shape[2]:
         raise ValueError("expected q [B*g,H,d], w [B*g,H], k_cache [sum P, d]")
@@ -419,7 +419,7 @@ def reuse_varlen(q, w, k_cache, offsets, topk: int, g: int, *, scores: bool = Fa
                  ws: Optional[Workspace] = None, stream=None):
     """Eq. (3)-(6) for a batch of MTP decode groups.  Returns (indices [B*g,topk], scores|None)."""
     B, H, d, dt, off_h = _varlen_common(q, w, k_cache, offsets, g)
-    off_d = _offsets_dev(off_h, q.device, stream)
+    off_d = offsets.dev if isinstance(offsets, DeviceOffsets) else _offsets_dev(off_h, q.device, stream)
     idx = torch.empty((B * g, topk), dtype=torch.int32, device=q.device)
     sc = torch.empty((B * g, topk), dtype=torch.float32, device=q.device) if scores else None
     nbytes = varlen_workspace_size(OP_REUSE, off_h, H, d, topk, topk, g, dt)
@@ -434,7 +434,7 @@ def refine_varlen(q, w, k_cache, offsets, topk: int, c: int, g: int, *, scores: 
                   ws: Optional[Workspace] = None, stream=None):
     """Eq. (3)-(5),(7)-(9) for a batch of MTP decode groups."""
     B, H, d, dt, off_h = _varlen_common(q, w, k_cache, offsets, g)
-    off_d = _offsets_dev(off_h, q.device, stream)
+    off_d = offsets.dev if isinstance(offsets, DeviceOffsets) else _offsets_dev(off_h, q.device, stream)
     idx = torch.empty((B * g, topk), dtype=torch.int32, device=q.device)
     sc = torch.empty((B * g, topk), dtype=torch.float32, device=q.device) if scores else None
     cd = torch.empty((B, c), dtype=torch.int32, device=q.device) if cand else None
