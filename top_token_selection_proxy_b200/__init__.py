@@ -419,7 +419,8 @@ def reuse_varlen(q, w, k_cache, offsets, topk: int, g: int, *, scores: bool = Fa
                  ws: Optional[Workspace] = None, stream=None):
     """Eq. (3)-(6) for a batch of MTP decode groups.  Returns (indices [B*g,topk], scores|None)."""
     B, H, d, dt, off_h = _varlen_common(q, w, k_cache, offsets, g)
-    off_d = offsets.dev if isinstance(offsets, DeviceOffsets) else _offsets_dev(off_h, q.device, stream)
+    off_d = _offsets_pair(offsets, q.device, stream)[1] if isinstance(offsets, DeviceOffsets) else \
+        _offsets_dev(off_h, q.device, stream)
     idx = torch.empty((B * g, topk), dtype=torch.int32, device=q.device)
     sc = torch.empty((B * g, topk), dtype=torch.float32, device=q.device) if scores else None
     nbytes = varlen_workspace_size(OP_REUSE, off_h, H, d, topk, topk, g, dt)
@@ -434,7 +435,8 @@ def refine_varlen(q, w, k_cache, offsets, topk: int, c: int, g: int, *, scores: 
                   ws: Optional[Workspace] = None, stream=None):
     """Eq. (3)-(5),(7)-(9) for a batch of MTP decode groups."""
     B, H, d, dt, off_h = _varlen_common(q, w, k_cache, offsets, g)
-    off_d = offsets.dev if isinstance(offsets, DeviceOffsets) else _offsets_dev(off_h, q.device, stream)
+    off_d = _offsets_pair(offsets, q.device, stream)[1] if isinstance(offsets, DeviceOffsets) else \
+        _offsets_dev(off_h, q.device, stream)
     idx = torch.empty((B * g, topk), dtype=torch.int32, device=q.device)
     sc = torch.empty((B * g, topk), dtype=torch.float32, device=q.device) if scores else None
     cd = torch.empty((B, c), dtype=torch.int32, device=q.device) if cand else None
@@ -465,6 +467,8 @@ class DeviceOffsets:
 
 def _offsets_pair(offsets, device, stream):
     if isinstance(offsets, DeviceOffsets):
+        if offsets.dev.device != torch.device(device):
+            raise ValueError(f"offsets live on {offsets.dev.device}, the call runs on {device}")
         return offsets.host, offsets.dev
     h = torch.as_tensor(offsets, dtype=torch.int64).cpu().contiguous()
     return h, _offsets_dev(h, device, stream)
@@ -472,10 +476,11 @@ def _offsets_pair(offsets, device, stream):
 
 def _positions_dev(values, device, stream):
     """Per-sequence int64 values on the device (copied from pinned memory without blocking)."""
-    if isinstance(values, DeviceOffsets):
-        return values.dev
-    if isinstance(values, torch.Tensor) and values.is_cuda:
-        return values
+    if isinstance(values, DeviceOffsets) or (isinstance(values, torch.Tensor) and values.is_cuda):
+        d = values.dev if isinstance(values, DeviceOffsets) else values
+        if d.device != torch.device(device):
+            raise ValueError(f"positions live on {d.device}, the call runs on {device}")
+        return d
     return _offsets_pair(values, device, stream)[1]
 
 
